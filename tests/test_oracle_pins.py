@@ -1,0 +1,246 @@
+"""Pins for the fp64 oracle, checked against what the pages and the mathematics fix.
+
+Each test uses code independent of the oracle's recurrence: a dense
+brute-force semiseparable matrix, textbook special cases, closed forms, the
+pages' chunked algorithm (numpy restatement) and hand-worked values.
+Source: "Transformers are SSMs" (wikillm.com card, Method steps 1-8).
+"""
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+
+import oracle
+from oracle.chunked import ssd_chunked
+
+HERE = os.path.dirname(os.path.abspath(__file__))
+
+
+def rand_problem(rng, T, H, P, N, G, nseq=1):
+    x = rng.standard_normal((T, H, P))
+    dt = rng.uniform(0.01, 0.6, (T, H))
+    A = -rng.uniform(0.5, 3.0, H)
+    B = rng.standard_normal((T, G, N)) / math.sqrt(N)
+    C = rng.standard_normal((T, G, N)) / math.sqrt(N)
+    D = rng.standard_normal(H)
+    return x, dt, A, B, C, D
+
+
+def rel(a, b):
+    return np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-300)
+
+
+# ---------------------------------------------------------------- brute force
+def dense_M(dt, A, B, C, h, g):
+    """Dense lower-triangular M for one head (Method steps 1-2: M = L o (C B^T),
+    L[j, i] = prod_{r=i+1..j} a_r), with the dt input scaling folded into column i.
+    The decay product is formed by repeated multiplication, not by cumsum/exp differences."""
+    T = dt.shape[0]
+    a = np.exp(dt[:, h] * A[h])
+    M = np.zeros((T, T))
+    for j in range(T):
+        prod = 1.0
+        for i in range(j, -1, -1):
+            M[j, i] = (C[j, g] @ B[i, g]) * prod * dt[i, h]
+            prod *= a[i]
+    return M
+
+
+@pytest.mark.parametrize("T,H,P,N,G", [(1, 1, 1, 1, 1), (17, 2, 3, 5, 1), (48, 4, 3, 4, 2), (64, 2, 5, 3, 2)])
+def test_dense_semiseparable_matrix(T, H, P, N, G):
+    rng = np.random.default_rng(T * 100 + H)
+    x, dt, A, B, C, D = rand_problem(rng, T, H, P, N, G)
+    y, fin = oracle.ssd_forward(x, dt, A, B, C, D)
+    for h in range(H):
+        g = h // (H // G)
+        M = dense_M(dt, A, B, C, h, g)
+        y_ref = M @ x[:, h, :] + D[h] * x[:, h, :]
+        assert rel(y[:, h, :], y_ref) < 1e-12
+        # final state = sum_i (prod_{r>i} a_r) dt_i x_i B_i^T
+        a = np.exp(dt[:, h] * A[h])
+        S = np.zeros((P, N))
+        for i in range(T):
+            S += np.prod(a[i + 1:]) * dt[i, h] * np.outer(x[i, h], B[i, g])
+        assert rel(fin[0, h], S) < 1e-12
+
+
+# ------------------------------------------------------------ special cases
+def test_unit_decay_is_causal_linear_attention():
+    """a_t == 1 (A = 0): the layer is causal linear attention (Method step 3, sec. 5.2)."""
+    rng = np.random.default_rng(1)
+    T, H, P, N, G = 40, 3, 4, 6, 1
+    x, dt, A, B, C, D = rand_problem(rng, T, H, P, N, G)
+    A = np.zeros(H)
+    y, _ = oracle.ssd_forward(x, dt, A, B, C, D)
+    K = B[:, 0, :]  # keys
+    Qm = C[:, 0, :]  # queries
+    scores = np.tril(Qm @ K.T)  # causal, unnormalised
+    for h in range(H):
+        V = dt[:, h:h + 1] * x[:, h, :]
+        assert rel(y[:, h, :], scores @ V + D[h] * x[:, h, :]) < 1e-12
+
+
+def test_zero_decay_is_diagonal():
+    """a_t == 0: only the token's own term survives, y_t = (C_t . B_t) dt_t x_t + D x_t."""
+    rng = np.random.default_rng(2)
+    T, H, P, N, G = 25, 2, 3, 4, 1
+    x, _, _, B, C, D = rand_problem(rng, T, H, P, N, G)
+    dt = rng.uniform(0.5, 1.0, (T, H))
+    A = np.full(H, -2000.0)  # dt*A <= -1000: exp underflows to exactly 0 in fp64
+    assert np.all(np.exp(dt * A[None]) == 0.0)
+    y, fin = oracle.ssd_forward(x, dt, A, B, C, D)
+    cb = np.einsum("tn,tn->t", C[:, 0], B[:, 0])
+    y_ref = (cb * dt.T).T[:, :, None] * x + D[None, :, None] * x
+    assert rel(y, y_ref) < 1e-13
+    for h in range(H):
+        assert rel(fin[0, h], dt[-1, h] * np.outer(x[-1, h], B[-1, 0])) < 1e-13
+
+
+def test_skip_only_when_B_is_zero():
+    rng = np.random.default_rng(3)
+    x, dt, A, B, C, D = rand_problem(rng, 20, 2, 3, 4, 1)
+    y, fin = oracle.ssd_forward(x, dt, A, np.zeros_like(B), C, D)
+    assert np.array_equal(y, D[None, :, None] * x)
+    assert not fin.any()
+
+
+def test_free_response_closed_form():
+    """x = 0 with initial state h0: y_t = exp(sum_{r<=t} dt_r A) (h0 C_t)."""
+    rng = np.random.default_rng(4)
+    T, H, P, N = 30, 2, 3, 5
+    _, dt, A, B, C, D = rand_problem(rng, T, H, P, N, 1)
+    h0 = rng.standard_normal((1, H, P, N))
+    y, fin = oracle.ssd_forward(np.zeros((T, H, P)), dt, A, B, C, D, h0)
+    for h in range(H):
+        dec = np.exp(np.cumsum(dt[:, h] * A[h]))
+        y_ref = dec[:, None] * (C[:, 0] @ h0[0, h].T)
+        assert rel(y[:, h], y_ref) < 1e-12
+        assert rel(fin[0, h], dec[-1] * h0[0, h]) < 1e-12
+
+
+def test_group_mapping_contiguous_heads():
+    """Heads h share group h // (H/G): zeroing group 1's B silences heads 2 and 3 only."""
+    rng = np.random.default_rng(5)
+    T, H, P, N, G = 16, 4, 2, 3, 2
+    x, dt, A, B, C, D = rand_problem(rng, T, H, P, N, G)
+    B[:, 1] = 0.0
+    y, _ = oracle.ssd_forward(x, dt, A, B, C, D)
+    for h in (2, 3):
+        assert np.array_equal(y[:, h], D[h] * x[:, h])
+    for h in (0, 1):
+        assert np.abs(y[:, h] - D[h] * x[:, h]).max() > 1e-3
+
+
+@pytest.mark.parametrize("case", json.load(open(os.path.join(HERE, "golden", "handworked.json")))["cases"],
+                         ids=lambda c: c["name"])
+def test_handworked_golden(case):
+    T, H, P, N, G = case["T"], case["H"], case["P"], case["N"], case["G"]
+    x = np.asarray(case["x"], dtype=np.float64).reshape(T, H, P)
+    dt = np.asarray(case["dt"]).reshape(T, H)
+    B = np.asarray(case["B"]).reshape(T, G, N)
+    C = np.asarray(case["C"]).reshape(T, G, N)
+    y, fin = oracle.ssd_forward(x, dt, case["A"], B, C, case["D"])
+    np.testing.assert_allclose(y.reshape(-1), np.asarray(case["y"]).reshape(-1), rtol=0, atol=1e-12)
+    np.testing.assert_allclose(fin.reshape(-1), np.asarray(case["final"]).reshape(-1), rtol=0, atol=1e-12)
+
+
+# -------------------------------------------------- chunked algorithm (pages)
+@pytest.mark.parametrize("Q", [1, 4, 7, 16, 64, 100])
+def test_recurrence_equals_chunked_algorithm(Q):
+    """The chunked SSD (diag blocks + right/centre/left factors) equals the recurrence
+    for every chunk length, including a partial last chunk (Q = 7, 100)."""
+    rng = np.random.default_rng(6)
+    T, H, P, N, G = 96, 4, 3, 5, 2
+    x, dt, A, B, C, D = rand_problem(rng, T, H, P, N, G)
+    h0 = rng.standard_normal((1, H, P, N))
+    y, fin = oracle.ssd_forward(x, dt, A, B, C, D, h0)
+    gmap = np.arange(H) // (H // G)
+    Yc, Sc = ssd_chunked(dt[:, :, None] * x, dt * A[None], B[:, gmap], C[:, gmap], Q, h0[0])
+    Yc = Yc + D[None, :, None] * x
+    assert rel(y, Yc) < 1e-12
+    assert rel(fin[0], Sc) < 1e-12
+
+
+# ------------------------------------------------------- structural invariants
+def test_split_and_carry_equals_one_pass():
+    rng = np.random.default_rng(7)
+    T, H, P, N = 50, 2, 3, 4
+    x, dt, A, B, C, D = rand_problem(rng, T, H, P, N, 1)
+    y, fin = oracle.ssd_forward(x, dt, A, B, C, D)
+    t0 = 19
+    y1, f1 = oracle.ssd_forward(x[:t0], dt[:t0], A, B[:t0], C[:t0], D)
+    y2, f2 = oracle.ssd_forward(x[t0:], dt[t0:], A, B[t0:], C[t0:], D, f1)
+    assert rel(np.concatenate([y1, y2]), y) < 1e-12
+    assert rel(f2, fin) < 1e-12
+
+
+def test_linear_in_input_and_initial_state():
+    rng = np.random.default_rng(8)
+    T, H, P, N = 33, 2, 4, 3
+    x, dt, A, B, C, D = rand_problem(rng, T, H, P, N, 1)
+    h0 = rng.standard_normal((1, H, P, N))
+    y, f = oracle.ssd_forward(x, dt, A, B, C, D, h0)
+    ya, fa = oracle.ssd_forward(x, dt, A, B, C, D, None)
+    yb, fb = oracle.ssd_forward(np.zeros_like(x), dt, A, B, C, None, h0)
+    assert rel(y, ya + yb) < 1e-12
+    assert rel(f, fa + fb) < 1e-12
+
+
+def test_packed_equals_independent_sequences():
+    """Packed variable-length input: state resets at each boundary (zero-length sequence included)."""
+    rng = np.random.default_rng(9)
+    lens = [5, 0, 17, 1, 30]
+    offs = np.cumsum([0] + lens)
+    T, H, P, N, G = int(offs[-1]), 4, 3, 4, 2
+    x, dt, A, B, C, D = rand_problem(rng, T, H, P, N, G)
+    h0 = rng.standard_normal((len(lens), H, P, N))
+    y, fin = oracle.ssd_forward(x, dt, A, B, C, D, h0, offs)
+    for s, n in enumerate(lens):
+        a, b = offs[s], offs[s + 1]
+        ys, fs = oracle.ssd_forward(x[a:b], dt[a:b], A, B[a:b], C[a:b], D, h0[s:s + 1])
+        assert np.array_equal(y[a:b], ys)
+        assert np.array_equal(fin[s], fs[0])
+    assert np.array_equal(fin[1], h0[1])  # empty sequence: final = init
+
+
+def test_single_token_closed_form():
+    rng = np.random.default_rng(10)
+    x, dt, A, B, C, D = rand_problem(rng, 1, 2, 3, 4, 1)
+    h0 = rng.standard_normal((1, 2, 3, 4))
+    y, fin = oracle.ssd_forward(x, dt, A, B, C, D, h0)
+    for h in range(2):
+        S = math.exp(dt[0, h] * A[h]) * h0[0, h] + dt[0, h] * np.outer(x[0, h], B[0, 0])
+        assert rel(fin[0, h], S) < 1e-14
+        assert rel(y[0, h], S @ C[0, 0] + D[h] * x[0, h]) < 1e-14
+
+
+# ---------------------------------------------------------------- decode step
+def test_decode_steps_equal_dense_matrix():
+    """Repeated generation steps (Method step 8, sec. 6.3) reproduce the dense M x + D x."""
+    rng = np.random.default_rng(11)
+    T, H, P, N, G = 12, 4, 3, 5, 2
+    x, dt, A, B, C, D = rand_problem(rng, T, H, P, N, G)
+    state = np.zeros((1, H, P, N))
+    ys = []
+    for t in range(T):
+        yt, state = oracle.decode_step(x[t:t + 1], dt[t:t + 1], A, B[t:t + 1], C[t:t + 1], D, state)
+        ys.append(yt[0])
+    ys = np.stack(ys)
+    for h in range(H):
+        M = dense_M(dt, A, B, C, h, h // (H // G))
+        assert rel(ys[:, h], M @ x[:, h] + D[h] * x[:, h]) < 1e-12
+
+
+# ------------------------------------------------------- workload generator
+def test_sampled_problem_matches_full():
+    """The sampled-pairs harness returns exactly the full oracle's rows."""
+    import workloads
+    wl = workloads.custom(3, 40, H=4, P=4, N=8, G=2, chunk=16, dtype="bf16", init=True)
+    prob = workloads.generate(wl, seed=0)
+    y, f = oracle.ssd_forward_problem(prob)
+    ys, fs = oracle.ssd_forward_problem(prob, pairs=[(0, 1), (2, 3)])
+    assert np.array_equal(ys[0:40, 1], y[0:40, 1]) and np.array_equal(ys[80:120, 3], y[80:120, 3])
+    assert np.array_equal(fs[2, 3], f[2, 3])
+    assert np.isnan(ys[40:80]).all()
