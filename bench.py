@@ -1,0 +1,406 @@
+#!/usr/bin/env python
+"""Throughput of the chunked SSD forward pass on one or more B200s.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+A step is one ssd_forward call (every kernel of the path) over one batch of the
+Mamba-2-2.7B-like layer workload: batch 8 x 2048 tokens, 80 heads of dim 64,
+state 128, one B/C group, chunk 256, bf16 x/B/C with fp32 dt/A/D, synthetic
+seeded inputs resident in HBM.  With N > 1 (torchrun, one rank per GPU) every
+rank runs its own batch (weak scaling, no data-path collective); the time is
+the max over ranks.  Rank 0 prints one JSON line.
+
+``--impl reference`` times the fp64 CPU oracle instead (rank 0 only) on bounded
+samples of the same workload.
+"""
+from __future__ import annotations
+
+import argparse
+import datetime
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "SSD fwd tokens/s at Mamba-2-2.7B layer shape (1 B200); % of roofline"
+WORKLOAD = workloads.MAMBA2_2P7B
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+L2_FLUSH_BYTES = 256 << 20
+
+
+def log(*a):
+    print(*a, file=sys.stderr, flush=True)
+
+
+# ----------------------------------------------------------------- accounting
+def algorithmic_bytes(wl, init_present: bool, nseq: int) -> int:
+    """Compulsory I/O: read x, dt, B, C (and init when nonzero); write y and the fp32 final state."""
+    es = 2 if wl.dtype == "bf16" else 4
+    T, H, P, N, G = wl.tokens, wl.nheads, wl.headdim, wl.dstate, wl.ngroups
+    rd = T * H * P * es + T * H * 4 + 2 * T * G * N * es + 2 * H * 4
+    if init_present:
+        rd += nseq * H * P * N * 4
+    wr = T * H * P * es + nseq * H * P * N * 4
+    return rd + wr
+
+
+def algorithmic_flops(wl, seq_lengths) -> float:
+    """Causal block FLOPs of the chunked algorithm: per chunk of length q, q(q+1)N per group
+    for C B^T, q(q+1)P per head for the masked product, 4qNP per head for the chunk state
+    and the carried-state output."""
+    H, P, N, G, Q = wl.nheads, wl.headdim, wl.dstate, wl.ngroups, wl.chunk
+    tot = 0.0
+    for L in seq_lengths:
+        for t0 in range(0, L, Q):
+            q = min(Q, L - t0)
+            tot += G * q * (q + 1) * N + H * (q * (q + 1) * P + 4 * q * N * P)
+    return tot
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return pk, "measured"
+    except Exception:
+        return dict(FALLBACK_PEAKS), "fallback"
+
+
+def load_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on the current source."""
+    path = os.path.join(ROOT, "profiles", "traffic.json")
+    try:
+        with open(path) as f:
+            rec = json.load(f).get(kernel)
+    except Exception:
+        return None
+    if not rec:
+        return None
+    import hashlib
+
+    src = os.path.join(ROOT, rec["source"])
+    try:
+        sha = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except Exception:
+        return None
+    if sha != rec.get("source_sha"):
+        return None  # the kernel changed since the counters were taken
+    return rec.get("dram_bytes_per_launch")
+
+
+# --------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampling of SM clocks and throttle reasons around a timed region."""
+
+    FIELDS = ("timestamp,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu: str):
+        self.gpu = gpu
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(prefix="clocks_", suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu, f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+            return
+        t0 = time.time()
+        while time.time() - t0 < 5 and os.path.getsize(self.path) == 0:
+            time.sleep(0.05)
+        self.t_start = time.time()
+
+    def stop(self):
+        self.t_stop = time.time()
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.25)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        for line in open(self.path):
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                ts = datetime.datetime.strptime(parts[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+                rows.append((ts, float(parts[1]), float(parts[2]), parts[3], parts[4:]))
+            except ValueError:
+                continue
+        os.unlink(self.path)
+        inside = [r for r in rows if self.t_start - 0.1 <= r[0] <= self.t_stop + 0.1]
+        use = inside or rows
+        if not use:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in use for i, v in enumerate(r[4][1:5]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(r[1] for r in use), "sm_max_mhz": max(r[2] for r in use),
+                "reasons": reasons, "samples": len(use), "samples_in_window": len(inside)}
+
+
+def gpu_selector(local_rank: int) -> str:
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES")
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if local_rank < len(ids):
+            return ids[local_rank]
+    return str(local_rank)
+
+
+# ------------------------------------------------------------ CPU oracle timing
+def cpu_oracle_sample(prob, rows, heads, nthreads):
+    """Time the oracle on sequences ``rows`` x ``heads`` of ``prob``; returns (seconds, token-equivalents)."""
+    import oracle
+
+    pairs = [(s, h) for s in rows for h in heads]
+    t0 = time.perf_counter()
+    oracle.ssd_forward_problem(prob, pairs=pairs, nthreads=nthreads)
+    dt = time.perf_counter() - t0
+    toks = sum(prob.seq_offsets[s + 1] - prob.seq_offsets[s] for s in rows) * len(heads) / prob.wl.nheads
+    return dt, toks
+
+
+def cpu_baseline(prob, budget_s=10.0):
+    cores = len(os.sched_getaffinity(0))
+    H = prob.wl.nheads
+    spent, toks, rows = 0.0, 0.0, 0
+    while rows < prob.nseq and spent < budget_s:
+        dt, tk = cpu_oracle_sample(prob, [rows], list(range(H)), cores)
+        spent += dt
+        toks += tk
+        rows += 1
+    return {"value": toks / spent, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"first {rows} of {prob.nseq} sequences x all {H} heads ({int(toks)} tokens), "
+                      f"fp64 sequential recurrence, OpenMP over (sequence, head), {spent:.1f} s"}
+
+
+# ------------------------------------------------------------------ our arm
+def run_ours(args, rank, world, local_rank):
+    import ssd_sequence_mixing_b200 as ssd
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    wl = WORKLOAD
+    prob = workloads.generate(wl, seed=rank)
+    d = {k: (None if getattr(prob, k) is None else getattr(prob, k).to(dev))
+         for k in ("x", "dt", "A", "B", "C", "D", "init_state", "cu_seqlens")}
+    y = torch.empty_like(d["x"])
+    fin = torch.empty((prob.nseq, wl.nheads, wl.headdim, wl.dstate), dtype=torch.float32, device=dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    shape = ssd.make_shape(d["x"], d["B"], d["cu_seqlens"])
+    path = {ssd.PATH_SIMT: "simt", ssd.PATH_TC: "tc"}.get(ssd.select_path(shape, wl.chunk), "?")
+
+    def step():
+        ssd.ssd_forward(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["init_state"], d["cu_seqlens"], wl.chunk,
+                        y=y, final_state=fin, stream=stream)
+
+    for _ in range(args.warmup):
+        flush.zero_()
+        step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+
+    K = args.steps
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    dom = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    sampler = ClockSampler(gpu_selector(local_rank))
+    sampler.start()
+    launches0 = ssd.kernel_launch_count()
+    for k in range(K):
+        flush.zero_()  # evict L2 between timed steps (outside the events)
+        ssd.profile_dominant(*dom[k])
+        ev[k][0].record(stream)
+        step()
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    ssd.profile_dominant(None, None)
+    launches = ssd.kernel_launch_count() - launches0
+    clocks = sampler.stop()
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize()
+    assert ssd.query_status() == 0
+
+    step_ms = [a.elapsed_time(b) for a, b in ev]
+    dom_ms = [a.elapsed_time(b) for a, b in dom]
+    total_s = sum(step_ms) / 1e3
+    t = torch.tensor([total_s], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    max_total = float(t.item())
+    value = world * wl.tokens * K / max_total
+
+    # end to end through the host-buffer entry point: H2D inputs, compute, D2H outputs
+    pin = lambda v: None if v is None else v.pin_memory()
+    h = {k: pin(getattr(prob, k)) for k in ("x", "dt", "A", "B", "C", "D", "init_state", "cu_seqlens")}
+    yh = torch.empty(prob.x.shape, dtype=prob.x.dtype).pin_memory()
+    fh = torch.empty(fin.shape, dtype=torch.float32).pin_memory()
+    h2d = sum(v.numel() * v.element_size() for v in h.values() if v is not None)
+    d2h = yh.numel() * yh.element_size() + fh.numel() * fh.element_size()
+
+    def host_step():
+        ssd.ssd_forward_host(h["x"], h["dt"], h["A"], h["B"], h["C"], h["D"], h["init_state"], h["cu_seqlens"],
+                             wl.chunk, y=yh, final_state=fh, stream=stream)
+
+    host_step()
+    torch.cuda.synchronize()
+    if world > 1:
+        torch.distributed.barrier()
+    e2e_ms = []
+    for _ in range(args.e2e_steps):
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        host_step()
+        b.record(stream)
+        b.synchronize()
+        e2e_ms.append(a.elapsed_time(b))
+    te = torch.tensor([sum(e2e_ms) / 1e3], dtype=torch.float64, device=dev)
+    if world > 1:
+        torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
+    e2e_value = world * wl.tokens * args.e2e_steps / float(te.item())
+
+    if rank != 0:
+        return None
+
+    peaks, peak_kind = load_peaks()
+    nbytes = algorithmic_bytes(wl, prob.init_state is not None, prob.nseq)
+    lens = [prob.seq_offsets[i + 1] - prob.seq_offsets[i] for i in range(prob.nseq)]
+    flops = algorithmic_flops(wl, lens)
+    t_mem = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_flop = flops / (peaks["bf16_tflops"] * 1e12)
+    bound = "hbm" if t_mem >= t_flop else "tensor"
+    dom_s = statistics.mean(dom_ms) / 1e3
+    if bound == "hbm":
+        achieved, peak, unit = nbytes / dom_s / 1e9, peaks["hbm_gbs"], "GB/s"
+    else:
+        achieved, peak, unit = flops / dom_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    kernel = "ssd_fused_tc" if path == "tc" else "chunk_output_kernel"
+    roof_s = max(t_mem, t_flop)
+    step_s = max_total / K
+    out = {
+        "metric": METRIC,
+        "value": value,
+        "unit": "tokens/s",
+        "n_gpus": world,
+        "steps": K,
+        "warmup": args.warmup,
+        "ms_per_step": step_s * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16",
+        "data": "synthetic (seeded; Mamba-2 init distributions; inputs resident in HBM)",
+        "config": {"workload": wl.name, "batch": wl.batch, "seq_len": wl.seqlen, "nheads": wl.nheads,
+                   "headdim": wl.headdim, "dstate": wl.dstate, "ngroups": wl.ngroups, "chunk": wl.chunk,
+                   "io_dtype": "bf16 x/B/C/y, fp32 dt/A/D/states", "parallelism": f"dp{world} (independent batches)",
+                   "l2": "flushed between timed steps (256 MB write outside the events)", "path": path},
+        "roofline": {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+                     "traffic": load_traffic(kernel), "kernel": kernel, "peak_source": f"{peak_kind} ({unit})",
+                     "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
+                     "dominant_ms": statistics.mean(dom_ms),
+                     "step_roofline_us": roof_s * 1e6, "step_frac": roof_s / step_s},
+        "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "steps": args.e2e_steps, "ms_per_step": statistics.mean(e2e_ms),
+                "api": "ssd_forward_host (pinned host buffers)"},
+        "gpu_launches": int(launches),
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(prob, budget_s=args.cpu_budget)
+    return out
+
+
+# ------------------------------------------------------------ reference arm
+def run_reference(args):
+    """The fp64 CPU oracle on this workload: each step is a bounded sample (one sequence x
+    ``--ref-heads`` heads), reported in token-equivalents of the full workload per second."""
+    wl = WORKLOAD
+    prob = workloads.generate(wl, seed=0)
+    cores = len(os.sched_getaffinity(0))
+    H = wl.nheads
+    nh = min(args.ref_heads, H)
+    times, toks = [], []
+    for k in range(args.warmup + args.steps):
+        s = k % prob.nseq
+        heads = [(k * nh + i) % H for i in range(nh)]
+        dt, tk = cpu_oracle_sample(prob, [s], heads, cores)
+        if k >= args.warmup:
+            times.append(dt)
+            toks.append(tk)
+    value = sum(toks) / sum(times)
+    sample = f"per step 1 sequence x {nh} of {H} heads ({int(toks[0])} token-equivalents), fp64 recurrence"
+    return {
+        "metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": args.gpus, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": statistics.mean(times) * 1e3, "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": wl.name, "batch": wl.batch, "seq_len": wl.seqlen, "nheads": wl.nheads,
+                   "headdim": wl.headdim, "dstate": wl.dstate, "ngroups": wl.ngroups, "chunk": wl.chunk},
+        "impl": "reference",
+        "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+        "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--e2e-steps", type=int, default=3)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=10.0)
+    ap.add_argument("--ref-heads", type=int, default=16)
+    args = ap.parse_args()
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=180),
+                                             device_id=torch.device("cuda", local_rank))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            print(json.dumps(out), flush=True)
+    finally:
+        if world > 1:
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

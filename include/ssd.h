@@ -1,0 +1,151 @@
+/*
+ * ssd.h -- C ABI of the B200 (sm_100a) chunked SSD forward library, libssd.so.
+ *
+ * SSD ("structured state space duality") is the sequence-mixing core of the
+ * Mamba-2 layer ("Transformers are SSMs", Dao & Gu, ICML 2024).  For every
+ * sequence and head h (group g = h / (H/G)), with a P x N fp32 state S:
+ *
+ *     a_t = exp(dt_t * A_h)                          (scalar decay per head)
+ *     S_t = a_t * S_{t-1} + (dt_t * x_t) B_t^T       (x_t in R^P, B_t in R^N)
+ *     y_t = S_t C_t + D_h * x_t
+ *
+ * which equals multiplication by the 1-semiseparable-masked matrix
+ * M = L o (C B^T) (wikillm.com card, Method steps 1-3; sec. 2, 3, 5.1), computed
+ * by the chunked algorithm (Method step 5, sec. 6: diagonal blocks, right,
+ * centre and left factors) with chunk length `chunk`.  Discretisation follows
+ * the card's Method step 7 / "Paper vs code" item 7: dt scales the input and the
+ * decay; the D skip uses the unscaled x (item 3).
+ *
+ * Conventions for every entry point:
+ *  - All tensors are dense, row-major and contiguous.  Unless an entry point
+ *    says "host", every pointer is a DEVICE pointer of the current device and
+ *    must be 16-byte aligned.  The caller owns every buffer; the library keeps
+ *    no pointer after the call returns.
+ *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *    stream) unless stated otherwise.  Scratch memory, when needed, comes from
+ *    the stream-ordered allocator (cudaMallocAsync / cudaFreeAsync on `stream`).
+ *  - The return value is an ssd_status.  On any host-detected error nothing is
+ *    launched and no output is written.  Errors found on the device (bad
+ *    cu_seqlens values, a bounded wait that ran out) are recorded in a per-device
+ *    status word, read with ssd_query_status().
+ */
+#ifndef SSD_H_
+#define SSD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t / CUstream, declared here so this header needs no CUDA header. */
+typedef struct CUstream_st* ssd_stream_t;
+
+typedef enum { SSD_F32 = 0, SSD_BF16 = 1 } ssd_dtype;
+
+typedef enum {
+  SSD_OK = 0,
+  SSD_ERR_INVALID_ARG = 1,    /* null required pointer, negative size, bad dtype           */
+  SSD_ERR_UNSUPPORTED = 2,    /* chunk not in {64,128,256}, H % G != 0, P or N outside 1..256 */
+  SSD_ERR_MISALIGNED = 3,     /* a pointer is not 16-byte aligned                            */
+  SSD_ERR_CUDA = 4,           /* a CUDA runtime call or kernel launch failed                 */
+  SSD_ERR_DEVICE_TIMEOUT = 5, /* a bounded device-side wait gave up (kernel returned early)  */
+  SSD_ERR_BAD_SEQLENS = 6     /* cu_seqlens not 0 = c0 <= c1 <= ... <= c_nseq = seqlen        */
+} ssd_status;
+
+/*
+ * Problem shape.  Raw pointers carry no shapes, so every call takes one.
+ *   batch    dense batch rows (must be 1 when cu_seqlens is given)
+ *   seqlen   tokens per row; for a packed batch, the total number of tokens T
+ *   nheads   H;  headdim P;  dstate N;  ngroups G (H % G == 0, heads h*G/H share B, C)
+ *   nseq     number of packed sequences when cu_seqlens is given (ignored otherwise)
+ *   io_dtype dtype of x, B, C and y (dt, A, D and the states are always fp32)
+ *   cu_seqlens_host  optional HOST copy of cu_seqlens; when given it is validated on
+ *            the host (SSD_ERR_BAD_SEQLENS) before anything is launched.
+ */
+typedef struct {
+  int64_t batch, seqlen, nheads, headdim, dstate, ngroups, nseq;
+  ssd_dtype io_dtype;
+  const int32_t* cu_seqlens_host;
+} ssd_shape;
+
+/*
+ * ssd_forward -- the chunked SSD forward pass (wikillm.com card, Method step 5, sec. 6,
+ * Theorem 6.1; varlen per the GVA / variable-length note of the Chinese wiki page).
+ *
+ *   x           (batch, seqlen, H, P)  io_dtype   input
+ *   dt          (batch, seqlen, H)     fp32       step sizes, > 0 (already softplus'ed)
+ *   A           (H)                    fp32       decay rates, < 0 (A = -exp(A_log))
+ *   B, C        (batch, seqlen, G, N)  io_dtype   SSM input / output matrices
+ *   D           (H)                    fp32       skip weights, or NULL (= 0)
+ *   init_state  (nseq_or_batch, H, P, N) fp32     state before each sequence, or NULL (= 0)
+ *   cu_seqlens  (nseq + 1)             int32      packed-sequence offsets (device), or NULL
+ *                                                 for a dense batch; the state resets at each
+ *                                                 sequence start
+ *   chunk       Q in {64, 128, 256}: length of the chunks of the block decomposition
+ *   y           (batch, seqlen, H, P)  io_dtype   output (may not alias an input)
+ *   final_state (nseq_or_batch, H, P, N) fp32     state after each sequence, or NULL
+ * Returns SSD_OK or an error code (see ssd_status).  Asynchronous on `stream`.
+ */
+int ssd_forward(const ssd_shape* shape, const void* x, const float* dt, const float* A, const void* B,
+                const void* C, const float* D, const float* init_state, const int32_t* cu_seqlens, int chunk,
+                void* y, float* final_state, ssd_stream_t stream);
+
+/*
+ * ssd_forward_host -- the same computation on HOST buffers (pinned memory gives full
+ * copy bandwidth).  Device buffers are taken from the stream-ordered allocator, the
+ * inputs are copied in, ssd_forward runs, the outputs are copied back, and the call
+ * synchronises `stream` before returning.  Same layouts and errors as ssd_forward;
+ * cu_seqlens is a host pointer here.  Returns SSD_ERR_DEVICE_TIMEOUT or
+ * SSD_ERR_BAD_SEQLENS when the device reported one during this call.
+ */
+int ssd_forward_host(const ssd_shape* shape, const void* x, const float* dt, const float* A, const void* B,
+                     const void* C, const float* D, const float* init_state, const int32_t* cu_seqlens, int chunk,
+                     void* y, float* final_state, ssd_stream_t stream);
+
+/* Bytes of stream-ordered scratch ssd_forward takes for this shape (informational). */
+size_t ssd_workspace_bytes(const ssd_shape* shape, int chunk);
+
+/*
+ * Synchronises `stream`, then returns and clears the current device's status word:
+ * SSD_OK, SSD_ERR_BAD_SEQLENS or SSD_ERR_DEVICE_TIMEOUT (SSD_ERR_CUDA if the
+ * synchronisation itself failed).
+ */
+int ssd_query_status(ssd_stream_t stream);
+
+/* Static, human-readable text for a status code. */
+const char* ssd_status_string(int status);
+
+/*
+ * Kernel path selection, process-wide (not thread-safe; meant for tests and benches):
+ *   SSD_PATH_AUTO  the tensor-core (tcgen05) path where the shape supports it, else SIMT
+ *   SSD_PATH_SIMT  the general CUDA-core path for every shape and dtype
+ *   SSD_PATH_TC    the tensor-core path; shapes it cannot take return SSD_ERR_UNSUPPORTED
+ * Returns the previous setting.
+ */
+enum { SSD_PATH_AUTO = 0, SSD_PATH_SIMT = 1, SSD_PATH_TC = 2 };
+int ssd_set_path(int path);
+
+/* Which path ssd_forward would take for this shape and chunk under the current setting
+ * (SSD_PATH_SIMT or SSD_PATH_TC), or a negative ssd_status when it would fail. */
+int ssd_select_path(const ssd_shape* shape, int chunk);
+
+/* Same type as cudaEvent_t / CUevent. */
+typedef struct CUevent_st* ssd_event_t;
+
+/*
+ * Measurement hooks (process-wide, not thread-safe; meant for benches).
+ * ssd_profile_dominant: when both events are non-NULL, every later ssd_forward records
+ * `start` on its stream just before its dominant kernel (the one that moves the bulk
+ * of the bytes: the fused tensor-core kernel, or the SIMT output kernel) and `stop`
+ * just after it; NULL, NULL turns this off.  The events are the caller's.
+ * ssd_kernel_launch_count: kernels launched by this library so far in this process.
+ */
+int ssd_profile_dominant(ssd_event_t start, ssd_event_t stop);
+uint64_t ssd_kernel_launch_count(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* SSD_H_ */

@@ -1,0 +1,242 @@
+"""B200-native chunked SSD (Mamba-2 sequence mixing) forward pass.
+
+A thin ctypes binding over ``libssd.so`` (C ABI in ``include/ssd.h``).  This
+module only marshals arguments: shapes are read off torch tensors, outputs are
+allocated with torch when the caller does not pass them, and every step of the
+computation runs in the library's CUDA kernels.  There is no CPU fallback:
+without the built library, importing this package raises.
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+from typing import Optional, Tuple
+
+import torch
+
+_PKG = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_PKG, "libssd.so")
+
+SSD_F32, SSD_BF16 = 0, 1
+PATH_AUTO, PATH_SIMT, PATH_TC = 0, 1, 2
+STATUS = {
+    0: "SSD_OK",
+    1: "SSD_ERR_INVALID_ARG",
+    2: "SSD_ERR_UNSUPPORTED",
+    3: "SSD_ERR_MISALIGNED",
+    4: "SSD_ERR_CUDA",
+    5: "SSD_ERR_DEVICE_TIMEOUT",
+    6: "SSD_ERR_BAD_SEQLENS",
+}
+# Every entry point include/ssd.h declares.
+EXPORTS = (
+    "ssd_forward",
+    "ssd_forward_host",
+    "ssd_workspace_bytes",
+    "ssd_query_status",
+    "ssd_status_string",
+    "ssd_set_path",
+    "ssd_select_path",
+    "ssd_profile_dominant",
+    "ssd_kernel_launch_count",
+)
+
+
+class SsdShape(ctypes.Structure):
+    _fields_ = [
+        ("batch", ctypes.c_int64),
+        ("seqlen", ctypes.c_int64),
+        ("nheads", ctypes.c_int64),
+        ("headdim", ctypes.c_int64),
+        ("dstate", ctypes.c_int64),
+        ("ngroups", ctypes.c_int64),
+        ("nseq", ctypes.c_int64),
+        ("io_dtype", ctypes.c_int),
+        ("cu_seqlens_host", ctypes.c_void_p),
+    ]
+
+
+class SsdError(RuntimeError):
+    def __init__(self, code: int, where: str):
+        self.code = code
+        super().__init__(f"{where}: {STATUS.get(code, code)} ({_lib.ssd_status_string(code).decode()})")
+
+
+def _open() -> ctypes.CDLL:
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(f"{LIB_PATH} is not built; run `python ssd_sequence_mixing_b200/build.py`")
+    lib = ctypes.CDLL(LIB_PATH)
+    V, I, SP = ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(SsdShape)
+    fwd = [SP, V, V, V, V, V, V, V, V, I, V, V, V]
+    for name in ("ssd_forward", "ssd_forward_host"):
+        getattr(lib, name).argtypes = fwd
+        getattr(lib, name).restype = I
+    lib.ssd_workspace_bytes.argtypes = [SP, I]
+    lib.ssd_workspace_bytes.restype = ctypes.c_size_t
+    lib.ssd_query_status.argtypes = [V]
+    lib.ssd_query_status.restype = I
+    lib.ssd_status_string.argtypes = [I]
+    lib.ssd_status_string.restype = ctypes.c_char_p
+    lib.ssd_set_path.argtypes = [I]
+    lib.ssd_set_path.restype = I
+    lib.ssd_select_path.argtypes = [SP, I]
+    lib.ssd_select_path.restype = I
+    lib.ssd_profile_dominant.argtypes = [V, V]
+    lib.ssd_profile_dominant.restype = I
+    lib.ssd_kernel_launch_count.argtypes = []
+    lib.ssd_kernel_launch_count.restype = ctypes.c_uint64
+    return lib
+
+
+_lib = _open()
+
+
+def library() -> ctypes.CDLL:
+    return _lib
+
+
+def _ptr(t: Optional[torch.Tensor]):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _io_code(dtype: torch.dtype) -> int:
+    if dtype == torch.float32:
+        return SSD_F32
+    if dtype == torch.bfloat16:
+        return SSD_BF16
+    raise TypeError(f"x, B, C must be float32 or bfloat16, got {dtype}")
+
+
+def make_shape(x: torch.Tensor, B: torch.Tensor, cu_seqlens=None, cu_seqlens_host=None) -> SsdShape:
+    """ssd_shape from x (batch, T, H, P) and B (batch, T, G, N)."""
+    if x.dim() != 4 or B.dim() != 4:
+        raise ValueError("x must be (batch, seqlen, H, P) and B, C (batch, seqlen, G, N)")
+    batch, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    nseq = 0
+    if cu_seqlens is not None:
+        nseq = cu_seqlens.numel() - 1
+    s = SsdShape(batch, T, H, P, N, G, nseq, _io_code(x.dtype), None)
+    if cu_seqlens_host is not None:
+        s.cu_seqlens_host = ctypes.c_void_p(cu_seqlens_host.data_ptr())
+    return s
+
+
+def _check(name, t, device, dtype=None, shape=None):
+    if t is None:
+        return
+    if t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} has shape {tuple(t.shape)}, expected {tuple(shape)}")
+
+
+def _prepare(x, dt, A, B, C, D, init_state, cu_seqlens, y, final_state, return_final, device):
+    batch, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    rows = cu_seqlens.numel() - 1 if cu_seqlens is not None else batch
+    _check("x", x, device)
+    _check("dt", dt, device, torch.float32, (batch, T, H))
+    _check("A", A, device, torch.float32, (H,))
+    _check("B", B, device, x.dtype, (batch, T, G, N))
+    _check("C", C, device, x.dtype, (batch, T, G, N))
+    _check("D", D, device, torch.float32, (H,))
+    _check("init_state", init_state, device, torch.float32, (rows, H, P, N))
+    _check("cu_seqlens", cu_seqlens, device, torch.int32)
+    pin = device.type == "cpu" and x.is_pinned()
+    if y is None:
+        y = torch.empty(x.shape, dtype=x.dtype, device=device, pin_memory=pin)
+    _check("y", y, device, x.dtype, tuple(x.shape))
+    if final_state is None and return_final:
+        final_state = torch.empty((rows, H, P, N), dtype=torch.float32, device=device, pin_memory=pin)
+    _check("final_state", final_state, device, torch.float32, (rows, H, P, N))
+    return y, final_state
+
+
+def ssd_forward(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor, C: torch.Tensor,
+                D: Optional[torch.Tensor] = None, init_state: Optional[torch.Tensor] = None,
+                cu_seqlens: Optional[torch.Tensor] = None, chunk: int = 256, y: Optional[torch.Tensor] = None,
+                final_state: Optional[torch.Tensor] = None, return_final: bool = True, stream=None,
+                cu_seqlens_host: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, Optional[torch.Tensor]]:
+    """Chunked SSD forward on CUDA tensors (see ``ssd_forward`` in include/ssd.h).
+
+    x (batch, T, H, P) fp32/bf16; dt (batch, T, H) fp32; A (H,) fp32; B, C (batch, T, G, N);
+    D (H,) fp32 or None; init_state (rows, H, P, N) fp32 or None; cu_seqlens (nseq+1,) int32
+    (packed batch, batch == 1) or None.  Returns (y, final_state).  Asynchronous on ``stream``
+    (default: torch's current stream).
+    """
+    device = x.device
+    if device.type != "cuda":
+        raise ValueError("ssd_forward takes CUDA tensors; use ssd_forward_host for host buffers")
+    y, final_state = _prepare(x, dt, A, B, C, D, init_state, cu_seqlens, y, final_state, return_final, device)
+    shape = make_shape(x, B, cu_seqlens, cu_seqlens_host)
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    with torch.cuda.device(device):
+        rc = _lib.ssd_forward(ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                              _ptr(init_state), _ptr(cu_seqlens), int(chunk), _ptr(y), _ptr(final_state),
+                              ctypes.c_void_p(handle))
+    if rc:
+        raise SsdError(rc, "ssd_forward")
+    return y, final_state
+
+
+def ssd_forward_host(x, dt, A, B, C, D=None, init_state=None, cu_seqlens=None, chunk: int = 256, y=None,
+                     final_state=None, return_final: bool = True, stream=None):
+    """The same on host (CPU, ideally pinned) tensors: the library copies in, runs and copies out,
+    and returns after synchronising.  Runs on the current CUDA device."""
+    device = torch.device("cpu")
+    if x.device.type != "cpu":
+        raise ValueError("ssd_forward_host takes host tensors")
+    y, final_state = _prepare(x, dt, A, B, C, D, init_state, cu_seqlens, y, final_state, return_final, device)
+    shape = make_shape(x, B, cu_seqlens)
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    rc = _lib.ssd_forward_host(ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                               _ptr(init_state), _ptr(cu_seqlens), int(chunk), _ptr(y), _ptr(final_state),
+                               ctypes.c_void_p(handle))
+    if rc:
+        raise SsdError(rc, "ssd_forward_host")
+    return y, final_state
+
+
+def query_status(stream=None) -> int:
+    """Synchronise ``stream`` and return (and clear) the device status word as an ssd_status."""
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    return _lib.ssd_query_status(ctypes.c_void_p(handle))
+
+
+def set_path(path: int) -> int:
+    """Force the kernel path (PATH_AUTO, PATH_SIMT or PATH_TC); returns the previous one."""
+    rc = _lib.ssd_set_path(int(path))
+    if rc < 0:
+        raise SsdError(-rc, "ssd_set_path")
+    return rc
+
+
+def select_path(shape: SsdShape, chunk: int) -> int:
+    return _lib.ssd_select_path(ctypes.byref(shape), int(chunk))
+
+
+def workspace_bytes(shape: SsdShape, chunk: int) -> int:
+    return int(_lib.ssd_workspace_bytes(ctypes.byref(shape), int(chunk)))
+
+
+def profile_dominant(start=None, stop=None) -> None:
+    """Have later ssd_forward calls record torch.cuda.Event ``start``/``stop`` around their
+    dominant kernel (both None: off)."""
+    h = lambda e: None if e is None else ctypes.c_void_p(e.cuda_event)
+    _lib.ssd_profile_dominant(h(start), h(stop))
+
+
+def kernel_launch_count() -> int:
+    """Kernels launched by the library so far in this process."""
+    return int(_lib.ssd_kernel_launch_count())

@@ -1,0 +1,78 @@
+// ssd_common.cuh -- device-side problem description shared by the kernels of libssd.so.
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "ssd.h"
+
+namespace ssd {
+
+// Status bits OR-ed into the per-device status word by kernels.
+enum : unsigned int { kStatusBadSeqlens = 1u, kStatusTimeout = 2u };
+
+// One chunk of one sequence: tokens [t0, t0 + len) of sequence `seq`, the
+// `idx`-th chunk of that sequence.  Chunks never straddle a sequence boundary:
+// each sequence is cut into ceil(len / Q) chunks, the last one possibly partial.
+struct ChunkRec {
+  int32_t seq, t0, len, idx;
+};
+
+// Everything a launch needs, passed by value to every kernel.
+struct Problem {
+  int64_t tokens;  // total tokens over all sequences
+  int64_t seqlen;  // dense row length (dense batches)
+  int nseq, H, P, N, G, hpg, Q;
+  int bf16;  // io dtype: 1 = bf16, 0 = fp32
+  const void* x;
+  const float* dt;
+  const float* A;
+  const void* B;
+  const void* C;
+  const float* D;     // nullable
+  const float* init;  // nullable
+  const int32_t* cu;  // nullable (dense batch)
+  void* y;
+  float* final_state;  // nullable
+  unsigned int* status;
+  // scratch
+  ChunkRec* chunks;    // Cmax records
+  int32_t* nchunks;    // number of valid records, -1 when cu_seqlens was invalid
+  int32_t* seq_first;  // nseq + 1: first chunk of each sequence
+  float* cs;           // (Cmax, H, Q) in-chunk inclusive cumsum of dt * A
+  float* states;       // (Cmax, H, P, N) chunk states, then chunk start states
+  int Cmax;
+  // host-side measurement hooks (events around the dominant kernel, or null)
+  cudaEvent_t prof_start, prof_stop;
+};
+
+__device__ __forceinline__ int64_t seq_off(const Problem& pb, int s) {
+  return pb.cu ? (int64_t)pb.cu[s] : (int64_t)s * pb.seqlen;
+}
+
+__device__ __forceinline__ float to_f(float v) { return v; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+
+template <typename T>
+__device__ __forceinline__ T from_f(float v);
+template <>
+__device__ __forceinline__ float from_f<float>(float v) {
+  return v;
+}
+template <>
+__device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+// Upper bound on the number of chunks over all sequences: sum ceil(len_s/Q) <= ceil(T/Q) + nseq.
+inline int max_chunks(int64_t tokens, int nseq, int Q) { return (int)((tokens + Q - 1) / Q) + nseq; }
+
+// Adds n to the process-wide count of kernels launched by the library.
+void count_launches(int n);
+
+// Launchers implemented in the kernel files.
+cudaError_t launch_chunk_table(const Problem& pb, cudaStream_t st);
+cudaError_t launch_simt(const Problem& pb, cudaStream_t st);
+
+}  // namespace ssd

@@ -1,0 +1,151 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the same
+seeded inputs, at sizes the oracle finishes in seconds (several chunks and a ragged
+tail) and at the five full-size workloads on sampled (sequence, head) pairs."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import ssd_sequence_mixing_b200 as ssd
+import workloads
+from harness import assert_close, check, run, sample_pairs, to_device
+
+pytestmark = pytest.mark.gpu
+
+PATHS = {"simt": ssd.PATH_SIMT, "auto": ssd.PATH_AUTO}
+
+
+def tc_available(prob, chunk):
+    s = ssd.make_shape(prob.x, prob.B, prob.cu_seqlens)
+    old = ssd.set_path(ssd.PATH_TC)
+    try:
+        return ssd.select_path(s, chunk) == ssd.PATH_TC
+    finally:
+        ssd.set_path(old)
+
+
+def paths_for(prob, chunk):
+    out = [("simt", ssd.PATH_SIMT)]
+    if tc_available(prob, chunk):
+        out.append(("tc", ssd.PATH_TC))
+    return out
+
+
+# ------------------------------------------------------------------ small cases
+def test_tiny_fp32_workload():
+    prob = workloads.generate(workloads.TINY, seed=0)
+    for name, path in paths_for(prob, 64):
+        y, fin = run(prob, path=path)
+        check(prob, y, fin)
+
+
+SMALL = [
+    # batch, T, H, P, N, G, chunk, dtype, init
+    (2, 700, 4, 64, 128, 2, 256, "bf16", True),
+    (1, 513, 3, 64, 64, 1, 128, "bf16", False),
+    (3, 130, 2, 64, 128, 1, 64, "bf16", True),
+    (2, 300, 4, 32, 16, 4, 64, "f32", True),
+    (1, 257, 2, 17, 33, 2, 128, "f32", False),
+    (2, 200, 2, 64, 256, 1, 256, "bf16", False),
+    (1, 1, 2, 64, 128, 1, 256, "bf16", True),
+]
+
+
+@pytest.mark.parametrize("case", SMALL, ids=lambda c: "b{}_T{}_H{}_P{}_N{}_G{}_Q{}_{}_init{}".format(*c))
+def test_small_dense(case):
+    b, T, H, P, N, G, Q, dt, init = case
+    wl = workloads.custom(b, T, H, P, N, G, chunk=Q, dtype=dt, init=init)
+    prob = workloads.generate(wl, seed=1)
+    for name, path in paths_for(prob, Q):
+        y, fin = run(prob, path=path)
+        check(prob, y, fin)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "f32"])
+def test_small_packed_with_resets(dtype):
+    lens = [1, 63, 64, 65, 0, 300, 257, 511, 2]
+    wl = workloads.custom(1, 0, H=4, P=64, N=128, G=2, chunk=128, dtype=dtype, init=True, lengths=lens)
+    prob = workloads.generate(wl, seed=2, lengths=lens)
+    for name, path in paths_for(prob, 128):
+        y, fin = run(prob, path=path)
+        check(prob, y, fin)
+
+
+@pytest.mark.parametrize("Q", [64, 128, 256])
+def test_chunk_lengths_agree(Q):
+    wl = workloads.custom(2, 600, H=4, P=64, N=64, G=1, chunk=Q, dtype="bf16", init=True)
+    prob = workloads.generate(wl, seed=3)
+    for name, path in paths_for(prob, Q):
+        y, fin = run(prob, chunk=Q, path=path)
+        check(prob, y, fin)
+
+
+def test_tiny_dt_and_strong_decay():
+    """dt scaled down 1000x (decay ~1, long memory) and A = -1e4 (decay underflows to 0)."""
+    wl = workloads.custom(1, 400, H=4, P=64, N=128, G=1, chunk=256, dtype="bf16", init=True)
+    for kw in (dict(dt_scale=1e-3), dict(A_override=[-1e4, -1.0, -50.0, -1e-3])):
+        prob = workloads.generate(wl, seed=4, **kw)
+        for name, path in paths_for(prob, 256):
+            y, fin = run(prob, path=path)
+            check(prob, y, fin)
+
+
+def test_no_skip_no_init_no_final():
+    wl = workloads.custom(1, 300, H=2, P=64, N=64, G=1, chunk=128, dtype="bf16")
+    prob = workloads.generate(wl, seed=5)
+    prob.D = None
+    for name, path in paths_for(prob, 128):
+        y, fin = run(prob, path=path, return_final=False)
+        assert fin is None
+        check(prob, y, None)
+
+
+def test_deterministic():
+    wl = workloads.custom(2, 700, H=4, P=64, N=128, G=2, chunk=256, dtype="bf16", init=True)
+    prob = workloads.generate(wl, seed=6)
+    dev = to_device(prob)
+    for name, path in paths_for(prob, 256):
+        y1, f1 = run(prob, path=path, dev=dev)
+        y2, f2 = run(prob, path=path, dev=dev)
+        assert torch.equal(y1, y2) and torch.equal(f1, f2), name
+
+
+def test_host_entry_point_matches_device():
+    wl = workloads.custom(1, 500, H=4, P=64, N=64, G=2, chunk=128, dtype="bf16", init=True,
+                          lengths=[100, 0, 400])
+    prob = workloads.generate(wl, seed=7, lengths=[100, 0, 400])
+    y, fin = run(prob)
+    pin = lambda t: None if t is None else t.pin_memory()
+    yh, fh = ssd.ssd_forward_host(pin(prob.x), pin(prob.dt), pin(prob.A), pin(prob.B), pin(prob.C), pin(prob.D),
+                                  pin(prob.init_state), pin(prob.cu_seqlens), chunk=128)
+    assert torch.equal(yh, y.cpu()) and torch.equal(fh, fin.cpu())
+
+
+def test_bad_device_seqlens_sets_status_and_writes_nothing():
+    wl = workloads.custom(1, 300, H=2, P=64, N=64, G=1, chunk=128, dtype="bf16", lengths=[100, 200])
+    prob = workloads.generate(wl, seed=8, lengths=[100, 200])
+    dev = to_device(prob)
+    dev["cu_seqlens"] = torch.tensor([0, 250, 200], dtype=torch.int32, device="cuda")  # not monotone
+    assert ssd.query_status() == 0
+    y = torch.full_like(dev["x"], 7.0)
+    fin = torch.full((2, 2, 64, 64), 7.0, device="cuda")
+    ssd.ssd_forward(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], None, dev["cu_seqlens"], 128,
+                    y=y, final_state=fin)
+    assert ssd.query_status() == 6
+    assert ssd.query_status() == 0  # cleared by the read
+    assert bool((y == 7.0).all()) and bool((fin == 7.0).all())
+
+
+# ----------------------------------------------------------- full-size workloads
+FULL = [workloads.TINY, workloads.MAMBA2_2P7B] + workloads.STATE_SWEEP + workloads.LENGTH_SWEEP + [workloads.PACKED]
+
+
+@pytest.mark.parametrize("wl", FULL, ids=lambda w: w.name)
+def test_full_size_sampled(wl):
+    """Full-size inputs in the launch configuration the bench times (auto path), checked
+    on sampled (sequence, head) pairs against the oracle."""
+    prob = workloads.generate(wl, seed=0)
+    y, fin = run(prob)
+    pairs = sample_pairs(prob, k=6)
+    check(prob, y, fin, pairs=pairs)
+    assert torch.isfinite(y.float()).all()
