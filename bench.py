@@ -228,6 +228,10 @@ def run_ours(args, rank, world, local_rank):
     K = args.steps
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
     dom = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(K)]
+    for a, b in dom:  # torch creates the CUDA event on first record; the library re-records it
+        a.record(stream)
+        b.record(stream)
+    torch.cuda.synchronize()
     sampler = ClockSampler(gpu_selector(local_rank))
     sampler.start()
     launches0 = ssd.kernel_launch_count()
