@@ -51,7 +51,9 @@ typedef enum {
   SSD_ERR_MISALIGNED = 3,     /* a pointer is not 16-byte aligned                            */
   SSD_ERR_CUDA = 4,           /* a CUDA runtime call or kernel launch failed                 */
   SSD_ERR_DEVICE_TIMEOUT = 5, /* a bounded device-side wait gave up (kernel returned early)  */
-  SSD_ERR_BAD_SEQLENS = 6     /* cu_seqlens not 0 = c0 <= c1 <= ... <= c_nseq = seqlen        */
+  SSD_ERR_BAD_SEQLENS = 6,    /* cu_seqlens not 0 = c0 <= c1 <= ... <= c_nseq = seqlen        */
+  SSD_ERR_SCRATCH_LIMIT = 7   /* ssd_forward_noalloc: the shape needs more scratch than
+                                 SSD_NOALLOC_SCRATCH_BYTES                                   */
 } ssd_status;
 
 /*
@@ -103,6 +105,37 @@ int ssd_forward(const ssd_shape* shape, const void* x, const float* dt, const fl
 int ssd_forward_host(const ssd_shape* shape, const void* x, const float* dt, const float* A, const void* B,
                      const void* C, const float* D, const float* init_state, const int32_t* cu_seqlens, int chunk,
                      void* y, float* final_state, ssd_stream_t stream);
+
+/*
+ * ssd_forward_noalloc -- ssd_forward for callers that cannot allocate device memory.
+ * The paper has no counterpart to this entry point; it exists for integration.
+ *
+ * Who needs it: a caller that reserves the GPU's memory up front and hands it out
+ * itself (an inference server that gives nearly all HBM to weights and KV caches, or
+ * a runtime that accounts for every byte through its own pool) cannot let a library
+ * call cudaMallocAsync: the allocation can fail once the pool is spent, and it can
+ * stall a latency-critical loop while the driver grows or trims the pool.
+ *
+ * Same arguments, layouts and results as ssd_forward.  It always runs the SIMT
+ * kernels, and their scratch (chunk table, cumsums, chunk states) lives in one
+ * file-scope device array of SSD_NOALLOC_SCRATCH_BYTES that every GPU loading this
+ * library holds until the process exits.  No call allocates: no cudaMalloc,
+ * cudaMallocAsync, cudaFree or allocating library routine.
+ *  - Shapes whose scratch exceeds SSD_NOALLOC_SCRATCH_BYTES (ssd_workspace_bytes with
+ *    ssd_set_path(SSD_PATH_SIMT) gives the need) return SSD_ERR_SCRATCH_LIMIT and
+ *    launch nothing.
+ *  - The first call on a device looks up the array's device address on that device
+ *    (cudaGetSymbolAddress, with that device current); make that first call before any
+ *    stream capture.
+ *  - All calls share the one array and it keeps the last call's contents; each call
+ *    first resets the word that marks the chunk table as not yet built.  Calls whose
+ *    work overlaps on the GPU (different streams, or different host threads, without
+ *    ordering between them) race on the array: serialise them.
+ */
+#define SSD_NOALLOC_SCRATCH_BYTES (32u << 20)
+int ssd_forward_noalloc(const ssd_shape* shape, const void* x, const float* dt, const float* A, const void* B,
+                        const void* C, const float* D, const float* init_state, const int32_t* cu_seqlens,
+                        int chunk, void* y, float* final_state, ssd_stream_t stream);
 
 /* Bytes of stream-ordered scratch ssd_forward takes for this shape (informational). */
 size_t ssd_workspace_bytes(const ssd_shape* shape, int chunk);

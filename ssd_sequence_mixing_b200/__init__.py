@@ -27,7 +27,10 @@ STATUS = {
     4: "SSD_ERR_CUDA",
     5: "SSD_ERR_DEVICE_TIMEOUT",
     6: "SSD_ERR_BAD_SEQLENS",
+    7: "SSD_ERR_SCRATCH_LIMIT",
 }
+# Size of the static scratch array behind ssd_forward_noalloc (SSD_NOALLOC_SCRATCH_BYTES).
+NOALLOC_SCRATCH_BYTES = 32 << 20
 # Every entry point include/ssd.h declares.
 EXPORTS = (
     "ssd_forward",
@@ -39,6 +42,7 @@ EXPORTS = (
     "ssd_select_path",
     "ssd_profile_dominant",
     "ssd_kernel_launch_count",
+    "ssd_forward_noalloc",
 )
 
 
@@ -68,7 +72,7 @@ def _open() -> ctypes.CDLL:
     lib = ctypes.CDLL(LIB_PATH)
     V, I, SP = ctypes.c_void_p, ctypes.c_int, ctypes.POINTER(SsdShape)
     fwd = [SP, V, V, V, V, V, V, V, V, I, V, V, V]
-    for name in ("ssd_forward", "ssd_forward_host"):
+    for name in ("ssd_forward", "ssd_forward_host", "ssd_forward_noalloc"):
         getattr(lib, name).argtypes = fwd
         getattr(lib, name).restype = I
     lib.ssd_workspace_bytes.argtypes = [SP, I]
@@ -183,6 +187,36 @@ def ssd_forward(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Ten
                               ctypes.c_void_p(handle))
     if rc:
         raise SsdError(rc, "ssd_forward")
+    return y, final_state
+
+
+def ssd_forward_noalloc(x, dt, A, B, C, D=None, init_state=None, cu_seqlens=None, chunk: int = 256,
+                        y: Optional[torch.Tensor] = None, final_state: Optional[torch.Tensor] = None,
+                        return_final: bool = True, stream=None):
+    """ssd_forward for callers that cannot allocate device memory inside the call.
+
+    A caller that owns the GPU's memory through its own pool (a server that gives HBM to
+    weights and KV caches up front) cannot let the library call cudaMallocAsync.  The C entry
+    point allocates nothing: its scratch is a static device array of NOALLOC_SCRATCH_BYTES
+    shared by all calls (serialise calls; the first call on a device should precede any
+    stream capture).  Pass ``y`` and ``final_state`` to keep this wrapper allocation-free too;
+    otherwise it creates them with torch before the call.  Shapes needing more scratch raise
+    SsdError with SSD_ERR_SCRATCH_LIMIT.
+    """
+    device = x.device
+    if device.type != "cuda":
+        raise ValueError("ssd_forward_noalloc takes CUDA tensors")
+    y, final_state = _prepare(x, dt, A, B, C, D, init_state, cu_seqlens, y, final_state, return_final, device)
+    shape = make_shape(x, B, cu_seqlens)
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    with torch.cuda.device(device):
+        rc = _lib.ssd_forward_noalloc(ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                      _ptr(init_state), _ptr(cu_seqlens), int(chunk), _ptr(y), _ptr(final_state),
+                                      ctypes.c_void_p(handle))
+    if rc:
+        raise SsdError(rc, "ssd_forward_noalloc")
     return y, final_state
 
 

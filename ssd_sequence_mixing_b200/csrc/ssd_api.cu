@@ -158,6 +158,11 @@ int forward_impl(const ssd_shape* s, const void* x, const float* dt, const float
 
 namespace ssd {
 void count_launches(int n) { g_launches.fetch_add((uint64_t)n); }
+unsigned int* device_status_word() { return status_ptr(); }
+int check_shape(const ssd_shape* s, bool packed, int chunk) {
+  const void* f = (const void*)16;  // stands for every required pointer: only shapes are checked
+  return validate(s, f, (const float*)f, (const float*)f, f, f, packed ? (const int32_t*)f : nullptr, chunk, f);
+}
 }  // namespace ssd
 
 extern "C" {
@@ -261,6 +266,7 @@ const char* ssd_status_string(int status) {
     case SSD_ERR_CUDA: return "CUDA runtime error";
     case SSD_ERR_DEVICE_TIMEOUT: return "a bounded device-side wait gave up";
     case SSD_ERR_BAD_SEQLENS: return "cu_seqlens must be 0 = c0 <= c1 <= ... <= c_nseq = seqlen";
+    case SSD_ERR_SCRATCH_LIMIT: return "shape needs more scratch than SSD_NOALLOC_SCRATCH_BYTES";
     default: return "unknown status";
   }
 }

@@ -71,6 +71,12 @@ inline int max_chunks(int64_t tokens, int nseq, int Q) { return (int)((tokens + 
 // Adds n to the process-wide count of kernels launched by the library.
 void count_launches(int n);
 
+// Address of the current device's status word (looked up once per device), or null.
+unsigned int* device_status_word();
+
+// ssd_forward's shape and chunk rules (and the optional host cu_seqlens check), no launch.
+int check_shape(const ssd_shape* s, bool packed, int chunk);
+
 // Launchers implemented in the kernel files.
 cudaError_t launch_chunk_table(const Problem& pb, cudaStream_t st);
 cudaError_t launch_simt(const Problem& pb, cudaStream_t st);
