@@ -101,6 +101,20 @@ def load_traffic(kernel: str):
     return rec.get("dram_bytes_per_launch")
 
 
+# ----------------------------------------------------------- multi-rank timing
+def aggregate_max(seconds: float, world: int, device) -> float:
+    """Max over ranks of a per-rank device time (every rank must call it)."""
+    t = torch.tensor([seconds], dtype=torch.float64, device=device)
+    if world > 1:
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def weak_scaling_value(tokens_per_rank: int, steps: int, world: int, max_total_s: float) -> float:
+    """Whole-job tokens/s: every rank processed its own batch `steps` times."""
+    return world * tokens_per_rank * steps / max_total_s
+
+
 # --------------------------------------------------------------------- clocks
 class ClockSampler:
     """nvidia-smi sampling of SM clocks and throttle reasons around a timed region."""
@@ -252,12 +266,8 @@ def run_ours(args, rank, world, local_rank):
 
     step_ms = [a.elapsed_time(b) for a, b in ev]
     dom_ms = [a.elapsed_time(b) for a, b in dom]
-    total_s = sum(step_ms) / 1e3
-    t = torch.tensor([total_s], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-    max_total = float(t.item())
-    value = world * wl.tokens * K / max_total
+    max_total = aggregate_max(sum(step_ms) / 1e3, world, dev)
+    value = weak_scaling_value(wl.tokens, K, world, max_total)
 
     # end to end through the host-buffer entry point: H2D inputs, compute, D2H outputs
     pin = lambda v: None if v is None else v.pin_memory()
@@ -283,10 +293,7 @@ def run_ours(args, rank, world, local_rank):
         b.record(stream)
         b.synchronize()
         e2e_ms.append(a.elapsed_time(b))
-    te = torch.tensor([sum(e2e_ms) / 1e3], dtype=torch.float64, device=dev)
-    if world > 1:
-        torch.distributed.all_reduce(te, op=torch.distributed.ReduceOp.MAX)
-    e2e_value = world * wl.tokens * args.e2e_steps / float(te.item())
+    e2e_value = weak_scaling_value(wl.tokens, args.e2e_steps, world, aggregate_max(sum(e2e_ms) / 1e3, world, dev))
 
     if rank != 0:
         return None

@@ -65,8 +65,17 @@ int validate(const ssd_shape* s, const void* x, const float* dt, const float* A,
 }
 
 struct Scratch {
-  size_t table, seq_first, nchunks, cs, states, total;
+  size_t table, seq_first, nchunks, cs, states, seq_tiles, carry, carry_flag, total;
+  int ranges;
 };
+
+int device_sms() {
+  int dev = 0, sms = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) !=
+                                                 cudaSuccess)
+    return 148;
+  return sms;
+}
 
 Scratch scratch_layout(const ssd_shape* s, const int32_t* cu, int chunk, int path) {
   auto up = [](size_t v) { return (v + 255) & ~(size_t)255; };
@@ -84,7 +93,18 @@ Scratch scratch_layout(const ssd_shape* s, const int32_t* cu, int chunk, int pat
     st_bytes = up(sizeof(float) * (size_t)Cmax * s->nheads * s->headdim * s->dstate);
   }
   w.states = w.cs + cs_bytes;
-  w.total = w.states + st_bytes;
+  w.seq_tiles = w.states + st_bytes;
+  w.carry = w.seq_tiles;
+  w.carry_flag = w.seq_tiles;
+  w.total = w.seq_tiles;
+  w.ranges = 0;
+  if (path == SSD_PATH_TC) {
+    // one CTA per SM; each may hand a (2 heads x P x N) fp32 state and two cumsums on
+    w.ranges = device_sms();
+    w.carry = w.seq_tiles + up(sizeof(int32_t) * (size_t)(nseq + 1));
+    w.carry_flag = w.carry + up(sizeof(float) * (size_t)w.ranges * 2 * (s->headdim * s->dstate + 1));
+    w.total = w.carry_flag + up(sizeof(int32_t) * (size_t)w.ranges);
+  }
   return w;
 }
 
@@ -147,6 +167,10 @@ int forward_impl(const ssd_shape* s, const void* x, const float* dt, const float
   pb.nchunks = (int32_t*)(ws + w.nchunks);
   pb.cs = (float*)(ws + w.cs);
   pb.states = (float*)(ws + w.states);
+  pb.seq_tiles = path == SSD_PATH_TC ? (int32_t*)(ws + w.seq_tiles) : nullptr;
+  pb.carry = (float*)(ws + w.carry);
+  pb.carry_flag = (int32_t*)(ws + w.carry_flag);
+  pb.ranges = w.ranges;
 
   cudaError_t e = ssd::launch_chunk_table(pb, st);
   if (e == cudaSuccess) e = path == SSD_PATH_TC ? ssd::launch_tc(pb, st) : ssd::launch_simt(pb, st);

@@ -43,6 +43,11 @@ struct Problem {
   float* cs;           // (Cmax, H, Q) in-chunk inclusive cumsum of dt * A
   float* states;       // (Cmax, H, P, N) chunk states, then chunk start states
   int Cmax;
+  // tensor-core path scratch
+  int32_t* seq_tiles;  // nseq + 1: prefix over sequences of ceil(len / kTcTile)
+  float* carry;        // (ranges, 2, P, N) states handed between CTAs, then (ranges, 2) cumsums
+  int32_t* carry_flag; // (ranges) 1 once a CTA has published its carry
+  int ranges;          // CTAs of the tensor-core launch
   // host-side measurement hooks (events around the dominant kernel, or null)
   cudaEvent_t prof_start, prof_stop;
 };
@@ -64,6 +69,9 @@ template <>
 __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) {
   return __float2bfloat16_rn(v);
 }
+
+// Tile length (tokens) of the tensor-core path: the UMMA M dimension.
+constexpr int kTcTile = 128;
 
 // Upper bound on the number of chunks over all sequences: sum ceil(len_s/Q) <= ceil(T/Q) + nseq.
 inline int max_chunks(int64_t tokens, int nseq, int Q) { return (int)((tokens + Q - 1) / Q) + nseq; }

@@ -49,29 +49,38 @@ __global__ void __launch_bounds__(1024) chunk_table_kernel(Problem pb) {
     }
     return;
   }
-  for (int base = 0; base < pb.nseq; base += blockDim.x) {
-    const int s = base + tid;
-    int n = 0;
-    if (s < pb.nseq) {
-      const int64_t len = seq_off(pb, s + 1) - seq_off(pb, s);
-      n = (int)((len + pb.Q - 1) / pb.Q);
-    }
-    s_scan[tid] = n;
+  // Two prefix sums over sequences: chunks of Q tokens (SIMT path) and, when the
+  // tensor-core path asked for it, tiles of kTcTile tokens.
+  for (int pass = 0; pass < (pb.seq_tiles ? 2 : 1); ++pass) {
+    const int unit = pass == 0 ? pb.Q : kTcTile;
+    int32_t* out = pass == 0 ? pb.seq_first : pb.seq_tiles;
+    if (tid == 0) s_carry = 0;
     __syncthreads();
-    for (int off = 1; off < (int)blockDim.x; off <<= 1) {
-      const int v = tid >= off ? s_scan[tid - off] : 0;
+    for (int base = 0; base < pb.nseq; base += blockDim.x) {
+      const int s = base + tid;
+      int n = 0;
+      if (s < pb.nseq) {
+        const int64_t len = seq_off(pb, s + 1) - seq_off(pb, s);
+        n = (int)((len + unit - 1) / unit);
+      }
+      s_scan[tid] = n;
       __syncthreads();
-      s_scan[tid] += v;
+      for (int off = 1; off < (int)blockDim.x; off <<= 1) {
+        const int v = tid >= off ? s_scan[tid - off] : 0;
+        __syncthreads();
+        s_scan[tid] += v;
+        __syncthreads();
+      }
+      if (s < pb.nseq) out[s] = s_carry + s_scan[tid] - n;
+      __syncthreads();
+      if (tid == blockDim.x - 1) s_carry += s_scan[tid];
       __syncthreads();
     }
-    if (s < pb.nseq) pb.seq_first[s] = s_carry + s_scan[tid] - n;
+    if (tid == 0) {
+      out[pb.nseq] = s_carry;
+      if (pass == 0) *pb.nchunks = s_carry;
+    }
     __syncthreads();
-    if (tid == blockDim.x - 1) s_carry += s_scan[tid];
-    __syncthreads();
-  }
-  if (tid == 0) {
-    pb.seq_first[pb.nseq] = s_carry;
-    *pb.nchunks = s_carry;
   }
   for (int s = tid; s < pb.nseq; s += blockDim.x) {
     const int64_t off = seq_off(pb, s), len = seq_off(pb, s + 1) - off;

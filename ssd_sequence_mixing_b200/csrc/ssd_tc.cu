@@ -23,9 +23,35 @@
 // status word, drains what is in flight (bounded), frees tensor memory and exits.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <stdio.h>
+#include <stdlib.h>
 
 #include "sm100_ptx.cuh"
 #include "ssd_tc.cuh"
+
+#ifndef SSD_TRACE
+#define SSD_TRACE 0  // 1: record per-phase clock64 stamps of the first CTAs (profiling builds only)
+#endif
+#if SSD_TRACE
+namespace ssd {
+constexpr int kTraceCtas = 4, kTraceTiles = 64, kTraceMarks = 16;
+__device__ unsigned long long g_trace[2 * kTraceCtas * kTraceTiles * kTraceMarks];
+}  // namespace ssd
+extern "C" int ssd_trace_dump(unsigned long long* host, int n) {
+  return (int)cudaMemcpyFromSymbol(host, ssd::g_trace, sizeof(unsigned long long) * n);
+}
+#define TRACE_MARK(m)                                                                              \
+  do {                                                                                             \
+    if ((tid == 0 || tid == 128) && blockIdx.x < kTraceCtas && trace_tile < kTraceTiles)           \
+      g_trace[(((tid >> 7) * kTraceCtas + blockIdx.x) * kTraceTiles + trace_tile) * kTraceMarks + \
+              (m)] = clock64();                                                                    \
+  } while (0)
+#else
+#define TRACE_MARK(m) \
+  do {                \
+  } while (0)
+#endif
+
 
 namespace ssd {
 
@@ -33,328 +59,587 @@ namespace {
 
 using namespace sm100;
 
-constexpr int kTile = 128;         // tokens per tile (UMMA M)
-constexpr int kHeadDim = 64;       // P supported by this path
-constexpr int kWGThreads = 128;    // one warpgroup per head: thread i <-> TMEM lane i
-constexpr int kHeads = 2;          // heads of one B/C group processed together
-constexpr int kThreads = kHeads * kWGThreads;
+constexpr int kTile = 128;          // tokens per tile (UMMA M)
+constexpr int kHeadDim = 64;        // P supported by this path
+constexpr int kWGThreads = 128;     // a warpgroup: thread i <-> TMEM lane i
+constexpr int kHeads = 2;           // heads of one B/C group processed together
+constexpr int kComputeThreads = kHeads * kWGThreads;  // one warpgroup per head
+constexpr int kComputeWarps = kComputeThreads / 32;
+constexpr int kThreads = kComputeThreads + 32;  // + one issuer warp (TMA and UMMA)
+constexpr int kWGBarrier = 1;       // named barrier of the two compute warpgroups
 constexpr uint32_t kTmemCols = 512;
-// TMEM columns.  S (fp32, 128 cols) is reused for the right-factor accumulator s^T of
-// both heads once the masks have read it; P_h are bf16 pairs (64 cols per head).
-constexpr uint32_t kColS = 0, kColSt = 0, kColP = 128, kColY = 256, kColYo = 384;
+// TMEM columns: S = C B^T (fp32, 128), P_h (bf16 pairs, 64 per head), Y_h (64 per head;
+// the left factor is written first, row-scaled, then P_h x_h accumulates on top) and
+// the fp32 state h^T of each head (64 per head): every tile it is scaled by the tile's
+// decay in place and the right-factor MMA accumulates B^T (w o x) onto it.
+constexpr uint32_t kColS = 0, kColP = 128, kColY = 256, kColSt = 384;
 constexpr long long kWaitLimit = 4ll << 30;  // SM cycles (about 2 s) before a wait gives up
+constexpr uint32_t kSuspendHintNs = 1000;    // a waiting thread sleeps until the phase completes, at most 1 us per try
 constexpr uint32_t kAtom = kTile * 128;      // one 128-row x 128-byte swizzled operand column
+
+// mbarriers.  Issuer -> compute: tile loads (tx bytes) and UMMA commits.
+// Compute -> issuer (one arrival per compute warp): ht, xw, p, free; x-free has one arrival.
+enum {
+  kBarLoad0 = 0,  // x, B, C of a tile in x stage 0
+  kBarLoad1,      // ... stage 1
+  kBarS,          // S = C B^T done
+  kBarYo,         // left factor C h^T written into Y
+  kBarSt,         // right factor accumulated onto the state
+  kBarY,          // P x accumulated into Y
+  kBarHt,         // bf16 state for the next tile written
+  kBarXw,         // w o x written and the state scaled by this tile's decay
+  kBarP,          // P written and Y rows scaled
+  kBarFree,       // Y read (the next left factor may overwrite it)
+  kBarXfree,      // a stage's x buffer (which held that tile's y for the TMA store) is reusable
+  kNumBars
+};
 
 template <int NS>
 struct Layout {
   static constexpr uint32_t x = 0;                          // [stage][head] [128 tok][64 p]
   static constexpr uint32_t b = x + 2 * kHeads * kAtom;     // NS/64 atoms [128 tok][64 n]
   static constexpr uint32_t c = b + (NS / 64) * kAtom;
-  static constexpr uint32_t xw = c + (NS / 64) * kAtom;     // [head] [128 tok][64 p]  (N = 128 operand)
-  static constexpr uint32_t ht = xw + kHeads * kAtom;       // [head] [NS n][64 p]     (N = 128 operand)
-  static constexpr uint32_t cs = ht + kHeads * NS * 128;    // float[head][128] in-chunk cumsum
+  static constexpr uint32_t xw = c + (NS / 64) * kAtom;     // [head] [128 tok][64 p]
+  static constexpr uint32_t ht = xw + kHeads * kAtom;       // [head] [NS n][64 p]
+  static constexpr uint32_t cs = ht + kHeads * NS * 128;    // float[head][128] in-chunk cumsum (log2 units)
   static constexpr uint32_t dt = cs + kHeads * kTile * 4;   // float[head][128]
-  static constexpr uint32_t cc = dt + kHeads * kTile * 4;   // float[head][128] column factors
-  static constexpr uint32_t red = cc + kHeads * kTile * 4;  // float[head][4]
-  static constexpr uint32_t bars = red + kHeads * 16;       // load[2], s, mma
-  static constexpr uint32_t bytes = bars + 4 * 8;
+  static constexpr uint32_t dtn = dt + kHeads * kTile * 4;  // float[2][head][128] prefetched dt
+  static constexpr uint32_t cc = dtn + 2 * kHeads * kTile * 4;  // float[head][128] column factors
+  static constexpr uint32_t red = cc + kHeads * kTile * 4;  // float[warpgroup][4]
+  static constexpr uint32_t bars = red + kHeads * 16;       // uint64[kNumBars]
+  static constexpr uint32_t flag = bars + kNumBars * 8;     // int: a wait gave up
+  static constexpr uint32_t bytes = flag + 16;
 };
 template <int NS>
 constexpr uint32_t kDynSmem = Layout<NS>::bytes + 1024;  // + base alignment slack
 
-__device__ __forceinline__ float bf16_lo(uint32_t v) { return __uint_as_float(v << 16); }
-__device__ __forceinline__ float bf16_hi(uint32_t v) { return __uint_as_float(v & 0xFFFF0000u); }
-
-// The tiles one CTA walks: units (sequence, head pair) in a strided order, each
-// unit's 128-token tiles in sequence order.
+// Work split.  The tiles of all units (sequence, head pair), unit by unit and each
+// unit's 128-token tiles in order, form one flat list; CTA r takes the contiguous
+// range [W r / R, W (r + 1) / R).  A range may start inside a unit (it then needs the
+// state the previous CTA reached there: "carry in") and end inside one (it then hands
+// its state on: "carry out").  A CTA processes its last, truncated piece first, so the
+// state it hands on is ready early; then the whole units; then the piece that needs a
+// carry.  Issuer and compute threads walk the same sequence.
 struct TileCursor {
-  int unit, k0, len;
-  int64_t tb;
+  int unit, k0, len;  // k0: token offset of the tile in the sequence
+  int tb;             // first token of the sequence (tokens < 2^31 on this path)
+  int kend;           // token offset where this piece ends
+  int piece;
+  int flags;          // kCarryIn | kCarryOut | kUnitEnd
+};
+enum { kCarryIn = 1, kCarryOut = 2, kUnitEnd = 4 };
+
+struct RangePlan {
+  int u0, k0, u1, ke1, npieces;  // first unit/tile, last unit and its end tile (tiles)
+  int carry_src;                 // the CTA whose range holds the tile before this range's first
 };
 
-__device__ __forceinline__ bool cursor_load(const Problem& pb, int unit, TileCursor& c) {
-  const int units = pb.nseq * (pb.H / kHeads);
-  if (unit >= units) return false;
-  const int s = unit / (pb.H / kHeads);
-  c.unit = unit;
-  c.k0 = 0;
-  c.tb = seq_off(pb, s);
+__device__ __forceinline__ int unit_tiles(const Problem& pb, int u) {
+  const int s = u / (pb.H / kHeads);
+  return pb.seq_tiles[s + 1] - pb.seq_tiles[s];
+}
+
+__device__ __forceinline__ int64_t unit_first_tile(const Problem& pb, int u) {
+  const int pairs = pb.H / kHeads;
+  const int s = u / pairs;
+  return (int64_t)pb.seq_tiles[s] * pairs + (int64_t)(u % pairs) * (pb.seq_tiles[s + 1] - pb.seq_tiles[s]);
+}
+
+// The unit holding flat tile w (0 <= w < W).
+__device__ __forceinline__ int unit_of_tile(const Problem& pb, int64_t w) {
+  const int pairs = pb.H / kHeads;
+  int lo = 0, hi = pb.nseq;  // seq_tiles[lo] * pairs <= w < seq_tiles[hi] * pairs
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if ((int64_t)pb.seq_tiles[mid] * pairs <= w)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  const int T = pb.seq_tiles[lo + 1] - pb.seq_tiles[lo];
+  return lo * pairs + (int)((w - (int64_t)pb.seq_tiles[lo] * pairs) / T);
+}
+
+__device__ __forceinline__ RangePlan plan_range(const Problem& pb) {
+  RangePlan rp{};
+  const int64_t W = (int64_t)pb.seq_tiles[pb.nseq] * (pb.H / kHeads);
+  const int64_t w0 = W * blockIdx.x / gridDim.x, w1 = W * (blockIdx.x + 1) / gridDim.x;
+  if (w0 >= w1) return rp;
+  rp.u0 = unit_of_tile(pb, w0);
+  rp.k0 = (int)(w0 - unit_first_tile(pb, rp.u0));
+  rp.u1 = unit_of_tile(pb, w1 - 1);
+  rp.ke1 = (int)(w1 - unit_first_tile(pb, rp.u1));
+  rp.npieces = rp.u0 == rp.u1 ? 1 : rp.u1 - rp.u0 + 1;
+  // range r holds tiles [W r / R, W (r + 1) / R): tile w lies in range ceil((w + 1) R / W) - 1
+  // (empty ranges are skipped over when there are fewer tiles than CTAs)
+  if (w0 > 0) rp.carry_src = (int)((w0 * gridDim.x + W - 1) / W) - 1;
+  return rp;
+}
+
+// Loads piece `pi` (processing order) into c; false when it has no tiles.
+__device__ __forceinline__ bool load_piece(const Problem& pb, const RangePlan& rp, int pi, TileCursor& c) {
+  int u, kb, ke;
+  if (rp.npieces == 1) {
+    u = rp.u0, kb = rp.k0, ke = rp.ke1;
+  } else if (pi == 0) {  // the truncated last piece first
+    u = rp.u1, kb = 0, ke = rp.ke1;
+  } else if (pi < rp.npieces - 1) {  // whole units
+    u = rp.u0 + pi, kb = 0, ke = unit_tiles(pb, rp.u0 + pi);
+  } else {  // the first piece last: it may need the previous CTA's state
+    u = rp.u0, kb = rp.k0, ke = unit_tiles(pb, rp.u0);
+  }
+  if (ke <= kb) return false;
+  const int pairs = pb.H / kHeads;
+  const int s = u / pairs;
+  c.unit = u;
+  c.tb = (int)seq_off(pb, s);
   c.len = (int)(seq_off(pb, s + 1) - c.tb);
+  c.k0 = kb * kTile;
+  c.kend = min(ke * kTile, c.len);
+  c.piece = pi;
+  const bool unit_end = ke == unit_tiles(pb, u);
+  c.flags = (kb > 0 ? kCarryIn : 0) | (unit_end ? kUnitEnd : kCarryOut);
   return true;
 }
 
-// Advances to the next tile (skipping empty sequences' tile loops); false when done.
-__device__ __forceinline__ bool cursor_next(const Problem& pb, TileCursor& c) {
+__device__ __forceinline__ bool cursor_from(const Problem& pb, const RangePlan& rp, int pi, TileCursor& c) {
+  for (; pi < rp.npieces; ++pi)
+    if (load_piece(pb, rp, pi, c)) return true;
+  return false;
+}
+
+__device__ __forceinline__ bool cursor_first(const Problem& pb, const RangePlan& rp, TileCursor& c) {
+  return cursor_from(pb, rp, 0, c);
+}
+
+// Advances to the next tile of this CTA's range; false when done.
+__device__ __forceinline__ bool cursor_next(const Problem& pb, const RangePlan& rp, TileCursor& c) {
   c.k0 += kTile;
-  while (c.k0 >= c.len) {
-    if (!cursor_load(pb, c.unit + gridDim.x, c)) return false;
-    if (c.len > 0) return true;
+  if (c.k0 < c.kend) return true;
+  return cursor_from(pb, rp, c.piece + 1, c);
+}
+
+// One arrival for the whole warp, after every lane's prior work (the lanes' own fences
+// come before it).
+__device__ __forceinline__ void warp_arrive(uint64_t* bar) {
+  __syncwarp();
+  if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+  __syncwarp();
+}
+
+// Bounded wait that also gives up when another thread has recorded a failure.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (!mbar_try_wait_sleep(bar, parity, kSuspendHintNs)) {
+    if (*abort_flag) return false;
+    if (clock64() - t0 > kWaitLimit) {
+      *abort_flag = 1;
+      return false;
+    }
   }
   return true;
 }
 
+// ------------------------------------------------------------------ issuer
 template <int NS>
-__device__ __forceinline__ void issue_x(const CUtensorMap* tm_x, uint8_t* sx_stage, uint64_t* bar,
-                                        const Problem& pb, const TileCursor& c) {
-  const int h0 = (c.unit % (pb.H / kHeads)) * kHeads;
-#pragma unroll
-  for (int hh = 0; hh < kHeads; ++hh)
-    tma_load_3d(sx_stage + hh * kAtom, tm_x, 0, h0 + hh, (int)(c.tb + c.k0), bar);
-}
-
-template <int NS>
-__device__ __forceinline__ void issue_bc(const CUtensorMap* tm_b, const CUtensorMap* tm_c, uint8_t* sb,
-                                         uint8_t* sc, uint64_t* bar, const Problem& pb, const TileCursor& c) {
-  const int g = ((c.unit % (pb.H / kHeads)) * kHeads) / pb.hpg;
-#pragma unroll
-  for (int a = 0; a < NS / 64; ++a) {
-    tma_load_3d(sb + a * kAtom, tm_b, a * 64, g, (int)(c.tb + c.k0), bar);
-    tma_load_3d(sc + a * kAtom, tm_c, a * 64, g, (int)(c.tb + c.k0), bar);
-  }
-}
-
-template <int NS>
-__global__ void __launch_bounds__(kThreads, 1)
-    ssd_fused_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-                        const __grid_constant__ CUtensorMap tm_c, Problem pb) {
+__device__ void issuer_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, const CUtensorMap* tm_c,
+                            const Problem& pb, uint8_t* smem, uint32_t tmem, uint64_t* bars,
+                            volatile int* abort_flag) {
   using L = Layout<NS>;
-  extern __shared__ uint8_t smem_raw[];
-  __shared__ uint32_t s_tmem_base;
-  const int tid = threadIdx.x;
-  const int hw = tid / kWGThreads;     // which head of the pair this warpgroup handles
-  const int i = tid % kWGThreads;      // row / TMEM lane
-  const int wq = i >> 5, lane = i & 31;  // lane quarter of this warp
-  const bool issuer = tid == 0;
-
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint8_t* sx = smem + L::x;
   uint8_t* sb = smem + L::b;
   uint8_t* sc = smem + L::c;
+  constexpr uint32_t kLoadBytes = kHeads * kAtom + 2u * (NS / 64) * kAtom;
+  const uint32_t id_s = idesc_bf16(128, 128, 0, 0);
+  const uint32_t id_y = idesc_bf16(128, 64, 0, 1);
+  const uint32_t id_yo = idesc_bf16(128, 128, 0, 1);
+  const uint32_t id_st = idesc_bf16(128, 128, 1, 1);
+  const uint32_t a_sb = smem_u32(sb), a_sc = smem_u32(sc);
+  const uint32_t a_sxw = smem_u32(smem + L::xw), a_sht = smem_u32(smem + L::ht);
+  // For N = 64 the B^T operand has one M atom; the second (unused) half of s^T reads
+  // the C tile that follows it, and those lanes are ignored.
+  const uint32_t lbo_bt = kAtom;
+  const int pairs = pb.H / kHeads;
+
+  auto issue_x = [&](int stage, const TileCursor& c) {
+    const int h0 = (c.unit % pairs) * kHeads;
+#pragma unroll
+    for (int hh = 0; hh < kHeads; ++hh)
+      tma_load_3d(sx + (stage * kHeads + hh) * kAtom, tm_x, 0, h0 + hh, c.tb + c.k0, &bars[stage]);
+  };
+  auto issue_bc = [&](int stage, const TileCursor& c) {
+    const int g = ((c.unit % pairs) * kHeads) / pb.hpg;
+#pragma unroll
+    for (int a = 0; a < NS / 64; ++a) {
+      tma_load_3d(sb + a * kAtom, tm_b, a * 64, g, c.tb + c.k0, &bars[stage]);
+      tma_load_3d(sc + a * kAtom, tm_c, a * 64, g, c.tb + c.k0, &bars[stage]);
+    }
+  };
+
+  uint32_t phase = 0;    // bit k: parity of the next phase of bars[k] this thread waits for
+  uint32_t pending = 0;  // bit k: async work on bars[k] issued and not waited for
+  auto wait = [&](int k) -> bool {
+    if (!wait_or_abort(&bars[k], (phase >> k) & 1u, abort_flag)) return false;
+    phase ^= 1u << k;
+    pending &= ~(1u << k);
+    return true;
+  };
+
+  const RangePlan rp = plan_range(pb);
+  TileCursor cur;
+  bool have = cursor_first(pb, rp, cur);
+  int stage = 0, t = 0;
+  if (have) {
+    mbar_expect_tx(&bars[kBarLoad0], kLoadBytes);
+    issue_x(0, cur);
+    issue_bc(0, cur);
+    pending |= 1u << kBarLoad0;
+  }
+  bool ok = true;
+  while (have) {
+    TileCursor nxt = cur;
+    const bool have_next = cursor_next(pb, rp, nxt);
+    // S = C B^T once this tile's x, B, C are in (the previous mask finished with S).
+    if (!(ok = wait(stage))) break;
+    tc_fence_after();
+#pragma unroll
+    for (int kk = 0; kk < NS / 16; ++kk) {
+      const uint32_t koff = (kk >> 2) * kAtom + (kk & 3) * 32;
+      umma_f16(tmem + kColS, sdesc_sw128(a_sc + koff, 16, 1024), sdesc_sw128(a_sb + koff, 16, 1024), id_s, kk > 0);
+    }
+    umma_commit(&bars[kBarS]);
+    pending |= 1u << kBarS;
+    // Left factor C h^T into Y: needs the bf16 state and the previous epilogue done with Y.
+    if (!(ok = wait(kBarHt))) break;
+    if (t > 0 && !(ok = wait(kBarFree))) break;
+    tc_fence_after();
+#pragma unroll
+    for (int kk = 0; kk < NS / 16; ++kk) {
+      const uint32_t koff = (kk >> 2) * kAtom + (kk & 3) * 32;
+      umma_f16(tmem + kColY, sdesc_sw128(a_sc + koff, 16, 1024), sdesc_sw128(a_sht + kk * 2048, NS * 128, 1024),
+               id_yo, kk > 0);
+    }
+    umma_commit(&bars[kBarYo]);
+    pending |= 1u << kBarYo;
+    if (have_next) {  // the other x stage (tile t-1's x, then its y) is free once its y store read it
+      if (t > 0 && !(ok = wait(kBarXfree))) break;
+      fence_proxy_async();
+      mbar_expect_tx(&bars[stage ^ 1], kLoadBytes);
+      issue_x(stage ^ 1, nxt);
+      pending |= 1u << (stage ^ 1);
+    }
+    // Right factor onto the (decay-scaled) state: h^T += B^T [w0 x0 | w1 x1].
+    if (!(ok = wait(kBarXw))) break;
+    tc_fence_after();
+#pragma unroll
+    for (int kk = 0; kk < kTile / 16; ++kk)
+      umma_f16(tmem + kColSt, sdesc_sw128(a_sb + kk * 2048, lbo_bt, 1024),
+               sdesc_sw128(a_sxw + kk * 2048, kAtom, 1024), id_st, 1);
+    umma_commit(&bars[kBarSt]);
+    pending |= 1u << kBarSt;
+    // Y_h += P_h x_h (A from tensor memory).
+    if (!(ok = wait(kBarP))) break;
+    tc_fence_after();
+    {
+      const uint32_t a_sx = smem_u32(sx + stage * kHeads * kAtom);
+#pragma unroll
+      for (int hh = 0; hh < kHeads; ++hh) {
+#pragma unroll
+        for (int kk = 0; kk < kTile / 16; ++kk)
+          umma_f16_ta(tmem + kColY + hh * 64, tmem + kColP + hh * 64 + kk * 8,
+                      sdesc_sw128(a_sx + hh * kAtom + kk * 2048, kAtom, 1024), id_y, 1);
+      }
+    }
+    umma_commit(&bars[kBarY]);
+    pending |= 1u << kBarY;
+    // B and C are free once S and both factors are done: next tile's.
+    if (have_next) {
+      if (!(ok = wait(kBarS)) || !(ok = wait(kBarYo)) || !(ok = wait(kBarSt))) break;
+      fence_proxy_async();
+      issue_bc(stage ^ 1, nxt);
+    }
+    cur = nxt;
+    have = have_next;
+    stage ^= 1;
+    ++t;
+  }
+  if (!ok) {
+    *abort_flag = 1;
+    // Drain what this thread issued (again bounded) before tensor memory is freed.
+    for (int k = 0; k < kNumBars; ++k)
+      if (pending & (1u << k)) mbar_wait_bounded(&bars[k], (phase >> k) & 1u, kWaitLimit);
+  }
+}
+
+// --------------------------------------------------------- compute warpgroups
+// Two warpgroups, one per head of the pair.  Thread i owns TMEM lane / tile row i.
+template <int NS>
+__device__ void compute_loop(const CUtensorMap* tm_y, const Problem& pb, uint8_t* smem, uint32_t tmem,
+                             uint64_t* bars, volatile int* abort_flag) {
+  using L = Layout<NS>;
+  const int tid = threadIdx.x;
+  const int hw = tid / kWGThreads;       // head of the pair
+  const int i = tid % kWGThreads;        // row / TMEM lane
+  const int wq = i >> 5, lane = i & 31;  // lane quarter of this warp
+  const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+  uint8_t* sx = smem + L::x;
   uint8_t* sxw = smem + L::xw;
   uint8_t* sht = smem + L::ht;
   float* s_cs = reinterpret_cast<float*>(smem + L::cs) + hw * kTile;
   float* s_dt = reinterpret_cast<float*>(smem + L::dt) + hw * kTile;
   float* s_cc = reinterpret_cast<float*>(smem + L::cc) + hw * kTile;
   float* s_red = reinterpret_cast<float*>(smem + L::red) + hw * 4;
-  uint64_t* bar_load = reinterpret_cast<uint64_t*>(smem + L::bars);  // [2], one per x stage
-  uint64_t* bar_s = bar_load + 2;
-  uint64_t* bar_mma = bar_load + 3;
+  float* s_dtn = reinterpret_cast<float*>(smem + L::dtn) + hw * kTile;  // [buf][head][128]
+  const int pairs = pb.H / kHeads;
+  const int units = pb.nseq * pairs;
 
-  if (*pb.nchunks < 0) return;  // cu_seqlens rejected by the table kernel
+  uint32_t phase = 0;
+  // Uniform bounded wait of all compute threads on an issuer barrier.
+  auto wait = [&](int k) -> bool {
+    const bool mine = wait_or_abort(&bars[k], (phase >> k) & 1u, abort_flag);
+    if (bar_or(kWGBarrier, kComputeThreads, !mine)) return false;
+    phase ^= 1u << k;
+    return true;
+  };
 
-  if (tid < 32) {
-    tmem_alloc(&s_tmem_base, kTmemCols);
-    tmem_relinquish();
+  // Units whose sequences are empty have no tiles: CTA r writes final = init for the
+  // empty units u with u % R == r.
+  if (pb.final_state && i < NS) {
+    for (int u = blockIdx.x; u < units; u += gridDim.x) {
+      if (unit_tiles(pb, u) != 0) continue;
+      const int s = u / pairs;
+      const int h = (u % pairs) * kHeads + hw;
+      const int64_t base = ((int64_t)s * pb.H + h) * kHeadDim * NS;
+      for (int p = 0; p < kHeadDim; ++p)
+        pb.final_state[base + (int64_t)p * NS + i] = pb.init ? pb.init[base + (int64_t)p * NS + i] : 0.f;
+    }
   }
-  if (issuer) {
-    mbar_init(&bar_load[0], 1);
-    mbar_init(&bar_load[1], 1);
-    mbar_init(bar_s, 1);
-    mbar_init(bar_mma, 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    prefetch_tensormap(&tm_x);
-    prefetch_tensormap(&tm_b);
-    prefetch_tensormap(&tm_c);
-  }
-  tc_fence_before();
-  __syncthreads();
-  tc_fence_after();
-  const uint32_t tmem = s_tmem_base;
-  const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
 
-  constexpr uint32_t kLoadBytes = kHeads * kAtom + 2u * (NS / 64) * kAtom;
-  const uint32_t id_s = idesc_bf16(128, 128, 0, 0);
-  const uint32_t id_y = idesc_bf16(128, 64, 0, 1);
-  const uint32_t id_yo = idesc_bf16(128, 128, 0, 1);
-  const uint32_t id_st = idesc_bf16(128, 128, 1, 1);
-  const uint32_t a_sb = smem_u32(sb), a_sc = smem_u32(sc), a_sxw = smem_u32(sxw), a_sht = smem_u32(sht);
-  // For N = 64 the B^T operand has one M atom; the second (unused) half of s^T reads
-  // the C tile that follows it, and those lanes are ignored.
-  const uint32_t lbo_bt = kAtom;
-
-  uint32_t ph_load[2] = {0, 0}, ph_s = 0, ph_mma = 0;
-  bool ok = true;
-  int pend_load = 0;  // bit k: a load on bar_load[k] issued and not yet waited for
-  bool pend_s = false, pend_mma = false;
-
-  TileCursor cur;
-  bool have = cursor_load(pb, blockIdx.x, cur);
-  while (have && cur.len == 0) have = cursor_next(pb, cur);  // nothing to do for empty sequences
-
-  // Empty sequences still need final = init: handled by the units loop below on the fly.
-  float hst[kHeadDim];
-  int stage = 0;
-  int cur_unit = -1;
-  float cs_base = 0.f, dt_next = 0.f;
-
-  if (have && issuer) {
-    mbar_expect_tx(&bar_load[0], kLoadBytes);
-    issue_x<NS>(&tm_x, sx, &bar_load[0], pb, cur);
-    issue_bc<NS>(&tm_b, &tm_c, sb, sc, &bar_load[0], pb, cur);
-  }
-  if (have) pend_load = 1;
-
-  // Units of this CTA whose sequences are empty get their final state here.
-  auto finish_empty_units = [&](int from_unit, int to_unit) {
-    for (int u = from_unit; u < to_unit; u += gridDim.x) {
-      const int s = u / (pb.H / kHeads);
-      const int h = (u % (pb.H / kHeads)) * kHeads + hw;
-      if (seq_off(pb, s + 1) - seq_off(pb, s) != 0) continue;
-      if (pb.final_state && i < NS) {
-        const int64_t base = ((int64_t)s * pb.H + h) * kHeadDim * NS;
-        for (int p = 0; p < kHeadDim; ++p)
-          pb.final_state[base + (int64_t)p * NS + i] = pb.init ? pb.init[base + (int64_t)p * NS + i] : 0.f;
+  const RangePlan rp = plan_range(pb);
+  // This warpgroup's head state lives in tensor memory as h^T (lane n = state column n,
+  // 64 fp32 columns); its bf16 copy in shared memory is the B operand of the left factor.
+  const uint32_t t_state = tmem + lane_base + kColSt + hw * 64;
+  float cs_base = 0.f;  // in-chunk cumsum (log2 units) before the current tile
+  auto write_ht_from = [&](const uint32_t (&r)[32], int half) {
+    if (i < NS) {
+      uint8_t* hdst = sht + hw * NS * 128;
+#pragma unroll
+      for (int c4 = 0; c4 < 4; ++c4) {
+        uint4 hv;
+        hv.x = bf16x2_of(f2u(r[8 * c4 + 0], r[8 * c4 + 1]));
+        hv.y = bf16x2_of(f2u(r[8 * c4 + 2], r[8 * c4 + 3]));
+        hv.z = bf16x2_of(f2u(r[8 * c4 + 4], r[8 * c4 + 5]));
+        hv.w = bf16x2_of(f2u(r[8 * c4 + 6], r[8 * c4 + 7]));
+        *reinterpret_cast<uint4*>(hdst + sw128_off(i, half * 4 + c4)) = hv;
       }
     }
   };
-  finish_empty_units(blockIdx.x, have ? cur.unit : pb.nseq * (pb.H / kHeads));
+  // State at the start of piece c into tensor memory and its bf16 copy: the sequence's
+  // initial state, or (carry in) the state and cumsum the previous CTA published.
+  // False if that wait gave up.
+  auto load_state = [&](const TileCursor& c) -> bool {
+    const float* src_p = nullptr;
+    if (c.flags & kCarryIn) {
+      const int src = rp.carry_src;
+      bool mine = true;
+      if (tid == 0) {
+        const long long t0 = clock64();
+        while (ld_acquire_gpu(&pb.carry_flag[src]) == 0) {
+          if (*abort_flag || clock64() - t0 > kWaitLimit) {
+            *abort_flag = 1;
+            mine = false;
+            break;
+          }
+          __nanosleep(200);
+        }
+      }
+      __syncwarp();
+      if (bar_or(kWGBarrier, kComputeThreads, !mine)) return false;
+      __threadfence();
+      src_p = pb.carry + ((size_t)src * kHeads + hw) * kHeadDim * NS + i;
+      cs_base = __ldcg(pb.carry + (size_t)pb.ranges * kHeads * kHeadDim * NS + src * kHeads + hw);
+    } else {
+      const int s = c.unit / pairs;
+      const int h = (c.unit % pairs) * kHeads + hw;
+      if (pb.init) src_p = pb.init + ((int64_t)s * pb.H + h) * kHeadDim * NS + i;
+      cs_base = 0.f;
+    }
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      uint32_t r[32];
+#pragma unroll
+      for (int q = 0; q < 32; ++q)
+        r[q] = __float_as_uint((src_p && i < NS) ? __ldcg(src_p + (size_t)(half * 32 + q) * NS) : 0.f);
+      tmem_st32(t_state + half * 32, r);
+      write_ht_from(r, half);
+    }
+    tmem_st_wait();
+    fence_proxy_async();
+    return true;
+  };
+  auto head_of = [&](const TileCursor& c) { return (c.unit % pairs) * kHeads + hw; };
+  // dt of tile c for this thread's token, copied asynchronously into s_dtn[buf]
+  auto prefetch_dt = [&](const TileCursor& c, int buf) {
+    float* dst = s_dtn + buf * kHeads * kTile + i;
+    if (c.k0 + i < c.len)
+      cp_async4(dst, pb.dt + ((int64_t)c.tb + c.k0 + i) * pb.H + head_of(c));
+    else
+      *dst = 0.f;
+    cp_async_commit();
+  };
+  // P values of one 32-column block of S (fp32 bits in r) for row i.
+  auto mask_block = [&](int cb, const uint32_t (&r)[32], float cs_i, uint32_t (&pk)[16]) {
+    if (cb < wq) {  // strictly below the diagonal: exp(cs_i - cs_j) = rf * exp(cs_ref - cs_j)
+      const float rf = ex2(cs_i - s_cs[cb * 32 + 31]);
+      const uint64_t rf2 = f2(rf, rf);
+      const float4* cc4 = reinterpret_cast<const float4*>(s_cc + cb * 32);
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) {
+        const float4 c = cc4[q4];
+        const uint64_t f0 = mul2(rf2, f2(c.x, c.y)), f1 = mul2(rf2, f2(c.z, c.w));
+        pk[2 * q4] = bf16x2_of(mul2(f0, f2u(r[4 * q4], r[4 * q4 + 1])));
+        pk[2 * q4 + 1] = bf16x2_of(mul2(f1, f2u(r[4 * q4 + 2], r[4 * q4 + 3])));
+      }
+    } else {  // diagonal block: mask first (-inf), then exp
+      const float4* c4 = reinterpret_cast<const float4*>(s_cs + cb * 32);
+      const float4* d4 = reinterpret_cast<const float4*>(s_dt + cb * 32);
+#pragma unroll
+      for (int q4 = 0; q4 < 8; ++q4) {
+        const float4 cj = c4[q4], dj = d4[q4];
+        const int j0 = 4 * q4;  // column within the block; this row is `lane`
+        const float e0 = ex2(j0 <= lane ? cs_i - cj.x : -INFINITY);
+        const float e1 = ex2(j0 + 1 <= lane ? cs_i - cj.y : -INFINITY);
+        const float e2 = ex2(j0 + 2 <= lane ? cs_i - cj.z : -INFINITY);
+        const float e3 = ex2(j0 + 3 <= lane ? cs_i - cj.w : -INFINITY);
+        pk[2 * q4] = bf16x2_of(mul2(mul2(f2(e0, e1), f2(dj.x, dj.y)), f2u(r[j0], r[j0 + 1])));
+        pk[2 * q4 + 1] = bf16x2_of(mul2(mul2(f2(e2, e3), f2(dj.z, dj.w)), f2u(r[j0 + 2], r[j0 + 3])));
+      }
+    }
+  };
 
-  while (have && ok) {
-    const int pair = cur.unit % (pb.H / kHeads);
-    const int s = cur.unit / (pb.H / kHeads);
-    const int h = pair * kHeads + hw;
-    const float Ah = pb.A[h];
-    const float Dh = pb.D ? pb.D[h] : 0.f;
-    const int64_t st_base = ((int64_t)s * pb.H + h) * kHeadDim * NS;
+  TileCursor cur;
+  bool have = cursor_first(pb, rp, cur);
+  if (!have) return;
+  if (!load_state(cur)) return;
+  tc_fence_before();
+  warp_arrive(&bars[kBarHt]);
+  prefetch_dt(cur, 0);
+  float a2_cur = pb.A[head_of(cur)] * 1.4426950408889634f;  // A_h log2(e): cumsums are in log2 units
+  float d_cur = pb.D ? pb.D[head_of(cur)] : 0.f;
+  int stage = 0, tile_idx = 0;
+  int trace_tile = 0;
+  (void)trace_tile;
+
+  while (have) {
+    TRACE_MARK(0);
+    const int s = cur.unit / pairs;
+    const int h = head_of(cur);
     const int64_t t0 = cur.tb + cur.k0;
     const int rem = min(kTile, cur.len - cur.k0);
-
-    if (cur.unit != cur_unit) {  // first tile of a unit: initial state, first dt
-      cur_unit = cur.unit;
-#pragma unroll
-      for (int p = 0; p < kHeadDim; ++p) hst[p] = 0.f;
-      if (pb.init && i < NS) {
-#pragma unroll
-        for (int p = 0; p < kHeadDim; ++p) hst[p] = pb.init[st_base + (int64_t)p * NS + i];
-      }
-      dt_next = (i < cur.len) ? pb.dt[(cur.tb + i) * pb.H + h] : 0.f;
-    }
     if (cur.k0 % pb.Q == 0) cs_base = 0.f;
+    const float Ah2 = a2_cur, Dh = d_cur;
 
-    // ---- look ahead: the next tile's x goes to the other stage now
+    // look ahead: next tile's dt (and its head's parameters at a unit change)
     TileCursor nxt = cur;
-    const bool have_next = cursor_next(pb, nxt);
-    if (have_next && issuer) {
-      fence_proxy_async();
-      mbar_expect_tx(&bar_load[stage ^ 1], kLoadBytes);
-      issue_x<NS>(&tm_x, sx + (stage ^ 1) * kHeads * kAtom, &bar_load[stage ^ 1], pb, nxt);
+    const bool have_next = cursor_next(pb, rp, nxt);
+    cp_async_wait_all();  // this tile's dt (each thread reads back its own copy)
+    const float dtj = s_dtn[(tile_idx & 1) * kHeads * kTile + i];
+    if (have_next) {
+      prefetch_dt(nxt, (tile_idx & 1) ^ 1);
+      if (nxt.unit != cur.unit) {
+        a2_cur = pb.A[head_of(nxt)] * 1.4426950408889634f;
+        d_cur = pb.D ? pb.D[head_of(nxt)] : 0.f;
+      }
     }
-    if (have_next) pend_load |= 1 << (stage ^ 1);
 
-    // ---- in-chunk cumsum of dt*A; the next tile's dt is fetched meanwhile
-    const float dtj = dt_next;
-    dt_next = (cur.k0 + kTile + i < cur.len) ? pb.dt[(t0 + kTile + i) * pb.H + h] : 0.f;
-    float v = dtj * Ah;
+    // ---- in-chunk cumsum of dt*A (log2 units)
+    float v = dtj * Ah2;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const float u = __shfl_up_sync(0xffffffffu, v, o);
       if (lane >= o) v += u;
     }
     if (lane == 31) s_red[wq] = v;
-    __syncthreads();
+    bar_sync(kWGBarrier, kComputeThreads);
     float off = cs_base;
     for (int w = 0; w < wq; ++w) off += s_red[w];
     const float cs_i = off + v;
     s_cs[i] = cs_i;
-    __syncthreads();
+    bar_sync(kWGBarrier, kComputeThreads);
     const float cs_start = cs_base;
     const float cs_end = s_cs[kTile - 1];  // tokens past the end add 0
     cs_base = cs_end;
     // column factor for blocks below the diagonal: exp(cs_ref - cs_i) dt_i, with cs_ref
     // the cumsum at the end of i's 32-token block
-    s_cc[i] = __expf(s_cs[wq * 32 + 31] - cs_i) * dtj;
+    s_cc[i] = ex2(s_cs[wq * 32 + 31] - cs_i) * dtj;
     s_dt[i] = dtj;
-    const float w_i = __expf(cs_end - cs_i) * dtj;  // right-factor weight (0 past the end)
+    const float w_i = ex2(cs_end - cs_i) * dtj;  // right-factor weight (0 past the end)
+    const float carry = ex2(cs_i - cs_start);    // decay of the carried-in state to token i
+    TRACE_MARK(1);
 
-    // ---- wait for x, B, C of this tile, then S = C B^T (shared by both heads)
-    ok = mbar_wait_bounded(&bar_load[stage], ph_load[stage], kWaitLimit);
-    if (__syncthreads_or(!ok)) {
-      ok = false;
-      break;
-    }
-    ph_load[stage] ^= 1;
-    pend_load &= ~(1 << stage);
-    pend_s = true;
-    if (issuer) {
-      tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < NS / 16; ++kk) {
-        const uint32_t koff = (kk >> 2) * kAtom + (kk & 3) * 32;
-        umma_f16(tmem + kColS, sdesc_sw128(a_sc + koff, 16, 1024), sdesc_sw128(a_sb + koff, 16, 1024), id_s,
-                 kk > 0);
-      }
-      umma_commit(bar_s);
-    }
-
-    // ---- w o x (right-factor input) and the bf16 state copy, while S runs
+    // ---- this tile's x: w o x, the right-factor input
+    if (!wait(stage)) return;
+    TRACE_MARK(2);
     const uint8_t* sxh = sx + (stage * kHeads + hw) * kAtom;
     {
       uint8_t* dst = sxw + hw * kAtom;
+      const uint32_t w2 = pack_bf16(w_i, w_i);
 #pragma unroll
       for (int c = 0; c < 8; ++c) {
         const uint32_t o = sw128_off(i, c);
         uint4 xv = *reinterpret_cast<const uint4*>(sxh + o);
-        uint32_t* u = reinterpret_cast<uint32_t*>(&xv);
-#pragma unroll
-        for (int q = 0; q < 4; ++q) u[q] = pack_bf16(bf16_lo(u[q]) * w_i, bf16_hi(u[q]) * w_i);
+        xv.x = mul_bf16x2(xv.x, w2);
+        xv.y = mul_bf16x2(xv.y, w2);
+        xv.z = mul_bf16x2(xv.z, w2);
+        xv.w = mul_bf16x2(xv.w, w2);
         *reinterpret_cast<uint4*>(dst + o) = xv;
-      }
-      if (i < NS) {
-        uint8_t* hdst = sht + hw * NS * 128;
-#pragma unroll
-        for (int c = 0; c < 8; ++c) {
-          uint4 hv;
-          hv.x = pack_bf16(hst[8 * c + 0], hst[8 * c + 1]);
-          hv.y = pack_bf16(hst[8 * c + 2], hst[8 * c + 3]);
-          hv.z = pack_bf16(hst[8 * c + 4], hst[8 * c + 5]);
-          hv.w = pack_bf16(hst[8 * c + 6], hst[8 * c + 7]);
-          *reinterpret_cast<uint4*>(hdst + sw128_off(i, c)) = hv;
-        }
       }
     }
     fence_proxy_async();
-
-    // ---- P_h = mask_h(S), bf16 pairs in tensor memory
-    ok = mbar_wait_bounded(bar_s, ph_s, kWaitLimit);
-    if (__syncthreads_or(!ok)) {
-      ok = false;
-      break;
+    {  // state scaled by this tile's decay; the right-factor MMA then accumulates onto it
+      const float decay = ex2(cs_end - cs_start);
+      const uint64_t decay2 = f2(decay, decay);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t r[32];
+        tmem_ld32(t_state + half * 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          float lo, hi;
+          unf2(mul2(decay2, f2u(r[2 * q], r[2 * q + 1])), lo, hi);
+          r[2 * q] = __float_as_uint(lo);
+          r[2 * q + 1] = __float_as_uint(hi);
+        }
+        tmem_st32(t_state + half * 32, r);
+      }
+      tmem_st_wait();
+      tc_fence_before();
     }
-    ph_s ^= 1;
-    pend_s = false;
+    warp_arrive(&bars[kBarXw]);
+    if (tid == 0 && tile_idx > 0) {
+  // the previous tile's y store has read its x stage: release it
+      bulk_wait_read();
+      mbar_arrive(&bars[kBarXfree]);
+    }
+    __syncwarp();
+    TRACE_MARK(3);
+
+    // ---- P_h = mask_h(S), bf16 pairs in tensor memory; S blocks loaded two at a time
+    if (!wait(kBarS)) return;
+    TRACE_MARK(4);
     tc_fence_after();
     {
       const uint32_t colp = kColP + hw * 64;
 #pragma unroll 1
       for (int cb = 0; cb < 4; ++cb) {  // 32-column blocks of S -> P columns 16cb..16cb+15
         uint32_t pk[16];
-        if (cb < wq) {  // strictly below the diagonal: exp(cs_i - cs_j) = rf * exp(cs_ref - cs_j)
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_base + kColS + cb * 32, r);
-          const float rf = __expf(cs_i - s_cs[cb * 32 + 31]);
-          tmem_ld_wait();
-#pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            const float e0 = __uint_as_float(r[2 * q]) * rf * s_cc[cb * 32 + 2 * q];
-            const float e1 = __uint_as_float(r[2 * q + 1]) * rf * s_cc[cb * 32 + 2 * q + 1];
-            pk[q] = pack_bf16(e0, e1);
-          }
-        } else if (cb == wq) {  // diagonal block: mask first, then exp
+        if (cb <= wq) {
           uint32_t r[32];
           tmem_ld32(tmem + lane_base + kColS + cb * 32, r);
           tmem_ld_wait();
-#pragma unroll
-          for (int q = 0; q < 16; ++q) {
-            float e[2];
-#pragma unroll
-            for (int u = 0; u < 2; ++u) {
-              const int jj = 2 * q + u;  // column within the block; this row is `lane`
-              e[u] = 0.f;
-              if (jj <= lane)
-                e[u] = __uint_as_float(r[jj]) * __expf(cs_i - s_cs[cb * 32 + jj]) * s_dt[cb * 32 + jj];
-            }
-            pk[q] = pack_bf16(e[0], e[1]);
-          }
+          mask_block(cb, r, cs_i, pk);
         } else {  // above the diagonal: zero
 #pragma unroll
           for (int q = 0; q < 16; ++q) pk[q] = 0u;
@@ -362,110 +647,187 @@ __global__ void __launch_bounds__(kThreads, 1)
         tmem_st16(tmem + lane_base + colp + cb * 16, pk);
       }
     }
+    TRACE_MARK(5);
+
+    // ---- scale the left factor's row by exp(cs_i - cs_start), in place in Y
+    if (!wait(kBarYo)) return;
+    tc_fence_after();
+    {
+      const uint64_t carry2 = f2(carry, carry);
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t r[32];
+        tmem_ld32(tmem + lane_base + kColY + hw * 64 + half * 32, r);
+        tmem_ld_wait();
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          float lo, hi;
+          unf2(mul2(carry2, f2u(r[2 * q], r[2 * q + 1])), lo, hi);
+          r[2 * q] = __float_as_uint(lo);
+          r[2 * q + 1] = __float_as_uint(hi);
+        }
+        tmem_st32(tmem + lane_base + kColY + hw * 64 + half * 32, r);
+      }
+    }
     tmem_st_wait();
     tc_fence_before();
-    __syncthreads();
+    warp_arrive(&bars[kBarP]);
+    TRACE_MARK(6);
 
-    // ---- Y_h = P_h x_h, Yo = C [h0 h1]^T, s^T = B^T [w0 x0 | w1 x1]
-    pend_mma = true;
-    if (issuer) {
-      tc_fence_after();
-      const uint32_t a_sx = smem_u32(sx + stage * kHeads * kAtom);
-#pragma unroll
-      for (int hh = 0; hh < kHeads; ++hh) {
-#pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          umma_f16_ta(tmem + kColY + hh * 64, tmem + kColP + hh * 64 + kk * 8,
-                      sdesc_sw128(a_sx + hh * kAtom + kk * 2048, kAtom, 1024), id_y, kk > 0);
-      }
-#pragma unroll
-      for (int kk = 0; kk < NS / 16; ++kk) {
-        const uint32_t koff = (kk >> 2) * kAtom + (kk & 3) * 32;
-        umma_f16(tmem + kColYo, sdesc_sw128(a_sc + koff, 16, 1024),
-                 sdesc_sw128(a_sht + kk * 2048, NS * 128, 1024), id_yo, kk > 0);
-      }
-#pragma unroll
-      for (int kk = 0; kk < kTile / 16; ++kk)
-        umma_f16(tmem + kColSt, sdesc_sw128(a_sb + kk * 2048, lbo_bt, 1024),
-                 sdesc_sw128(a_sxw + kk * 2048, kAtom, 1024), id_st, kk > 0);
-      umma_commit(bar_mma);
-    }
-    ok = mbar_wait_bounded(bar_mma, ph_mma, kWaitLimit);
-    if (__syncthreads_or(!ok)) {
-      ok = false;
-      break;
-    }
-    ph_mma ^= 1;
-    pend_mma = false;
+    // ---- the state after this tile: its bf16 copy for the next tile; at the end of a
+    // piece the final state or the hand-on to the next CTA, then the next piece's state
+    if (!wait(kBarSt)) return;
     tc_fence_after();
-
-    // ---- B and C are free: fetch the next tile's (its x is already on the way)
-    if (have_next && issuer) {
-      fence_proxy_async();
-      issue_bc<NS>(&tm_b, &tm_c, sb, sc, &bar_load[stage ^ 1], pb, nxt);
-    }
-
-    // ---- epilogue: y rows and the state update
     {
-      const float carry = __expf(cs_i - cs_start);
+      const bool piece_done = !have_next || nxt.piece != cur.piece;
+      const bool to_final = piece_done && (cur.flags & kUnitEnd) && pb.final_state && i < NS;
+      const bool to_carry = piece_done && (cur.flags & kCarryOut);
+      float* fp = pb.final_state ? pb.final_state + ((int64_t)s * pb.H + h) * kHeadDim * NS + i : nullptr;
+      float* cp = pb.carry + ((size_t)blockIdx.x * kHeads + hw) * kHeadDim * NS + i;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        uint32_t r[32];
+        tmem_ld32(t_state + half * 32, r);
+        tmem_ld_wait();
+        if (!piece_done) write_ht_from(r, half);
+        if (to_final) {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) fp[(size_t)(half * 32 + q) * NS] = __uint_as_float(r[q]);
+        }
+        if (to_carry && i < NS) {
+#pragma unroll
+          for (int q = 0; q < 32; ++q) cp[(size_t)(half * 32 + q) * NS] = __uint_as_float(r[q]);
+        }
+      }
+      if (to_carry) {  // hand the state on to the CTA whose range continues this unit
+        if (i == 0) pb.carry[(size_t)pb.ranges * kHeads * kHeadDim * NS + blockIdx.x * kHeads + hw] = cs_base;
+        __threadfence();
+        bar_sync(kWGBarrier, kComputeThreads);
+        if (tid == 0) st_release_gpu(&pb.carry_flag[blockIdx.x], 1);
+        __syncwarp();
+      }
+      if (piece_done && have_next) {
+        tc_fence_before();
+        bar_sync(kWGBarrier, kComputeThreads);  // every lane has read the finished state
+        tc_fence_after();
+        if (!load_state(nxt)) return;
+      }
+    }
+    fence_proxy_async();
+    tc_fence_before();
+    warp_arrive(&bars[kBarHt]);
+    TRACE_MARK(7);
+
+    // ---- epilogue: y = Y + D x, staged over this tile's x and stored by TMA
+    if (!wait(kBarY)) return;
+    TRACE_MARK(8);
+    tc_fence_after();
+    {
+      const bool full = rem == kTile;
+      uint8_t* ystage = const_cast<uint8_t*>(sxh);  // each thread overwrites the x chunks it reads
       __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(pb.y) + ((t0 + i) * pb.H + h) * kHeadDim;
 #pragma unroll
       for (int half = 0; half < 2; ++half) {
-        uint32_t ry[32], ro[32];
+        uint32_t ry[32];
         tmem_ld32(tmem + lane_base + kColY + hw * 64 + half * 32, ry);
-        tmem_ld32(tmem + lane_base + kColYo + hw * 64 + half * 32, ro);
         tmem_ld_wait();
 #pragma unroll
         for (int c4 = 0; c4 < 4; ++c4) {
-          const int c = half * 4 + c4;  // 16-byte chunk of the 64-wide row: p = 8c..8c+7
-          const uint4 xv = *reinterpret_cast<const uint4*>(sxh + sw128_off(i, c));
-          const uint32_t* xu = reinterpret_cast<const uint32_t*>(&xv);
+          const int c = half * 4 + c4;
+          const uint32_t o = sw128_off(i, c);
+          const uint4 xv = *reinterpret_cast<const uint4*>(sxh + o);
+          const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
           uint32_t out[4];
 #pragma unroll
           for (int q = 0; q < 4; ++q) {
-            const int e0 = c4 * 8 + 2 * q;
-            const float y0 = __uint_as_float(ry[e0]) + carry * __uint_as_float(ro[e0]) + Dh * bf16_lo(xu[q]);
-            const float y1 = __uint_as_float(ry[e0 + 1]) + carry * __uint_as_float(ro[e0 + 1]) + Dh * bf16_hi(xu[q]);
-            out[q] = pack_bf16(y0, y1);
+            const float x0 = __uint_as_float(xu[q] << 16), x1 = __uint_as_float(xu[q] & 0xFFFF0000u);
+            out[q] = pack_bf16(fmaf(Dh, x0, __uint_as_float(ry[8 * c4 + 2 * q])),
+                               fmaf(Dh, x1, __uint_as_float(ry[8 * c4 + 2 * q + 1])));
           }
-          if (i < rem) *reinterpret_cast<uint4*>(yrow + 8 * c) = make_uint4(out[0], out[1], out[2], out[3]);
+          const uint4 ov = make_uint4(out[0], out[1], out[2], out[3]);
+          if (full)
+            *reinterpret_cast<uint4*>(ystage + o) = ov;
+          else if (i < rem)
+            *reinterpret_cast<uint4*>(yrow + 8 * c) = ov;
         }
       }
-      const float decay = __expf(cs_end - cs_start);
+      tc_fence_before();
+      if (full) fence_proxy_async();
+      bar_sync(kWGBarrier, kComputeThreads);
+      if (full && tid == 0) {
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t rs[32];
-        tmem_ld32(tmem + lane_base + kColSt + hw * 64 + half * 32, rs);
-        tmem_ld_wait();
-#pragma unroll
-        for (int q = 0; q < 32; ++q) hst[half * 32 + q] = fmaf(decay, hst[half * 32 + q], __uint_as_float(rs[q]));
+        for (int hh = 0; hh < kHeads; ++hh)
+          tma_store_3d(tm_y, sx + (stage * kHeads + hh) * kAtom, 0, (cur.unit % pairs) * kHeads + hh, (int)t0);
+        bulk_commit();
       }
+      __syncwarp();
     }
-
-    const bool unit_done = !have_next || nxt.unit != cur.unit;
-    if (unit_done && pb.final_state && i < NS) {
-#pragma unroll
-      for (int p = 0; p < kHeadDim; ++p) pb.final_state[st_base + (int64_t)p * NS + i] = hst[p];
-    }
-    if (unit_done) finish_empty_units(cur.unit + gridDim.x, have_next ? nxt.unit : pb.nseq * (pb.H / kHeads));
-    tc_fence_before();
-    __syncthreads();  // this stage's x and tensor memory are free again
+    warp_arrive(&bars[kBarFree]);
+    TRACE_MARK(9);
+    ++trace_tile;
+    ++tile_idx;
     cur = nxt;
     have = have_next;
     stage ^= 1;
   }
+}
 
-  if (!ok) {
-    // A wait gave up: drain what is still in flight (again bounded), record the failure.
-    for (int k = 0; k < 2; ++k)
-      if (pend_load & (1 << k)) mbar_wait_bounded(&bar_load[k], ph_load[k], kWaitLimit);
-    if (pend_s) mbar_wait_bounded(bar_s, ph_s, kWaitLimit);
-    if (pend_mma) mbar_wait_bounded(bar_mma, ph_mma, kWaitLimit);
-    if (tid == 0) atomicOr(pb.status, kStatusTimeout);
+template <int NS>
+__global__ void __launch_bounds__(kThreads, 1)
+    ssd_fused_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
+                        const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
+                        Problem pb) {
+  using L = Layout<NS>;
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ uint32_t s_tmem_base;
+  const int tid = threadIdx.x, warp = tid >> 5;
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::bars);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::flag);
+
+  if (*pb.nchunks < 0) return;  // cu_seqlens rejected by the table kernel
+
+  if (warp == 0) {
+    tmem_alloc(&s_tmem_base, kTmemCols);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(&bars[kBarLoad0], 1);
+    mbar_init(&bars[kBarLoad1], 1);
+    mbar_init(&bars[kBarS], 1);
+    mbar_init(&bars[kBarYo], 1);
+    mbar_init(&bars[kBarSt], 1);
+    mbar_init(&bars[kBarY], 1);
+    mbar_init(&bars[kBarHt], kComputeWarps);
+    mbar_init(&bars[kBarXw], kComputeWarps);
+    mbar_init(&bars[kBarP], kComputeWarps);
+    mbar_init(&bars[kBarFree], kComputeWarps);
+    mbar_init(&bars[kBarXfree], 1);
+    *abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    prefetch_tensormap(&tm_x);
+    prefetch_tensormap(&tm_b);
+    prefetch_tensormap(&tm_c);
+    prefetch_tensormap(&tm_y);
   }
   tc_fence_before();
   __syncthreads();
-  if (tid < 32) {
+  tc_fence_after();
+  const uint32_t tmem = s_tmem_base;
+
+  if (warp == kComputeThreads / 32) {
+    if ((tid & 31) == 0) issuer_loop<NS>(&tm_x, &tm_b, &tm_c, pb, smem, tmem, bars, abort_flag);
+    __syncwarp();  // the issuer warp reconverges before the CTA-wide barrier
+  } else {
+    compute_loop<NS>(&tm_y, pb, smem, tmem, bars, abort_flag);
+    if (tid == 0) bulk_wait_all();  // y stores complete before the CTA exits
+    __syncwarp();
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (tid == 0 && *abort_flag) atomicOr(pb.status, kStatusTimeout);
+  if (warp == 0) {
     tc_fence_after();
     tmem_dealloc(s_tmem_base, kTmemCols);
   }
@@ -499,25 +861,43 @@ bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, ui
 
 template <int NS>
 cudaError_t launch_ns(const Problem& pb, cudaStream_t st) {
-  CUtensorMap mx, mb, mc;
+  CUtensorMap mx, mb, mc, my;
   const uint64_t tokens = (uint64_t)pb.tokens;
   if (!make_map(&mx, pb.x, kHeadDim, pb.H, tokens) || !make_map(&mb, pb.B, NS, pb.G, tokens) ||
-      !make_map(&mc, pb.C, NS, pb.G, tokens))
+      !make_map(&mc, pb.C, NS, pb.G, tokens) || !make_map(&my, pb.y, kHeadDim, pb.H, tokens))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(ssd_fused_tc_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kDynSmem<NS>);
-  if (e != cudaSuccess) return e;
-  int dev = 0, sms = 0;
-  cudaGetDevice(&dev);
-  cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
-  const int units = pb.nseq * (pb.H / kHeads);
-  const int grid = units < sms ? units : sms;
+  if (e != cudaSuccess) {
+    if (getenv("SSD_DEBUG")) fprintf(stderr, "ssd: smem attribute failed: %s\n", cudaGetErrorString(e));
+    return e;
+  }
+  // One CTA per SM (at most), each on an equal share of the flat tile list; a flat tile
+  // count is not known on the host for packed batches, so the grid covers every SM and
+  // ranges may be empty when there are fewer tiles than SMs.
+  const int grid = pb.ranges;
   if (grid <= 0) return cudaSuccess;
+  e = cudaMemsetAsync(pb.carry_flag, 0, sizeof(int32_t) * (size_t)grid, st);
+  if (e != cudaSuccess) return e;
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = dim3(grid);
+  cfg.blockDim = dim3(kThreads);
+  cfg.dynamicSmemBytes = kDynSmem<NS>;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // all CTAs resident: carry waits always end
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
   if (pb.prof_start) cudaEventRecord(pb.prof_start, st);
-  ssd_fused_tc_kernel<NS><<<grid, kThreads, kDynSmem<NS>, st>>>(mx, mb, mc, pb);
+  e = cudaLaunchKernelEx(&cfg, ssd_fused_tc_kernel<NS>, mx, mb, mc, my, pb);
   if (pb.prof_stop) cudaEventRecord(pb.prof_stop, st);
   count_launches(1);
-  return cudaGetLastError();
+  if (e == cudaSuccess) e = cudaGetLastError();
+  if (e != cudaSuccess && getenv("SSD_DEBUG"))
+    fprintf(stderr, "ssd: fused kernel launch failed: %s (smem %u, threads %d)\n", cudaGetErrorString(e),
+            (unsigned)kDynSmem<NS>, kThreads);
+  return e;
 }
 
 }  // namespace

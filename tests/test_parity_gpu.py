@@ -48,6 +48,10 @@ SMALL = [
     (1, 257, 2, 17, 33, 2, 128, "f32", False),
     (2, 200, 2, 64, 256, 1, 256, "bf16", False),
     (1, 1, 2, 64, 128, 1, 256, "bf16", True),
+    # one long sequence and one head pair: its 64 tiles are spread over many CTAs,
+    # which hand the state on to one another
+    (1, 8192, 2, 64, 128, 1, 256, "bf16", True),
+    (3, 1000, 16, 64, 64, 2, 128, "bf16", True),
 ]
 
 
@@ -69,6 +73,18 @@ def test_small_packed_with_resets(dtype):
     for name, path in paths_for(prob, 128):
         y, fin = run(prob, path=path)
         check(prob, y, fin)
+
+
+def test_packed_many_sequences_grouped():
+    """Many packed sequences of mixed lengths (some shorter than a tile, some empty) with
+    8 heads per B/C group: the flat tile list is cut across CTAs mid-sequence."""
+    rng = np.random.default_rng(9)
+    lens = [int(v) for v in rng.integers(0, 700, 40)]
+    wl = workloads.custom(1, 0, H=16, P=64, N=128, G=2, chunk=256, dtype="bf16", init=True, lengths=lens)
+    prob = workloads.generate(wl, seed=9, lengths=lens)
+    for name, path in paths_for(prob, 256):
+        y, fin = run(prob, path=path)
+        check(prob, y, fin, pairs=sample_pairs(prob, k=12))
 
 
 @pytest.mark.parametrize("Q", [64, 128, 256])
