@@ -66,7 +66,6 @@ constexpr int kHeads = 2;           // heads of one B/C group processed together
 constexpr int kComputeThreads = kHeads * kWGThreads;  // one warpgroup per head
 constexpr int kComputeWarps = kComputeThreads / 32;
 constexpr int kThreads = kComputeThreads + 32;  // + one issuer warp (TMA and UMMA)
-constexpr int kWGBarrier = 1;       // named barrier of the two compute warpgroups
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns: S = C B^T (fp32, 128), P_h (bf16 pairs, 64 per head), Y_h (64 per head;
 // the left factor is written first, row-scaled, then P_h x_h accumulates on top) and
@@ -78,7 +77,7 @@ constexpr uint32_t kSuspendHintNs = 1000;    // a waiting thread sleeps until th
 constexpr uint32_t kAtom = kTile * 128;      // one 128-row x 128-byte swizzled operand column
 
 // mbarriers.  Issuer -> compute: tile loads (tx bytes) and UMMA commits.
-// Compute -> issuer (one arrival per compute warp): ht, xw, p, free; x-free has one arrival.
+// Compute -> issuer (one arrival per compute warp): ht, xw, p, free, x-free.
 enum {
   kBarLoad0 = 0,  // x, B, C of a tile in x stage 0
   kBarLoad1,      // ... stage 1
@@ -90,7 +89,9 @@ enum {
   kBarXw,         // w o x written and the state scaled by this tile's decay
   kBarP,          // P written and Y rows scaled
   kBarFree,       // Y read (the next left factor may overwrite it)
-  kBarXfree,      // a stage's x buffer (which held that tile's y for the TMA store) is reusable
+  kBarXfree,      // a stage's x buffer (which held that tile's y for the TMA stores) is reusable
+  kBarDt0,        // dt of a tile (4 heads x 128 tokens) in dt stage 0
+  kBarDt1,        // ... stage 1
   kNumBars
 };
 
@@ -101,12 +102,13 @@ struct Layout {
   static constexpr uint32_t c = b + (NS / 64) * kAtom;
   static constexpr uint32_t xw = c + (NS / 64) * kAtom;     // [head] [128 tok][64 p]
   static constexpr uint32_t ht = xw + kHeads * kAtom;       // [head] [NS n][64 p]
-  static constexpr uint32_t cs = ht + kHeads * NS * 128;    // float[head][128] in-chunk cumsum (log2 units)
-  static constexpr uint32_t dt = cs + kHeads * kTile * 4;   // float[head][128]
-  static constexpr uint32_t dtn = dt + kHeads * kTile * 4;  // float[2][head][128] prefetched dt
-  static constexpr uint32_t cc = dtn + 2 * kHeads * kTile * 4;  // float[head][128] column factors
-  static constexpr uint32_t red = cc + kHeads * kTile * 4;  // float[warpgroup][4]
-  static constexpr uint32_t bars = red + kHeads * 16;       // uint64[kNumBars]
+  // per compute warp: the tile's in-chunk cumsum (log2 units), column factors, dt, and
+  // the dt prefetch (two buffers)
+  static constexpr uint32_t wcs = ht + kHeads * NS * 128;            // float[warp][128]
+  static constexpr uint32_t wcc = wcs + kComputeWarps * kTile * 4;   // float[warp][128]
+  static constexpr uint32_t wdt = wcc + kComputeWarps * kTile * 4;   // float[warp][128]
+  static constexpr uint32_t sdt = wdt + kComputeWarps * kTile * 4;  // float[stage][128 tok][4 heads]
+  static constexpr uint32_t bars = sdt + 2 * kTile * 16;             // uint64[kNumBars]
   static constexpr uint32_t flag = bars + kNumBars * 8;     // int: a wait gave up
   static constexpr uint32_t bytes = flag + 16;
 };
@@ -244,8 +246,8 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 // ------------------------------------------------------------------ issuer
 template <int NS>
 __device__ void issuer_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, const CUtensorMap* tm_c,
-                            const Problem& pb, uint8_t* smem, uint32_t tmem, uint64_t* bars,
-                            volatile int* abort_flag) {
+                            const CUtensorMap* tm_dt, const Problem& pb, uint8_t* smem, uint32_t tmem,
+                            uint64_t* bars, volatile int* abort_flag) {
   using L = Layout<NS>;
   uint8_t* sx = smem + L::x;
   uint8_t* sb = smem + L::b;
@@ -267,6 +269,14 @@ __device__ void issuer_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, co
 #pragma unroll
     for (int hh = 0; hh < kHeads; ++hh)
       tma_load_3d(sx + (stage * kHeads + hh) * kAtom, tm_x, 0, h0 + hh, c.tb + c.k0, &bars[stage]);
+  };
+  // dt of the tile's 128 tokens for the 4 heads starting at h0 rounded down to 4 (16-byte rows)
+  int dt_issued[2] = {0, 0};  // dt loads per stage (the compute warps wait for them)
+  auto issue_dt = [&](int stage, const TileCursor& c) {
+    ++dt_issued[stage];
+    const int h0 = (c.unit % pairs) * kHeads;
+    mbar_expect_tx(&bars[kBarDt0 + stage], kTile * 16);
+    tma_load_2d(smem + L::sdt + stage * kTile * 16, tm_dt, h0 & ~3, c.tb + c.k0, &bars[kBarDt0 + stage]);
   };
   auto issue_bc = [&](int stage, const TileCursor& c) {
     const int g = ((c.unit % pairs) * kHeads) / pb.hpg;
@@ -291,6 +301,7 @@ __device__ void issuer_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, co
   bool have = cursor_first(pb, rp, cur);
   int stage = 0, t = 0;
   if (have) {
+    issue_dt(0, cur);
     mbar_expect_tx(&bars[kBarLoad0], kLoadBytes);
     issue_x(0, cur);
     issue_bc(0, cur);
@@ -325,6 +336,7 @@ __device__ void issuer_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, co
     if (have_next) {  // the other x stage (tile t-1's x, then its y) is free once its y store read it
       if (t > 0 && !(ok = wait(kBarXfree))) break;
       fence_proxy_async();
+      issue_dt(stage ^ 1, nxt);
       mbar_expect_tx(&bars[stage ^ 1], kLoadBytes);
       issue_x(stage ^ 1, nxt);
       pending |= 1u << (stage ^ 1);
@@ -369,36 +381,41 @@ __device__ void issuer_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, co
     // Drain what this thread issued (again bounded) before tensor memory is freed.
     for (int k = 0; k < kNumBars; ++k)
       if (pending & (1u << k)) mbar_wait_bounded(&bars[k], (phase >> k) & 1u, kWaitLimit);
+    for (int st = 0; st < 2; ++st)  // the last dt load of each stage (its phases complete in order)
+      if (dt_issued[st] > 0) mbar_wait_bounded(&bars[kBarDt0 + st], (dt_issued[st] - 1) & 1, kWaitLimit);
   }
 }
 
 // --------------------------------------------------------- compute warpgroups
-// Two warpgroups, one per head of the pair.  Thread i owns TMEM lane / tile row i.
+// Two warpgroups, one per head of the pair; thread i owns TMEM lane / tile row i.  The
+// warps run free of each other inside a tile: each computes the whole tile's cumsum and
+// column factors into its own shared arrays and stores its own 32 rows of y, so no
+// compute-wide barrier sits in the tile loop.  Every wait is warp-uniform.
 template <int NS>
-__device__ void compute_loop(const CUtensorMap* tm_y, const Problem& pb, uint8_t* smem, uint32_t tmem,
+__device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8_t* smem, uint32_t tmem,
                              uint64_t* bars, volatile int* abort_flag) {
   using L = Layout<NS>;
   const int tid = threadIdx.x;
   const int hw = tid / kWGThreads;       // head of the pair
   const int i = tid % kWGThreads;        // row / TMEM lane
   const int wq = i >> 5, lane = i & 31;  // lane quarter of this warp
+  const int wid = tid >> 5;              // compute warp 0..7
   const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
   uint8_t* sx = smem + L::x;
   uint8_t* sxw = smem + L::xw;
   uint8_t* sht = smem + L::ht;
-  float* s_cs = reinterpret_cast<float*>(smem + L::cs) + hw * kTile;
-  float* s_dt = reinterpret_cast<float*>(smem + L::dt) + hw * kTile;
-  float* s_cc = reinterpret_cast<float*>(smem + L::cc) + hw * kTile;
-  float* s_red = reinterpret_cast<float*>(smem + L::red) + hw * 4;
-  float* s_dtn = reinterpret_cast<float*>(smem + L::dtn) + hw * kTile;  // [buf][head][128]
+  // this warp's copies of the tile's cumsum, column factors and dt, and its dt prefetch
+  float* w_cs = reinterpret_cast<float*>(smem + L::wcs) + wid * kTile;
+  float* w_cc = reinterpret_cast<float*>(smem + L::wcc) + wid * kTile;
+  float* w_dt = reinterpret_cast<float*>(smem + L::wdt) + wid * kTile;
   const int pairs = pb.H / kHeads;
   const int units = pb.nseq * pairs;
 
   uint32_t phase = 0;
-  // Uniform bounded wait of all compute threads on an issuer barrier.
+  // Warp-uniform bounded wait on an issuer barrier.
   auto wait = [&](int k) -> bool {
     const bool mine = wait_or_abort(&bars[k], (phase >> k) & 1u, abort_flag);
-    if (bar_or(kWGBarrier, kComputeThreads, !mine)) return false;
+    if (__any_sync(0xffffffffu, !mine)) return false;
     phase ^= 1u << k;
     return true;
   };
@@ -421,17 +438,17 @@ __device__ void compute_loop(const CUtensorMap* tm_y, const Problem& pb, uint8_t
   // 64 fp32 columns); its bf16 copy in shared memory is the B operand of the left factor.
   const uint32_t t_state = tmem + lane_base + kColSt + hw * 64;
   float cs_base = 0.f;  // in-chunk cumsum (log2 units) before the current tile
-  auto write_ht_from = [&](const uint32_t (&r)[32], int half) {
+  auto write_ht_from = [&](const uint32_t (&r)[64]) {
     if (i < NS) {
       uint8_t* hdst = sht + hw * NS * 128;
 #pragma unroll
-      for (int c4 = 0; c4 < 4; ++c4) {
+      for (int c = 0; c < 8; ++c) {
         uint4 hv;
-        hv.x = bf16x2_of(f2u(r[8 * c4 + 0], r[8 * c4 + 1]));
-        hv.y = bf16x2_of(f2u(r[8 * c4 + 2], r[8 * c4 + 3]));
-        hv.z = bf16x2_of(f2u(r[8 * c4 + 4], r[8 * c4 + 5]));
-        hv.w = bf16x2_of(f2u(r[8 * c4 + 6], r[8 * c4 + 7]));
-        *reinterpret_cast<uint4*>(hdst + sw128_off(i, half * 4 + c4)) = hv;
+        hv.x = bf16x2_of(f2u(r[8 * c + 0], r[8 * c + 1]));
+        hv.y = bf16x2_of(f2u(r[8 * c + 2], r[8 * c + 3]));
+        hv.z = bf16x2_of(f2u(r[8 * c + 4], r[8 * c + 5]));
+        hv.w = bf16x2_of(f2u(r[8 * c + 6], r[8 * c + 7]));
+        *reinterpret_cast<uint4*>(hdst + sw128_off(i, c)) = hv;
       }
     }
   };
@@ -443,9 +460,9 @@ __device__ void compute_loop(const CUtensorMap* tm_y, const Problem& pb, uint8_t
     if (c.flags & kCarryIn) {
       const int src = rp.carry_src;
       bool mine = true;
-      if (tid == 0) {
+      if (lane == 0) {
         const long long t0 = clock64();
-        while (ld_acquire_gpu(&pb.carry_flag[src]) == 0) {
+        while (ld_acquire_gpu(&pb.carry_flag[src]) < kComputeWarps) {
           if (*abort_flag || clock64() - t0 > kWaitLimit) {
             *abort_flag = 1;
             mine = false;
@@ -454,8 +471,7 @@ __device__ void compute_loop(const CUtensorMap* tm_y, const Problem& pb, uint8_t
           __nanosleep(200);
         }
       }
-      __syncwarp();
-      if (bar_or(kWGBarrier, kComputeThreads, !mine)) return false;
+      if (__any_sync(0xffffffffu, !mine)) return false;
       __threadfence();
       src_p = pb.carry + ((size_t)src * kHeads + hw) * kHeadDim * NS + i;
       cs_base = __ldcg(pb.carry + (size_t)pb.ranges * kHeads * kHeadDim * NS + src * kHeads + hw);
@@ -465,35 +481,22 @@ __device__ void compute_loop(const CUtensorMap* tm_y, const Problem& pb, uint8_t
       if (pb.init) src_p = pb.init + ((int64_t)s * pb.H + h) * kHeadDim * NS + i;
       cs_base = 0.f;
     }
+    uint32_t r[64];
 #pragma unroll
-    for (int half = 0; half < 2; ++half) {
-      uint32_t r[32];
-#pragma unroll
-      for (int q = 0; q < 32; ++q)
-        r[q] = __float_as_uint((src_p && i < NS) ? __ldcg(src_p + (size_t)(half * 32 + q) * NS) : 0.f);
-      tmem_st32(t_state + half * 32, r);
-      write_ht_from(r, half);
-    }
+    for (int q = 0; q < 64; ++q) r[q] = __float_as_uint((src_p && i < NS) ? __ldcg(src_p + (size_t)q * NS) : 0.f);
+    tmem_st64(t_state, r);
+    write_ht_from(r);
     tmem_st_wait();
     fence_proxy_async();
     return true;
   };
   auto head_of = [&](const TileCursor& c) { return (c.unit % pairs) * kHeads + hw; };
-  // dt of tile c for this thread's token, copied asynchronously into s_dtn[buf]
-  auto prefetch_dt = [&](const TileCursor& c, int buf) {
-    float* dst = s_dtn + buf * kHeads * kTile + i;
-    if (c.k0 + i < c.len)
-      cp_async4(dst, pb.dt + ((int64_t)c.tb + c.k0 + i) * pb.H + head_of(c));
-    else
-      *dst = 0.f;
-    cp_async_commit();
-  };
   // P values of one 32-column block of S (fp32 bits in r) for row i.
-  auto mask_block = [&](int cb, const uint32_t (&r)[32], float cs_i, uint32_t (&pk)[16]) {
+  auto mask_block = [&](int cb, const uint32_t* r, float cs_i, uint32_t (&pk)[16]) {
     if (cb < wq) {  // strictly below the diagonal: exp(cs_i - cs_j) = rf * exp(cs_ref - cs_j)
-      const float rf = ex2(cs_i - s_cs[cb * 32 + 31]);
+      const float rf = ex2(cs_i - w_cs[cb * 32 + 31]);
       const uint64_t rf2 = f2(rf, rf);
-      const float4* cc4 = reinterpret_cast<const float4*>(s_cc + cb * 32);
+      const float4* cc4 = reinterpret_cast<const float4*>(w_cc + cb * 32);
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4) {
         const float4 c = cc4[q4];
@@ -502,8 +505,8 @@ __device__ void compute_loop(const CUtensorMap* tm_y, const Problem& pb, uint8_t
         pk[2 * q4 + 1] = bf16x2_of(mul2(f1, f2u(r[4 * q4 + 2], r[4 * q4 + 3])));
       }
     } else {  // diagonal block: mask first (-inf), then exp
-      const float4* c4 = reinterpret_cast<const float4*>(s_cs + cb * 32);
-      const float4* d4 = reinterpret_cast<const float4*>(s_dt + cb * 32);
+      const float4* c4 = reinterpret_cast<const float4*>(w_cs + cb * 32);
+      const float4* d4 = reinterpret_cast<const float4*>(w_dt + cb * 32);
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4) {
         const float4 cj = c4[q4], dj = d4[q4];
@@ -524,7 +527,6 @@ __device__ void compute_loop(const CUtensorMap* tm_y, const Problem& pb, uint8_t
   if (!load_state(cur)) return;
   tc_fence_before();
   warp_arrive(&bars[kBarHt]);
-  prefetch_dt(cur, 0);
   float a2_cur = pb.A[head_of(cur)] * 1.4426950408889634f;  // A_h log2(e): cumsums are in log2 units
   float d_cur = pb.D ? pb.D[head_of(cur)] : 0.f;
   int stage = 0, tile_idx = 0;
@@ -543,42 +545,69 @@ __device__ void compute_loop(const CUtensorMap* tm_y, const Problem& pb, uint8_t
     // look ahead: next tile's dt (and its head's parameters at a unit change)
     TileCursor nxt = cur;
     const bool have_next = cursor_next(pb, rp, nxt);
-    cp_async_wait_all();  // this tile's dt (each thread reads back its own copy)
-    const float dtj = s_dtn[(tile_idx & 1) * kHeads * kTile + i];
+    TRACE_MARK(10);
+    if (!wait(kBarDt0 + stage)) return;  // this tile's dt (the issuer loaded it a tile ahead)
+    TRACE_MARK(11);
+    float4 d4;  // dt of tokens 4 lane .. 4 lane + 3 (0 past the end of the sequence)
+    {
+      // Row 4 lane + j holds the 4 heads' dt of one token.  Lane reads its rows in the
+      // order j = (k + rot) & 3, rot = (lane / 2) & 3, so each quarter warp's 16-byte
+      // loads fall in distinct banks; then the rows go back in order and the head is picked.
+      const float4* rows = reinterpret_cast<const float4*>(smem + L::sdt + stage * kTile * 16) + 4 * lane;
+      const int rot = (lane >> 1) & 3, hh = h & 3;
+      float v[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float4 q = rows[(k + rot) & 3];
+        v[k] = hh == 0 ? q.x : hh == 1 ? q.y : hh == 2 ? q.z : q.w;
+      }
+      float dj[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {  // token j came in as k = (j - rot) & 3
+        const int k = (j - rot) & 3;
+        dj[j] = k == 0 ? v[0] : k == 1 ? v[1] : k == 2 ? v[2] : v[3];
+      }
+      const int left = cur.len - cur.k0 - 4 * lane;
+      d4.x = 0 < left ? dj[0] : 0.f;
+      d4.y = 1 < left ? dj[1] : 0.f;
+      d4.z = 2 < left ? dj[2] : 0.f;
+      d4.w = 3 < left ? dj[3] : 0.f;
+    }
     if (have_next) {
-      prefetch_dt(nxt, (tile_idx & 1) ^ 1);
       if (nxt.unit != cur.unit) {
         a2_cur = pb.A[head_of(nxt)] * 1.4426950408889634f;
         d_cur = pb.D ? pb.D[head_of(nxt)] : 0.f;
       }
     }
 
-    // ---- in-chunk cumsum of dt*A (log2 units)
-    float v = dtj * Ah2;
+    // ---- in-chunk cumsum of dt*A over the whole tile, by every warp (log2 units)
+    float c0 = d4.x * Ah2, c1 = c0 + d4.y * Ah2, c2 = c1 + d4.z * Ah2, c3 = c2 + d4.w * Ah2;
+    float v = c3;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const float u = __shfl_up_sync(0xffffffffu, v, o);
       if (lane >= o) v += u;
     }
-    if (lane == 31) s_red[wq] = v;
-    bar_sync(kWGBarrier, kComputeThreads);
-    float off = cs_base;
-    for (int w = 0; w < wq; ++w) off += s_red[w];
-    const float cs_i = off + v;
-    s_cs[i] = cs_i;
-    bar_sync(kWGBarrier, kComputeThreads);
+    const float base = cs_base + v - c3;  // cumsum before token 4 lane
+    c0 += base, c1 += base, c2 += base, c3 += base;
+    reinterpret_cast<float4*>(w_cs)[lane] = make_float4(c0, c1, c2, c3);
+    reinterpret_cast<float4*>(w_dt)[lane] = d4;
+    // block ends (tokens 31, 63, 95, 127) live in lanes 7, 15, 23, 31
+    const float ref = __shfl_sync(0xffffffffu, c3, (lane & ~7) | 7);  // end of this lane's 32-block
+    reinterpret_cast<float4*>(w_cc)[lane] =
+        make_float4(ex2(ref - c0) * d4.x, ex2(ref - c1) * d4.y, ex2(ref - c2) * d4.z, ex2(ref - c3) * d4.w);
+    TRACE_MARK(12);
+    const float cs_end = __shfl_sync(0xffffffffu, c3, 31);  // tokens past the end add 0
     const float cs_start = cs_base;
-    const float cs_end = s_cs[kTile - 1];  // tokens past the end add 0
     cs_base = cs_end;
-    // column factor for blocks below the diagonal: exp(cs_ref - cs_i) dt_i, with cs_ref
-    // the cumsum at the end of i's 32-token block
-    s_cc[i] = ex2(s_cs[wq * 32 + 31] - cs_i) * dtj;
-    s_dt[i] = dtj;
+    __syncwarp();
+    const float cs_i = w_cs[i];
+    const float dtj = w_dt[i];
     const float w_i = ex2(cs_end - cs_i) * dtj;  // right-factor weight (0 past the end)
     const float carry = ex2(cs_i - cs_start);    // decay of the carried-in state to token i
     TRACE_MARK(1);
 
-    // ---- this tile's x: w o x, the right-factor input
+    // ---- this tile's x: w o x, the right-factor input; the state scaled by this tile's decay
     if (!wait(stage)) return;
     TRACE_MARK(2);
     const uint8_t* sxh = sx + (stage * kHeads + hw) * kAtom;
@@ -597,54 +626,56 @@ __device__ void compute_loop(const CUtensorMap* tm_y, const Problem& pb, uint8_t
       }
     }
     fence_proxy_async();
-    {  // state scaled by this tile's decay; the right-factor MMA then accumulates onto it
+    {
       const float decay = ex2(cs_end - cs_start);
       const uint64_t decay2 = f2(decay, decay);
+      uint32_t r[64];
+      tmem_ld64(t_state, r);
+      tmem_ld_wait();
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t r[32];
-        tmem_ld32(t_state + half * 32, r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          float lo, hi;
-          unf2(mul2(decay2, f2u(r[2 * q], r[2 * q + 1])), lo, hi);
-          r[2 * q] = __float_as_uint(lo);
-          r[2 * q + 1] = __float_as_uint(hi);
-        }
-        tmem_st32(t_state + half * 32, r);
+      for (int q = 0; q < 32; ++q) {
+        float lo, hi;
+        unf2(mul2(decay2, f2u(r[2 * q], r[2 * q + 1])), lo, hi);
+        r[2 * q] = __float_as_uint(lo);
+        r[2 * q + 1] = __float_as_uint(hi);
       }
+      tmem_st64(t_state, r);
       tmem_st_wait();
       tc_fence_before();
     }
     warp_arrive(&bars[kBarXw]);
-    if (tid == 0 && tile_idx > 0) {
-  // the previous tile's y store has read its x stage: release it
-      bulk_wait_read();
-      mbar_arrive(&bars[kBarXfree]);
+    if (tile_idx > 0) {  // this warp's y store of the previous tile has read its x stage: release it
+      if (lane == 0) bulk_wait_read();
+      warp_arrive(&bars[kBarXfree]);
     }
-    __syncwarp();
     TRACE_MARK(3);
 
-    // ---- P_h = mask_h(S), bf16 pairs in tensor memory; S blocks loaded two at a time
+    // ---- P_h = mask_h(S), bf16 pairs in tensor memory
     if (!wait(kBarS)) return;
     TRACE_MARK(4);
     tc_fence_after();
     {
       const uint32_t colp = kColP + hw * 64;
 #pragma unroll 1
-      for (int cb = 0; cb < 4; ++cb) {  // 32-column blocks of S -> P columns 16cb..16cb+15
-        uint32_t pk[16];
+      for (int cb = 0; cb < 4; cb += 2) {  // blocks cb, cb + 1 (64 columns of S) -> P columns 16cb..16cb+31
+        uint32_t pk0[16], pk1[16];
         if (cb <= wq) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_base + kColS + cb * 32, r);
+          uint32_t r[64];
+          tmem_ld64(tmem + lane_base + kColS + cb * 32, r);
           tmem_ld_wait();
-          mask_block(cb, r, cs_i, pk);
+          mask_block(cb, r, cs_i, pk0);
+          if (cb + 1 <= wq) {
+            mask_block(cb + 1, r + 32, cs_i, pk1);
+          } else {
+#pragma unroll
+            for (int q = 0; q < 16; ++q) pk1[q] = 0u;
+          }
         } else {  // above the diagonal: zero
 #pragma unroll
-          for (int q = 0; q < 16; ++q) pk[q] = 0u;
+          for (int q = 0; q < 16; ++q) pk0[q] = pk1[q] = 0u;
         }
-        tmem_st16(tmem + lane_base + colp + cb * 16, pk);
+        tmem_st16(tmem + lane_base + colp + cb * 16, pk0);
+        tmem_st16(tmem + lane_base + colp + (cb + 1) * 16, pk1);
       }
     }
     TRACE_MARK(5);
@@ -654,20 +685,17 @@ __device__ void compute_loop(const CUtensorMap* tm_y, const Problem& pb, uint8_t
     tc_fence_after();
     {
       const uint64_t carry2 = f2(carry, carry);
+      uint32_t r[64];
+      tmem_ld64(tmem + lane_base + kColY + hw * 64, r);
+      tmem_ld_wait();
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t r[32];
-        tmem_ld32(tmem + lane_base + kColY + hw * 64 + half * 32, r);
-        tmem_ld_wait();
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          float lo, hi;
-          unf2(mul2(carry2, f2u(r[2 * q], r[2 * q + 1])), lo, hi);
-          r[2 * q] = __float_as_uint(lo);
-          r[2 * q + 1] = __float_as_uint(hi);
-        }
-        tmem_st32(tmem + lane_base + kColY + hw * 64 + half * 32, r);
+      for (int q = 0; q < 32; ++q) {
+        float lo, hi;
+        unf2(mul2(carry2, f2u(r[2 * q], r[2 * q + 1])), lo, hi);
+        r[2 * q] = __float_as_uint(lo);
+        r[2 * q + 1] = __float_as_uint(hi);
       }
+      tmem_st64(tmem + lane_base + kColY + hw * 64, r);
     }
     tmem_st_wait();
     tc_fence_before();
@@ -684,80 +712,68 @@ __device__ void compute_loop(const CUtensorMap* tm_y, const Problem& pb, uint8_t
       const bool to_carry = piece_done && (cur.flags & kCarryOut);
       float* fp = pb.final_state ? pb.final_state + ((int64_t)s * pb.H + h) * kHeadDim * NS + i : nullptr;
       float* cp = pb.carry + ((size_t)blockIdx.x * kHeads + hw) * kHeadDim * NS + i;
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t r[32];
-        tmem_ld32(t_state + half * 32, r);
+      {
+        uint32_t r[64];
+        tmem_ld64(t_state, r);
         tmem_ld_wait();
-        if (!piece_done) write_ht_from(r, half);
+        if (!piece_done) write_ht_from(r);
         if (to_final) {
 #pragma unroll
-          for (int q = 0; q < 32; ++q) fp[(size_t)(half * 32 + q) * NS] = __uint_as_float(r[q]);
+          for (int q = 0; q < 64; ++q) fp[(size_t)q * NS] = __uint_as_float(r[q]);
         }
         if (to_carry && i < NS) {
 #pragma unroll
-          for (int q = 0; q < 32; ++q) cp[(size_t)(half * 32 + q) * NS] = __uint_as_float(r[q]);
+          for (int q = 0; q < 64; ++q) cp[(size_t)q * NS] = __uint_as_float(r[q]);
         }
       }
-      if (to_carry) {  // hand the state on to the CTA whose range continues this unit
+      if (to_carry) {  // hand the state on: one release increment per warp once its part is out
         if (i == 0) pb.carry[(size_t)pb.ranges * kHeads * kHeadDim * NS + blockIdx.x * kHeads + hw] = cs_base;
         __threadfence();
-        bar_sync(kWGBarrier, kComputeThreads);
-        if (tid == 0) st_release_gpu(&pb.carry_flag[blockIdx.x], 1);
+        __syncwarp();
+        if (lane == 0) red_add_release_gpu(&pb.carry_flag[blockIdx.x], 1);
         __syncwarp();
       }
-      if (piece_done && have_next) {
-        tc_fence_before();
-        bar_sync(kWGBarrier, kComputeThreads);  // every lane has read the finished state
-        tc_fence_after();
-        if (!load_state(nxt)) return;
-      }
+      if (piece_done && have_next && !load_state(nxt)) return;
     }
     fence_proxy_async();
     tc_fence_before();
     warp_arrive(&bars[kBarHt]);
     TRACE_MARK(7);
 
-    // ---- epilogue: y = Y + D x, staged over this tile's x and stored by TMA
+    // ---- epilogue: y = Y + D x, staged over this tile's x; each warp stores its 32 rows by TMA
     if (!wait(kBarY)) return;
     TRACE_MARK(8);
     tc_fence_after();
     {
-      const bool full = rem == kTile;
+      const bool full = cur.k0 + 32 * wq + 32 <= cur.len;  // all 32 rows of this warp are in the sequence
       uint8_t* ystage = const_cast<uint8_t*>(sxh);  // each thread overwrites the x chunks it reads
       __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(pb.y) + ((t0 + i) * pb.H + h) * kHeadDim;
+      uint32_t ry[64];
+      tmem_ld64(tmem + lane_base + kColY + hw * 64, ry);
+      tmem_ld_wait();
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        uint32_t ry[32];
-        tmem_ld32(tmem + lane_base + kColY + hw * 64 + half * 32, ry);
-        tmem_ld_wait();
+      for (int c = 0; c < 8; ++c) {
+        const uint32_t o = sw128_off(i, c);
+        const uint4 xv = *reinterpret_cast<const uint4*>(sxh + o);
+        const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
+        uint32_t out[4];
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          const int c = half * 4 + c4;
-          const uint32_t o = sw128_off(i, c);
-          const uint4 xv = *reinterpret_cast<const uint4*>(sxh + o);
-          const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
-          uint32_t out[4];
-#pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const float x0 = __uint_as_float(xu[q] << 16), x1 = __uint_as_float(xu[q] & 0xFFFF0000u);
-            out[q] = pack_bf16(fmaf(Dh, x0, __uint_as_float(ry[8 * c4 + 2 * q])),
-                               fmaf(Dh, x1, __uint_as_float(ry[8 * c4 + 2 * q + 1])));
-          }
-          const uint4 ov = make_uint4(out[0], out[1], out[2], out[3]);
-          if (full)
-            *reinterpret_cast<uint4*>(ystage + o) = ov;
-          else if (i < rem)
-            *reinterpret_cast<uint4*>(yrow + 8 * c) = ov;
+        for (int q = 0; q < 4; ++q) {
+          const float x0 = __uint_as_float(xu[q] << 16), x1 = __uint_as_float(xu[q] & 0xFFFF0000u);
+          out[q] = pack_bf16(fmaf(Dh, x0, __uint_as_float(ry[8 * c + 2 * q])),
+                             fmaf(Dh, x1, __uint_as_float(ry[8 * c + 2 * q + 1])));
         }
+        const uint4 ov = make_uint4(out[0], out[1], out[2], out[3]);
+        if (full)
+          *reinterpret_cast<uint4*>(ystage + o) = ov;
+        else if (i < rem)
+          *reinterpret_cast<uint4*>(yrow + 8 * c) = ov;
       }
       tc_fence_before();
       if (full) fence_proxy_async();
-      bar_sync(kWGBarrier, kComputeThreads);
-      if (full && tid == 0) {
-#pragma unroll
-        for (int hh = 0; hh < kHeads; ++hh)
-          tma_store_3d(tm_y, sx + (stage * kHeads + hh) * kAtom, 0, (cur.unit % pairs) * kHeads + hh, (int)t0);
+      __syncwarp();
+      if (full && lane == 0) {
+        tma_store_3d(tm_y32, ystage + wq * 32 * 128, 0, h, (int)(t0 + 32 * wq));
         bulk_commit();
       }
       __syncwarp();
@@ -775,8 +791,8 @@ __device__ void compute_loop(const CUtensorMap* tm_y, const Problem& pb, uint8_t
 template <int NS>
 __global__ void __launch_bounds__(kThreads, 1)
     ssd_fused_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
-                        const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y,
-                        Problem pb) {
+                        const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y32,
+                        const __grid_constant__ CUtensorMap tm_dt, Problem pb) {
   using L = Layout<NS>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem_base;
@@ -802,13 +818,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars[kBarXw], kComputeWarps);
     mbar_init(&bars[kBarP], kComputeWarps);
     mbar_init(&bars[kBarFree], kComputeWarps);
-    mbar_init(&bars[kBarXfree], 1);
+    mbar_init(&bars[kBarXfree], kComputeWarps);
+    mbar_init(&bars[kBarDt0], 1);
+    mbar_init(&bars[kBarDt1], 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tensormap(&tm_x);
     prefetch_tensormap(&tm_b);
     prefetch_tensormap(&tm_c);
-    prefetch_tensormap(&tm_y);
+    prefetch_tensormap(&tm_y32);
+    prefetch_tensormap(&tm_dt);
   }
   tc_fence_before();
   __syncthreads();
@@ -816,11 +835,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s_tmem_base;
 
   if (warp == kComputeThreads / 32) {
-    if ((tid & 31) == 0) issuer_loop<NS>(&tm_x, &tm_b, &tm_c, pb, smem, tmem, bars, abort_flag);
+    if ((tid & 31) == 0) issuer_loop<NS>(&tm_x, &tm_b, &tm_c, &tm_dt, pb, smem, tmem, bars, abort_flag);
     __syncwarp();  // the issuer warp reconverges before the CTA-wide barrier
   } else {
-    compute_loop<NS>(&tm_y, pb, smem, tmem, bars, abort_flag);
-    if (tid == 0) bulk_wait_all();  // y stores complete before the CTA exits
+    compute_loop<NS>(&tm_y32, pb, smem, tmem, bars, abort_flag);
+    if ((tid & 31) == 0) bulk_wait_all();  // this warp's y stores complete before the CTA exits
     __syncwarp();
   }
 
@@ -846,25 +865,40 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
-// 3-D bf16 map {inner, mid, tokens} with a {64, 1, 128} box and 128-byte swizzle.
-bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t tokens) {
+// 3-D bf16 map {inner, mid, tokens} with a {64, 1, rows} box and 128-byte swizzle.
+bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t tokens,
+              uint32_t rows = kTile) {
   auto fn = encode_fn();
   if (!fn) return false;
   cuuint64_t dims[3] = {inner, mid, tokens};
   cuuint64_t strides[2] = {inner * 2, inner * mid * 2};
-  cuuint32_t box[3] = {64, 1, (cuuint32_t)kTile};
+  cuuint32_t box[3] = {64, 1, rows};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D fp32 map of dt {H, tokens} with a {4 heads, 128 tokens} box (16-byte rows, no swizzle).
+bool make_dt_map(CUtensorMap* m, const float* dt, uint64_t H, uint64_t tokens) {
+  auto fn = encode_fn();
+  if (!fn) return false;
+  cuuint64_t dims[2] = {H, tokens};
+  cuuint64_t strides[1] = {H * 4};
+  cuuint32_t box[2] = {4, (cuuint32_t)kTile};
+  cuuint32_t estr[2] = {1, 1};
+  return fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<float*>(dt), dims, strides, box, estr,
+            CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_128B,
+            CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 template <int NS>
 cudaError_t launch_ns(const Problem& pb, cudaStream_t st) {
-  CUtensorMap mx, mb, mc, my;
+  CUtensorMap mx, mb, mc, my, mdt;
   const uint64_t tokens = (uint64_t)pb.tokens;
   if (!make_map(&mx, pb.x, kHeadDim, pb.H, tokens) || !make_map(&mb, pb.B, NS, pb.G, tokens) ||
-      !make_map(&mc, pb.C, NS, pb.G, tokens) || !make_map(&my, pb.y, kHeadDim, pb.H, tokens))
+      !make_map(&mc, pb.C, NS, pb.G, tokens) || !make_map(&my, pb.y, kHeadDim, pb.H, tokens, 32) ||
+      !make_dt_map(&mdt, pb.dt, pb.H, tokens))
     return cudaErrorInvalidValue;
   cudaError_t e = cudaFuncSetAttribute(ssd_fused_tc_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)kDynSmem<NS>);
@@ -890,7 +924,7 @@ cudaError_t launch_ns(const Problem& pb, cudaStream_t st) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (pb.prof_start) cudaEventRecord(pb.prof_start, st);
-  e = cudaLaunchKernelEx(&cfg, ssd_fused_tc_kernel<NS>, mx, mb, mc, my, pb);
+  e = cudaLaunchKernelEx(&cfg, ssd_fused_tc_kernel<NS>, mx, mb, mc, my, mdt, pb);
   if (pb.prof_stop) cudaEventRecord(pb.prof_stop, st);
   count_launches(1);
   if (e == cudaSuccess) e = cudaGetLastError();
@@ -906,6 +940,7 @@ bool tc_supports(const ssd_shape* s, int chunk) {
   if (!s || s->io_dtype != SSD_BF16 || s->headdim != kHeadDim) return false;
   if (s->dstate != 64 && s->dstate != 128) return false;
   if (s->nheads % kHeads || (s->nheads / s->ngroups) % kHeads) return false;  // head pairs share a group
+  if (s->nheads % 4) return false;  // dt rows of 4 heads (16 bytes) per TMA box
   if (chunk != 128 && chunk != 256) return false;
   const int64_t tokens = s->batch * s->seqlen;
   return tokens >= 1 && tokens < ((int64_t)1 << 31) - kTile;

@@ -47,10 +47,11 @@ SMALL = [
     (2, 300, 4, 32, 16, 4, 64, "f32", True),
     (1, 257, 2, 17, 33, 2, 128, "f32", False),
     (2, 200, 2, 64, 256, 1, 256, "bf16", False),
-    (1, 1, 2, 64, 128, 1, 256, "bf16", True),
-    # one long sequence and one head pair: its 64 tiles are spread over many CTAs,
+    (1, 1, 4, 64, 128, 1, 256, "bf16", True),
+    # one long sequence and two head pairs: their 128 tiles are spread over many CTAs,
     # which hand the state on to one another
-    (1, 8192, 2, 64, 128, 1, 256, "bf16", True),
+    (1, 8192, 4, 64, 128, 1, 256, "bf16", True),
+    (1, 2048, 2, 64, 128, 1, 256, "bf16", True),  # 2 heads: no 4-head dt rows, SIMT path
     (3, 1000, 16, 64, 64, 2, 128, "bf16", True),
 ]
 
@@ -107,7 +108,7 @@ def test_tiny_dt_and_strong_decay():
 
 
 def test_no_skip_no_init_no_final():
-    wl = workloads.custom(1, 300, H=2, P=64, N=64, G=1, chunk=128, dtype="bf16")
+    wl = workloads.custom(1, 300, H=4, P=64, N=64, G=1, chunk=128, dtype="bf16")
     prob = workloads.generate(wl, seed=5)
     prob.D = None
     for name, path in paths_for(prob, 128):
@@ -138,13 +139,13 @@ def test_host_entry_point_matches_device():
 
 
 def test_bad_device_seqlens_sets_status_and_writes_nothing():
-    wl = workloads.custom(1, 300, H=2, P=64, N=64, G=1, chunk=128, dtype="bf16", lengths=[100, 200])
+    wl = workloads.custom(1, 300, H=4, P=64, N=64, G=1, chunk=128, dtype="bf16", lengths=[100, 200])
     prob = workloads.generate(wl, seed=8, lengths=[100, 200])
     dev = to_device(prob)
     dev["cu_seqlens"] = torch.tensor([0, 250, 200], dtype=torch.int32, device="cuda")  # not monotone
     assert ssd.query_status() == 0
     y = torch.full_like(dev["x"], 7.0)
-    fin = torch.full((2, 2, 64, 64), 7.0, device="cuda")
+    fin = torch.full((2, 4, 64, 64), 7.0, device="cuda")
     ssd.ssd_forward(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], None, dev["cu_seqlens"], 128,
                     y=y, final_state=fin)
     assert ssd.query_status() == 6
