@@ -34,19 +34,27 @@
 #endif
 #if SSD_TRACE
 namespace ssd {
-constexpr int kTraceCtas = 4, kTraceTiles = 64, kTraceMarks = 16;
-__device__ unsigned long long g_trace[2 * kTraceCtas * kTraceTiles * kTraceMarks];
+constexpr int kTraceCtas = 4, kTraceTiles = 64, kTraceMarks = 24;
+__device__ unsigned long long g_trace[3 * kTraceCtas * kTraceTiles * kTraceMarks];
 }  // namespace ssd
 extern "C" int ssd_trace_dump(unsigned long long* host, int n) {
   return (int)cudaMemcpyFromSymbol(host, ssd::g_trace, sizeof(unsigned long long) * n);
 }
 #define TRACE_MARK(m)                                                                              \
   do {                                                                                             \
-    if ((tid == 0 || tid == 128) && blockIdx.x < kTraceCtas && trace_tile < kTraceTiles)           \
-      g_trace[(((tid >> 7) * kTraceCtas + blockIdx.x) * kTraceTiles + trace_tile) * kTraceMarks + \
+    if ((tid == 0 || tid == 96) && blockIdx.x < kTraceCtas && trace_tile < kTraceTiles)            \
+      g_trace[(((tid != 0) * kTraceCtas + blockIdx.x) * kTraceTiles + trace_tile) * kTraceMarks +  \
               (m)] = clock64();                                                                    \
   } while (0)
+#define TRACE_ISSUE(m)                                                                             \
+  do {                                                                                             \
+    if (blockIdx.x < kTraceCtas && t < kTraceTiles)                                                \
+      g_trace[((2 * kTraceCtas + blockIdx.x) * kTraceTiles + t) * kTraceMarks + (m)] = clock64();  \
+  } while (0)
 #else
+#define TRACE_ISSUE(m) \
+  do {                 \
+  } while (0)
 #define TRACE_MARK(m) \
   do {                \
   } while (0)
@@ -63,9 +71,13 @@ constexpr int kTile = 128;          // tokens per tile (UMMA M)
 constexpr int kHeadDim = 64;        // P supported by this path
 constexpr int kWGThreads = 128;     // a warpgroup: thread i <-> TMEM lane i
 constexpr int kHeads = 2;           // heads of one B/C group processed together
-constexpr int kComputeThreads = kHeads * kWGThreads;  // one warpgroup per head
+constexpr int kHalves = 2;          // each head's Y and state columns split over two warpgroups
+constexpr int kComputeThreads = kHeads * kHalves * kWGThreads;
 constexpr int kComputeWarps = kComputeThreads / 32;
-constexpr int kThreads = kComputeThreads + 32;  // + one issuer warp (TMA and UMMA)
+constexpr int kThreads = kComputeThreads + 64;  // + the issuer warp (TMA and UMMA) and the helper warp
+constexpr int kIssuerWarp = kComputeWarps, kHelperWarp = kComputeWarps + 1;
+constexpr int kDescSlots = 2;  // tile descriptors the helper warp may run ahead
+constexpr int kDtStages = 4;   // dt tiles in flight
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns: S = C B^T (fp32, 128), P_h (bf16 pairs, 64 per head), Y_h (64 per head;
 // the left factor is written first, row-scaled, then P_h x_h accumulates on top) and
@@ -78,6 +90,7 @@ constexpr uint32_t kAtom = kTile * 128;      // one 128-row x 128-byte swizzled 
 
 // mbarriers.  Issuer -> compute: tile loads (tx bytes) and UMMA commits.
 // Compute -> issuer (one arrival per compute warp): ht, xw, p, free, x-free.
+// Helper -> compute: a tile descriptor is written; compute -> helper: it was used up.
 enum {
   kBarLoad0 = 0,  // x, B, C of a tile in x stage 0
   kBarLoad1,      // ... stage 1
@@ -90,10 +103,40 @@ enum {
   kBarP,          // P written and Y rows scaled
   kBarFree,       // Y read (the next left factor may overwrite it)
   kBarXfree,      // a stage's x buffer (which held that tile's y for the TMA stores) is reusable
-  kBarDt0,        // dt of a tile (4 heads x 128 tokens) in dt stage 0
-  kBarDt1,        // ... stage 1
-  kNumBars
+  kBarDt0,        // kDtStages barriers: dt of a tile (4 heads x 128 tokens) in that stage
+  kBarDescFull0 = kBarDt0 + kDtStages,  // kDescSlots barriers: descriptor written
+  kBarDescFree0 = kBarDescFull0 + kDescSlots,  // kDescSlots barriers: descriptor used up
+  kBarPair0 = kBarDescFree0 + kDescSlots,  // 8 barriers: the column-half-1 warp of a row quarter staged its y
+  kNumBars = kBarPair0 + kHeads * 4
 };
+
+// One tile as the helper warp lays it out for the compute warps: where it is, what to do
+// with the state around it, and per head the in-chunk cumsum of dt A (log2 units), the
+// 32-block column factors exp(cs(block end) - cs_j) dt_j, and dt.
+enum {
+  kDescFirst = 1,    // first tile of a piece: load the state (initial or handed on) before it
+  kDescCarryIn = 2,  // ... from the carry of CTA carry_src
+  kDescToFinal = 4,  // last tile of a unit: the state after it is the final state
+  kDescToCarry = 8,  // last tile of a range that ends inside a unit: hand the state on
+  kDescEnd = 16      // no tile: the range is done
+};
+struct TileDesc {
+  int t0;         // token index of row 0
+  int rem;        // rows of the tile inside the sequence (1..128)
+  int s;          // sequence
+  int h0;         // first head of the pair
+  int flags;
+  int carry_src;
+  int pad[2];
+  float cs_start[kHeads];  // cumsum before row 0
+  float cs_end[kHeads];    // cumsum after the last row (rows past the end add 0)
+  float decay[kHeads];     // exp2(cs_end - cs_start)
+  float dskip[kHeads];     // D
+  float cs[kHeads][kTile];
+  float cc[kHeads][kTile];
+  float dtv[kHeads][kTile];  // 0 past the end of the sequence
+};
+constexpr uint32_t kDescBytes = (sizeof(TileDesc) + 127) / 128 * 128;
 
 template <int NS>
 struct Layout {
@@ -102,18 +145,16 @@ struct Layout {
   static constexpr uint32_t c = b + (NS / 64) * kAtom;
   static constexpr uint32_t xw = c + (NS / 64) * kAtom;     // [head] [128 tok][64 p]
   static constexpr uint32_t ht = xw + kHeads * kAtom;       // [head] [NS n][64 p]
-  // per compute warp: the tile's in-chunk cumsum (log2 units), column factors, dt, and
-  // the dt prefetch (two buffers)
-  static constexpr uint32_t wcs = ht + kHeads * NS * 128;            // float[warp][128]
-  static constexpr uint32_t wcc = wcs + kComputeWarps * kTile * 4;   // float[warp][128]
-  static constexpr uint32_t wdt = wcc + kComputeWarps * kTile * 4;   // float[warp][128]
-  static constexpr uint32_t sdt = wdt + kComputeWarps * kTile * 4;  // float[stage][128 tok][4 heads]
-  static constexpr uint32_t bars = sdt + 2 * kTile * 16;             // uint64[kNumBars]
+  static constexpr uint32_t desc = ht + kHeads * NS * 128;           // TileDesc[kDescSlots]
+  static constexpr uint32_t sdt = desc + kDescSlots * kDescBytes;    // float[stage][128 tok][4 heads]
+  static constexpr uint32_t bars = sdt + kDtStages * kTile * 16;     // uint64[kNumBars]
   static constexpr uint32_t flag = bars + kNumBars * 8;     // int: a wait gave up
   static constexpr uint32_t bytes = flag + 16;
 };
 template <int NS>
 constexpr uint32_t kDynSmem = Layout<NS>::bytes + 1024;  // + base alignment slack
+static_assert(kDynSmem<128> <= 227 * 1024, "shared memory per CTA");
+static_assert(kNumBars <= 32, "phase bits of a 32-bit mask");
 
 // Work split.  The tiles of all units (sequence, head pair), unit by unit and each
 // unit's 128-token tiles in order, form one flat list; CTA r takes the contiguous
@@ -246,8 +287,8 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
 // ------------------------------------------------------------------ issuer
 template <int NS>
 __device__ void issuer_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, const CUtensorMap* tm_c,
-                            const CUtensorMap* tm_dt, const Problem& pb, uint8_t* smem, uint32_t tmem,
-                            uint64_t* bars, volatile int* abort_flag) {
+                            const Problem& pb, uint8_t* smem, uint32_t tmem, uint64_t* bars,
+                            volatile int* abort_flag) {
   using L = Layout<NS>;
   uint8_t* sx = smem + L::x;
   uint8_t* sb = smem + L::b;
@@ -269,14 +310,6 @@ __device__ void issuer_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, co
 #pragma unroll
     for (int hh = 0; hh < kHeads; ++hh)
       tma_load_3d(sx + (stage * kHeads + hh) * kAtom, tm_x, 0, h0 + hh, c.tb + c.k0, &bars[stage]);
-  };
-  // dt of the tile's 128 tokens for the 4 heads starting at h0 rounded down to 4 (16-byte rows)
-  int dt_issued[2] = {0, 0};  // dt loads per stage (the compute warps wait for them)
-  auto issue_dt = [&](int stage, const TileCursor& c) {
-    ++dt_issued[stage];
-    const int h0 = (c.unit % pairs) * kHeads;
-    mbar_expect_tx(&bars[kBarDt0 + stage], kTile * 16);
-    tma_load_2d(smem + L::sdt + stage * kTile * 16, tm_dt, h0 & ~3, c.tb + c.k0, &bars[kBarDt0 + stage]);
   };
   auto issue_bc = [&](int stage, const TileCursor& c) {
     const int g = ((c.unit % pairs) * kHeads) / pb.hpg;
@@ -301,7 +334,6 @@ __device__ void issuer_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, co
   bool have = cursor_first(pb, rp, cur);
   int stage = 0, t = 0;
   if (have) {
-    issue_dt(0, cur);
     mbar_expect_tx(&bars[kBarLoad0], kLoadBytes);
     issue_x(0, cur);
     issue_bc(0, cur);
@@ -311,8 +343,10 @@ __device__ void issuer_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, co
   while (have) {
     TileCursor nxt = cur;
     const bool have_next = cursor_next(pb, rp, nxt);
+    TRACE_ISSUE(0);
     // S = C B^T once this tile's x, B, C are in (the previous mask finished with S).
     if (!(ok = wait(stage))) break;
+    TRACE_ISSUE(1);
     tc_fence_after();
 #pragma unroll
     for (int kk = 0; kk < NS / 16; ++kk) {
@@ -323,7 +357,9 @@ __device__ void issuer_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, co
     pending |= 1u << kBarS;
     // Left factor C h^T into Y: needs the bf16 state and the previous epilogue done with Y.
     if (!(ok = wait(kBarHt))) break;
+    TRACE_ISSUE(2);
     if (t > 0 && !(ok = wait(kBarFree))) break;
+    TRACE_ISSUE(3);
     tc_fence_after();
 #pragma unroll
     for (int kk = 0; kk < NS / 16; ++kk) {
@@ -335,14 +371,15 @@ __device__ void issuer_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, co
     pending |= 1u << kBarYo;
     if (have_next) {  // the other x stage (tile t-1's x, then its y) is free once its y store read it
       if (t > 0 && !(ok = wait(kBarXfree))) break;
+      TRACE_ISSUE(4);
       fence_proxy_async();
-      issue_dt(stage ^ 1, nxt);
       mbar_expect_tx(&bars[stage ^ 1], kLoadBytes);
       issue_x(stage ^ 1, nxt);
       pending |= 1u << (stage ^ 1);
     }
     // Right factor onto the (decay-scaled) state: h^T += B^T [w0 x0 | w1 x1].
     if (!(ok = wait(kBarXw))) break;
+    TRACE_ISSUE(5);
     tc_fence_after();
 #pragma unroll
     for (int kk = 0; kk < kTile / 16; ++kk)
@@ -350,8 +387,17 @@ __device__ void issuer_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, co
                sdesc_sw128(a_sxw + kk * 2048, kAtom, 1024), id_st, 1);
     umma_commit(&bars[kBarSt]);
     pending |= 1u << kBarSt;
+    // B and C are free once S and both factors are done: next tile's, issued now so that
+    // the load runs under this tile's masked product and epilogue.
+    if (have_next) {
+      if (!(ok = wait(kBarS)) || !(ok = wait(kBarYo)) || !(ok = wait(kBarSt))) break;
+      TRACE_ISSUE(6);
+      fence_proxy_async();
+      issue_bc(stage ^ 1, nxt);
+    }
     // Y_h += P_h x_h (A from tensor memory).
     if (!(ok = wait(kBarP))) break;
+    TRACE_ISSUE(7);
     tc_fence_after();
     {
       const uint32_t a_sx = smem_u32(sx + stage * kHeads * kAtom);
@@ -365,12 +411,6 @@ __device__ void issuer_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, co
     }
     umma_commit(&bars[kBarY]);
     pending |= 1u << kBarY;
-    // B and C are free once S and both factors are done: next tile's.
-    if (have_next) {
-      if (!(ok = wait(kBarS)) || !(ok = wait(kBarYo)) || !(ok = wait(kBarSt))) break;
-      fence_proxy_async();
-      issue_bc(stage ^ 1, nxt);
-    }
     cur = nxt;
     have = have_next;
     stage ^= 1;
@@ -381,38 +421,40 @@ __device__ void issuer_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, co
     // Drain what this thread issued (again bounded) before tensor memory is freed.
     for (int k = 0; k < kNumBars; ++k)
       if (pending & (1u << k)) mbar_wait_bounded(&bars[k], (phase >> k) & 1u, kWaitLimit);
-    for (int st = 0; st < 2; ++st)  // the last dt load of each stage (its phases complete in order)
-      if (dt_issued[st] > 0) mbar_wait_bounded(&bars[kBarDt0 + st], (dt_issued[st] - 1) & 1, kWaitLimit);
   }
 }
 
 // --------------------------------------------------------- compute warpgroups
-// Two warpgroups, one per head of the pair; thread i owns TMEM lane / tile row i.  The
-// warps run free of each other inside a tile: each computes the whole tile's cumsum and
-// column factors into its own shared arrays and stores its own 32 rows of y, so no
-// compute-wide barrier sits in the tile loop.  Every wait is warp-uniform.
+// Four warpgroups: two per head of the pair, one per 32-column half of that head's Y and
+// state columns in tensor memory.  Warp (head hw, half ch, quarter wq) owns TMEM lanes /
+// tile rows 32 wq .. 32 wq + 31 and columns 32 ch .. 32 ch + 31 of its head's Y and state;
+// of the masked product it computes the 32-column blocks ch and ch + 2.  What is the same
+// for every row of a tile (where it is, the cumsums and column factors) comes from the
+// helper warp's tile descriptor.  The two halves of a row quarter meet once a tile, on a
+// one-arrival barrier, before the half-0 warp stores their 32 rows of y by TMA.  Every
+// wait is warp-uniform and bounded.
 template <int NS>
 __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8_t* smem, uint32_t tmem,
                              uint64_t* bars, volatile int* abort_flag) {
   using L = Layout<NS>;
   const int tid = threadIdx.x;
-  const int hw = tid / kWGThreads;       // head of the pair
-  const int i = tid % kWGThreads;        // row / TMEM lane
-  const int wq = i >> 5, lane = i & 31;  // lane quarter of this warp
-  const int wid = tid >> 5;              // compute warp 0..7
+  const int wid = tid >> 5;                 // compute warp 0..15
+  const int hw = wid >> 3;                  // head of the pair
+  const int ch = (wid >> 2) & 1;            // column half
+  const int wq = wid & 3, lane = tid & 31;  // lane quarter (a warp reaches TMEM lanes 32 (warp % 4) ..)
+  const int i = wq * 32 + lane;             // row / TMEM lane
+  const int pair_bar = kBarPair0 + hw * 4 + wq;
   const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+  const uint32_t col_h = hw * 64 + ch * 32;  // this warp's Y and state columns
   uint8_t* sx = smem + L::x;
   uint8_t* sxw = smem + L::xw;
   uint8_t* sht = smem + L::ht;
-  // this warp's copies of the tile's cumsum, column factors and dt, and its dt prefetch
-  float* w_cs = reinterpret_cast<float*>(smem + L::wcs) + wid * kTile;
-  float* w_cc = reinterpret_cast<float*>(smem + L::wcc) + wid * kTile;
-  float* w_dt = reinterpret_cast<float*>(smem + L::wdt) + wid * kTile;
+  const TileDesc* descs = reinterpret_cast<const TileDesc*>(smem + L::desc);
   const int pairs = pb.H / kHeads;
   const int units = pb.nseq * pairs;
 
   uint32_t phase = 0;
-  // Warp-uniform bounded wait on an issuer barrier.
+  // Warp-uniform bounded wait on a barrier.
   auto wait = [&](int k) -> bool {
     const bool mine = wait_or_abort(&bars[k], (phase >> k) & 1u, abort_flag);
     if (__any_sync(0xffffffffu, !mine)) return false;
@@ -428,37 +470,35 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
       const int s = u / pairs;
       const int h = (u % pairs) * kHeads + hw;
       const int64_t base = ((int64_t)s * pb.H + h) * kHeadDim * NS;
-      for (int p = 0; p < kHeadDim; ++p)
+      for (int p = 32 * ch; p < 32 * ch + 32; ++p)
         pb.final_state[base + (int64_t)p * NS + i] = pb.init ? pb.init[base + (int64_t)p * NS + i] : 0.f;
     }
   }
 
-  const RangePlan rp = plan_range(pb);
-  // This warpgroup's head state lives in tensor memory as h^T (lane n = state column n,
-  // 64 fp32 columns); its bf16 copy in shared memory is the B operand of the left factor.
-  const uint32_t t_state = tmem + lane_base + kColSt + hw * 64;
-  float cs_base = 0.f;  // in-chunk cumsum (log2 units) before the current tile
-  auto write_ht_from = [&](const uint32_t (&r)[64]) {
+  // The head state lives in tensor memory as h^T (lane n = state column n, 64 fp32
+  // columns, 32 per half); its bf16 copy in shared memory is the B operand of the left factor.
+  const uint32_t t_state = tmem + lane_base + kColSt + col_h;
+  auto write_ht_from = [&](const uint32_t (&r)[32]) {
     if (i < NS) {
       uint8_t* hdst = sht + hw * NS * 128;
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int c = 0; c < 4; ++c) {
         uint4 hv;
         hv.x = bf16x2_of(f2u(r[8 * c + 0], r[8 * c + 1]));
         hv.y = bf16x2_of(f2u(r[8 * c + 2], r[8 * c + 3]));
         hv.z = bf16x2_of(f2u(r[8 * c + 4], r[8 * c + 5]));
         hv.w = bf16x2_of(f2u(r[8 * c + 6], r[8 * c + 7]));
-        *reinterpret_cast<uint4*>(hdst + sw128_off(i, c)) = hv;
+        *reinterpret_cast<uint4*>(hdst + sw128_off(i, 4 * ch + c)) = hv;
       }
     }
   };
-  // State at the start of piece c into tensor memory and its bf16 copy: the sequence's
-  // initial state, or (carry in) the state and cumsum the previous CTA published.
-  // False if that wait gave up.
-  auto load_state = [&](const TileCursor& c) -> bool {
+  // The state at the start of the piece whose first tile d describes, into r: the
+  // sequence's initial state (or zero), or the state the previous CTA handed on.
+  // False if the wait for that hand-on gave up.
+  auto load_state = [&](const TileDesc& d, uint32_t (&r)[32]) -> bool {
     const float* src_p = nullptr;
-    if (c.flags & kCarryIn) {
-      const int src = rp.carry_src;
+    if (d.flags & kDescCarryIn) {
+      const int src = d.carry_src;
       bool mine = true;
       if (lane == 0) {
         const long long t0 = clock64();
@@ -474,29 +514,37 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
       if (__any_sync(0xffffffffu, !mine)) return false;
       __threadfence();
       src_p = pb.carry + ((size_t)src * kHeads + hw) * kHeadDim * NS + i;
-      cs_base = __ldcg(pb.carry + (size_t)pb.ranges * kHeads * kHeadDim * NS + src * kHeads + hw);
-    } else {
-      const int s = c.unit / pairs;
-      const int h = (c.unit % pairs) * kHeads + hw;
-      if (pb.init) src_p = pb.init + ((int64_t)s * pb.H + h) * kHeadDim * NS + i;
-      cs_base = 0.f;
+    } else if (pb.init) {
+      src_p = pb.init + ((int64_t)d.s * pb.H + d.h0 + hw) * kHeadDim * NS + i;
     }
-    uint32_t r[64];
 #pragma unroll
-    for (int q = 0; q < 64; ++q) r[q] = __float_as_uint((src_p && i < NS) ? __ldcg(src_p + (size_t)q * NS) : 0.f);
-    tmem_st64(t_state, r);
-    write_ht_from(r);
-    tmem_st_wait();
-    fence_proxy_async();
+    for (int q = 0; q < 32; ++q)
+      r[q] = __float_as_uint((src_p && i < NS) ? __ldcg(src_p + (size_t)(32 * ch + q) * NS) : 0.f);
     return true;
   };
-  auto head_of = [&](const TileCursor& c) { return (c.unit % pairs) * kHeads + hw; };
+  // r holds the state at the start of the tile d describes: its bf16 copy is the left
+  // factor's operand; scaled by the tile's decay it is what the right factor accumulates onto.
+  auto start_tile_state = [&](const TileDesc& d, uint32_t (&r)[32]) {
+    write_ht_from(r);
+    const float decay = d.decay[hw];
+    const uint64_t decay2 = f2(decay, decay);
+#pragma unroll
+    for (int q = 0; q < 16; ++q) {
+      float lo, hi;
+      unf2(mul2(decay2, f2u(r[2 * q], r[2 * q + 1])), lo, hi);
+      r[2 * q] = __float_as_uint(lo);
+      r[2 * q + 1] = __float_as_uint(hi);
+    }
+    tmem_st32(t_state, r);
+    tmem_st_wait();
+  };
   // P values of one 32-column block of S (fp32 bits in r) for row i.
-  auto mask_block = [&](int cb, const uint32_t* r, float cs_i, uint32_t (&pk)[16]) {
+  auto mask_block = [&](int cb, const uint32_t* r, float cs_i, const float* dcs, const float* dcc,
+                        const float* ddt, uint32_t (&pk)[16]) {
     if (cb < wq) {  // strictly below the diagonal: exp(cs_i - cs_j) = rf * exp(cs_ref - cs_j)
-      const float rf = ex2(cs_i - w_cs[cb * 32 + 31]);
+      const float rf = ex2(cs_i - dcs[cb * 32 + 31]);
       const uint64_t rf2 = f2(rf, rf);
-      const float4* cc4 = reinterpret_cast<const float4*>(w_cc + cb * 32);
+      const float4* cc4 = reinterpret_cast<const float4*>(dcc + cb * 32);
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4) {
         const float4 c = cc4[q4];
@@ -505,8 +553,8 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
         pk[2 * q4 + 1] = bf16x2_of(mul2(f1, f2u(r[4 * q4 + 2], r[4 * q4 + 3])));
       }
     } else {  // diagonal block: mask first (-inf), then exp
-      const float4* c4 = reinterpret_cast<const float4*>(w_cs + cb * 32);
-      const float4* d4 = reinterpret_cast<const float4*>(w_dt + cb * 32);
+      const float4* c4 = reinterpret_cast<const float4*>(dcs + cb * 32);
+      const float4* d4 = reinterpret_cast<const float4*>(ddt + cb * 32);
 #pragma unroll
       for (int q4 = 0; q4 < 8; ++q4) {
         const float4 cj = c4[q4], dj = d4[q4];
@@ -521,93 +569,35 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
     }
   };
 
-  TileCursor cur;
-  bool have = cursor_first(pb, rp, cur);
-  if (!have) return;
-  if (!load_state(cur)) return;
+  if (!wait(kBarDescFull0)) return;
+  if (descs[0].flags & kDescEnd) return;
+  {
+    uint32_t r[32];
+    if (!load_state(descs[0], r)) return;
+    start_tile_state(descs[0], r);
+  }
+  fence_proxy_async();
   tc_fence_before();
   warp_arrive(&bars[kBarHt]);
-  float a2_cur = pb.A[head_of(cur)] * 1.4426950408889634f;  // A_h log2(e): cumsums are in log2 units
-  float d_cur = pb.D ? pb.D[head_of(cur)] : 0.f;
-  int stage = 0, tile_idx = 0;
   int trace_tile = 0;
   (void)trace_tile;
 
-  while (have) {
+  for (int t = 0;; ++t) {
+    const int slot = t % kDescSlots, stage = t & 1;
+    const TileDesc& d = descs[slot];
     TRACE_MARK(0);
-    const int s = cur.unit / pairs;
-    const int h = head_of(cur);
-    const int64_t t0 = cur.tb + cur.k0;
-    const int rem = min(kTile, cur.len - cur.k0);
-    if (cur.k0 % pb.Q == 0) cs_base = 0.f;
-    const float Ah2 = a2_cur, Dh = d_cur;
-
-    // look ahead: next tile's dt (and its head's parameters at a unit change)
-    TileCursor nxt = cur;
-    const bool have_next = cursor_next(pb, rp, nxt);
-    TRACE_MARK(10);
-    if (!wait(kBarDt0 + stage)) return;  // this tile's dt (the issuer loaded it a tile ahead)
-    TRACE_MARK(11);
-    float4 d4;  // dt of tokens 4 lane .. 4 lane + 3 (0 past the end of the sequence)
-    {
-      // Row 4 lane + j holds the 4 heads' dt of one token.  Lane reads its rows in the
-      // order j = (k + rot) & 3, rot = (lane / 2) & 3, so each quarter warp's 16-byte
-      // loads fall in distinct banks; then the rows go back in order and the head is picked.
-      const float4* rows = reinterpret_cast<const float4*>(smem + L::sdt + stage * kTile * 16) + 4 * lane;
-      const int rot = (lane >> 1) & 3, hh = h & 3;
-      float v[4];
-#pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float4 q = rows[(k + rot) & 3];
-        v[k] = hh == 0 ? q.x : hh == 1 ? q.y : hh == 2 ? q.z : q.w;
-      }
-      float dj[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {  // token j came in as k = (j - rot) & 3
-        const int k = (j - rot) & 3;
-        dj[j] = k == 0 ? v[0] : k == 1 ? v[1] : k == 2 ? v[2] : v[3];
-      }
-      const int left = cur.len - cur.k0 - 4 * lane;
-      d4.x = 0 < left ? dj[0] : 0.f;
-      d4.y = 1 < left ? dj[1] : 0.f;
-      d4.z = 2 < left ? dj[2] : 0.f;
-      d4.w = 3 < left ? dj[3] : 0.f;
-    }
-    if (have_next) {
-      if (nxt.unit != cur.unit) {
-        a2_cur = pb.A[head_of(nxt)] * 1.4426950408889634f;
-        d_cur = pb.D ? pb.D[head_of(nxt)] : 0.f;
-      }
-    }
-
-    // ---- in-chunk cumsum of dt*A over the whole tile, by every warp (log2 units)
-    float c0 = d4.x * Ah2, c1 = c0 + d4.y * Ah2, c2 = c1 + d4.z * Ah2, c3 = c2 + d4.w * Ah2;
-    float v = c3;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const float u = __shfl_up_sync(0xffffffffu, v, o);
-      if (lane >= o) v += u;
-    }
-    const float base = cs_base + v - c3;  // cumsum before token 4 lane
-    c0 += base, c1 += base, c2 += base, c3 += base;
-    reinterpret_cast<float4*>(w_cs)[lane] = make_float4(c0, c1, c2, c3);
-    reinterpret_cast<float4*>(w_dt)[lane] = d4;
-    // block ends (tokens 31, 63, 95, 127) live in lanes 7, 15, 23, 31
-    const float ref = __shfl_sync(0xffffffffu, c3, (lane & ~7) | 7);  // end of this lane's 32-block
-    reinterpret_cast<float4*>(w_cc)[lane] =
-        make_float4(ex2(ref - c0) * d4.x, ex2(ref - c1) * d4.y, ex2(ref - c2) * d4.z, ex2(ref - c3) * d4.w);
-    TRACE_MARK(12);
-    const float cs_end = __shfl_sync(0xffffffffu, c3, 31);  // tokens past the end add 0
-    const float cs_start = cs_base;
-    cs_base = cs_end;
-    __syncwarp();
-    const float cs_i = w_cs[i];
-    const float dtj = w_dt[i];
-    const float w_i = ex2(cs_end - cs_i) * dtj;  // right-factor weight (0 past the end)
-    const float carry = ex2(cs_i - cs_start);    // decay of the carried-in state to token i
+    const int h = d.h0 + hw;
+    const int t0 = d.t0, rem = d.rem, flags = d.flags;
+    const float* dcs = d.cs[hw];
+    const float* dcc = d.cc[hw];
+    const float* ddt = d.dtv[hw];
+    const float cs_start = d.cs_start[hw], cs_end = d.cs_end[hw];
+    const float cs_i = dcs[i];
+    const float w_i = ex2(cs_end - cs_i) * ddt[i];  // right-factor weight (0 past the end)
+    const float carry = ex2(cs_i - cs_start);      // decay of the carried-in state to token i
     TRACE_MARK(1);
 
-    // ---- this tile's x: w o x, the right-factor input; the state scaled by this tile's decay
+    // ---- this tile's x: w o x, the right-factor input
     if (!wait(stage)) return;
     TRACE_MARK(2);
     const uint8_t* sxh = sx + (stage * kHeads + hw) * kAtom;
@@ -615,8 +605,8 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
       uint8_t* dst = sxw + hw * kAtom;
       const uint32_t w2 = pack_bf16(w_i, w_i);
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
-        const uint32_t o = sw128_off(i, c);
+      for (int cc = 0; cc < 4; ++cc) {
+        const uint32_t o = sw128_off(i, 4 * ch + cc);
         uint4 xv = *reinterpret_cast<const uint4*>(sxh + o);
         xv.x = mul_bf16x2(xv.x, w2);
         xv.y = mul_bf16x2(xv.y, w2);
@@ -626,25 +616,8 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
       }
     }
     fence_proxy_async();
-    {
-      const float decay = ex2(cs_end - cs_start);
-      const uint64_t decay2 = f2(decay, decay);
-      uint32_t r[64];
-      tmem_ld64(t_state, r);
-      tmem_ld_wait();
-#pragma unroll
-      for (int q = 0; q < 32; ++q) {
-        float lo, hi;
-        unf2(mul2(decay2, f2u(r[2 * q], r[2 * q + 1])), lo, hi);
-        r[2 * q] = __float_as_uint(lo);
-        r[2 * q + 1] = __float_as_uint(hi);
-      }
-      tmem_st64(t_state, r);
-      tmem_st_wait();
-      tc_fence_before();
-    }
     warp_arrive(&bars[kBarXw]);
-    if (tile_idx > 0) {  // this warp's y store of the previous tile has read its x stage: release it
+    if (t > 0) {  // this warp's y store of the previous tile has read its x stage: release it
       if (lane == 0) bulk_wait_read();
       warp_arrive(&bars[kBarXfree]);
     }
@@ -655,27 +628,21 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
     TRACE_MARK(4);
     tc_fence_after();
     {
+      // blocks ch and ch + 2 (32 columns of S each) -> P columns 16 cb .. 16 cb + 15
       const uint32_t colp = kColP + hw * 64;
 #pragma unroll 1
-      for (int cb = 0; cb < 4; cb += 2) {  // blocks cb, cb + 1 (64 columns of S) -> P columns 16cb..16cb+31
-        uint32_t pk0[16], pk1[16];
+      for (int cb = ch; cb < 4; cb += 2) {
+        uint32_t pk[16];
         if (cb <= wq) {
-          uint32_t r[64];
-          tmem_ld64(tmem + lane_base + kColS + cb * 32, r);
+          uint32_t r[32];
+          tmem_ld32(tmem + lane_base + kColS + cb * 32, r);
           tmem_ld_wait();
-          mask_block(cb, r, cs_i, pk0);
-          if (cb + 1 <= wq) {
-            mask_block(cb + 1, r + 32, cs_i, pk1);
-          } else {
-#pragma unroll
-            for (int q = 0; q < 16; ++q) pk1[q] = 0u;
-          }
+          mask_block(cb, r, cs_i, dcs, dcc, ddt, pk);
         } else {  // above the diagonal: zero
 #pragma unroll
-          for (int q = 0; q < 16; ++q) pk0[q] = pk1[q] = 0u;
+          for (int q = 0; q < 16; ++q) pk[q] = 0u;
         }
-        tmem_st16(tmem + lane_base + colp + cb * 16, pk0);
-        tmem_st16(tmem + lane_base + colp + (cb + 1) * 16, pk1);
+        tmem_st16(tmem + lane_base + colp + cb * 16, pk);
       }
     }
     TRACE_MARK(5);
@@ -685,74 +652,81 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
     tc_fence_after();
     {
       const uint64_t carry2 = f2(carry, carry);
-      uint32_t r[64];
-      tmem_ld64(tmem + lane_base + kColY + hw * 64, r);
+      uint32_t r[32];
+      tmem_ld32(tmem + lane_base + kColY + col_h, r);
       tmem_ld_wait();
 #pragma unroll
-      for (int q = 0; q < 32; ++q) {
+      for (int q = 0; q < 16; ++q) {
         float lo, hi;
         unf2(mul2(carry2, f2u(r[2 * q], r[2 * q + 1])), lo, hi);
         r[2 * q] = __float_as_uint(lo);
         r[2 * q + 1] = __float_as_uint(hi);
       }
-      tmem_st64(tmem + lane_base + kColY + hw * 64, r);
+      tmem_st32(tmem + lane_base + kColY + col_h, r);
     }
     tmem_st_wait();
     tc_fence_before();
     warp_arrive(&bars[kBarP]);
     TRACE_MARK(6);
 
-    // ---- the state after this tile: its bf16 copy for the next tile; at the end of a
-    // piece the final state or the hand-on to the next CTA, then the next piece's state
+    // ---- the state after this tile: at the end of a piece the final state or the
+    // hand-on to the next CTA; then the next tile's start state (this one, or the next
+    // piece's) as its bf16 copy and, decay-scaled, in tensor memory
     if (!wait(kBarSt)) return;
     tc_fence_after();
+    const int nslot = (t + 1) % kDescSlots;
+    bool more;
     {
-      const bool piece_done = !have_next || nxt.piece != cur.piece;
-      const bool to_final = piece_done && (cur.flags & kUnitEnd) && pb.final_state && i < NS;
-      const bool to_carry = piece_done && (cur.flags & kCarryOut);
-      float* fp = pb.final_state ? pb.final_state + ((int64_t)s * pb.H + h) * kHeadDim * NS + i : nullptr;
-      float* cp = pb.carry + ((size_t)blockIdx.x * kHeads + hw) * kHeadDim * NS + i;
-      {
-        uint32_t r[64];
-        tmem_ld64(t_state, r);
-        tmem_ld_wait();
-        if (!piece_done) write_ht_from(r);
-        if (to_final) {
+      uint32_t r[32];
+      tmem_ld32(t_state, r);
+      tmem_ld_wait();
+      if ((flags & kDescToFinal) && i < NS) {
+        float* fp = pb.final_state + ((int64_t)d.s * pb.H + h) * kHeadDim * NS + i;
 #pragma unroll
-          for (int q = 0; q < 64; ++q) fp[(size_t)q * NS] = __uint_as_float(r[q]);
-        }
-        if (to_carry && i < NS) {
-#pragma unroll
-          for (int q = 0; q < 64; ++q) cp[(size_t)q * NS] = __uint_as_float(r[q]);
-        }
+        for (int q = 0; q < 32; ++q) fp[(size_t)(32 * ch + q) * NS] = __uint_as_float(r[q]);
       }
-      if (to_carry) {  // hand the state on: one release increment per warp once its part is out
-        if (i == 0) pb.carry[(size_t)pb.ranges * kHeads * kHeadDim * NS + blockIdx.x * kHeads + hw] = cs_base;
+      if (flags & kDescToCarry) {  // hand the state on: one release increment per warp once its part is out
+        if (i < NS) {
+          float* cp = pb.carry + ((size_t)blockIdx.x * kHeads + hw) * kHeadDim * NS + i;
+#pragma unroll
+          for (int q = 0; q < 32; ++q) cp[(size_t)(32 * ch + q) * NS] = __uint_as_float(r[q]);
+        }
+        if (i == 0 && ch == 0)
+          pb.carry[(size_t)pb.ranges * kHeads * kHeadDim * NS + blockIdx.x * kHeads + hw] = cs_end;
         __threadfence();
         __syncwarp();
         if (lane == 0) red_add_release_gpu(&pb.carry_flag[blockIdx.x], 1);
         __syncwarp();
       }
-      if (piece_done && have_next && !load_state(nxt)) return;
+      if (!wait(kBarDescFull0 + nslot)) return;
+      const TileDesc& dn = descs[nslot];
+      more = !(dn.flags & kDescEnd);
+      if (more) {
+        if ((dn.flags & kDescFirst) && !load_state(dn, r)) return;
+        start_tile_state(dn, r);
+      }
     }
     fence_proxy_async();
     tc_fence_before();
     warp_arrive(&bars[kBarHt]);
     TRACE_MARK(7);
 
-    // ---- epilogue: y = Y + D x, staged over this tile's x; each warp stores its 32 rows by TMA
+    // ---- epilogue: y = Y + D x, staged over this tile's x; the half-0 warp of each row
+    // quarter stores the quarter's 32 rows by TMA once the half-1 warp has staged its columns
     if (!wait(kBarY)) return;
     TRACE_MARK(8);
     tc_fence_after();
     {
-      const bool full = cur.k0 + 32 * wq + 32 <= cur.len;  // all 32 rows of this warp are in the sequence
+      const float Dh = d.dskip[hw];
+      const bool full = rem >= 32 * wq + 32;  // all 32 rows of this quarter are in the sequence
       uint8_t* ystage = const_cast<uint8_t*>(sxh);  // each thread overwrites the x chunks it reads
-      __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(pb.y) + ((t0 + i) * pb.H + h) * kHeadDim;
-      uint32_t ry[64];
-      tmem_ld64(tmem + lane_base + kColY + hw * 64, ry);
+      __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(pb.y) + ((int64_t)(t0 + i) * pb.H + h) * kHeadDim;
+      uint32_t ry[32];
+      tmem_ld32(tmem + lane_base + kColY + col_h, ry);
       tmem_ld_wait();
 #pragma unroll
-      for (int c = 0; c < 8; ++c) {
+      for (int cc = 0; cc < 4; ++cc) {
+        const int c = 4 * ch + cc;
         const uint32_t o = sw128_off(i, c);
         const uint4 xv = *reinterpret_cast<const uint4*>(sxh + o);
         const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
@@ -760,8 +734,8 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
 #pragma unroll
         for (int q = 0; q < 4; ++q) {
           const float x0 = __uint_as_float(xu[q] << 16), x1 = __uint_as_float(xu[q] & 0xFFFF0000u);
-          out[q] = pack_bf16(fmaf(Dh, x0, __uint_as_float(ry[8 * c + 2 * q])),
-                             fmaf(Dh, x1, __uint_as_float(ry[8 * c + 2 * q + 1])));
+          out[q] = pack_bf16(fmaf(Dh, x0, __uint_as_float(ry[8 * cc + 2 * q])),
+                             fmaf(Dh, x1, __uint_as_float(ry[8 * cc + 2 * q + 1])));
         }
         const uint4 ov = make_uint4(out[0], out[1], out[2], out[3]);
         if (full)
@@ -772,19 +746,208 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
       tc_fence_before();
       if (full) fence_proxy_async();
       __syncwarp();
-      if (full && lane == 0) {
-        tma_store_3d(tm_y32, ystage + wq * 32 * 128, 0, h, (int)(t0 + 32 * wq));
-        bulk_commit();
+      if (ch == 1) {
+        if (lane == 0) mbar_arrive(&bars[pair_bar]);
+      } else {
+        if (!wait(pair_bar)) return;
+        if (full && lane == 0) {
+          tma_store_3d(tm_y32, ystage + wq * 32 * 128, 0, h, t0 + 32 * wq);
+          bulk_commit();
+        }
       }
       __syncwarp();
     }
-    warp_arrive(&bars[kBarFree]);
+    // Y is free for the next left factor; this tile's descriptor is used up
+    __syncwarp();
+    if (lane == 0) {
+      mbar_arrive(&bars[kBarFree]);
+      mbar_arrive(&bars[kBarDescFree0 + slot]);
+    }
+    __syncwarp();
     TRACE_MARK(9);
     ++trace_tile;
-    ++tile_idx;
+    if (!more) break;
+  }
+}
+
+// ------------------------------------------------------------------ helper warp
+// Walks the CTA's tile sequence a few tiles ahead of the compute warps: loads each tile's
+// dt by TMA (kDtStages tiles in flight) and writes the tile's descriptor into a ring of
+// kDescSlots: where the tile is, what happens to the state around it, and per head of the
+// pair the in-chunk cumsum of dt A in log2 units (restarted at every chunk boundary, and
+// continued from the handing-on CTA's value at a hand-on), the column factors
+// exp2(cs(end of 32-block) - cs_j) dt_j, dt (0 past the sequence end) and D.
+template <int NS>
+__device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t* smem, uint64_t* bars,
+                            volatile int* abort_flag) {
+  using L = Layout<NS>;
+  const int lane = threadIdx.x & 31;
+  const int pairs = pb.H / kHeads;
+  TileDesc* descs = reinterpret_cast<TileDesc*>(smem + L::desc);
+  uint32_t phase = 0;
+  auto wait = [&](int k) -> bool {
+    const bool mine = wait_or_abort(&bars[k], (phase >> k) & 1u, abort_flag);
+    if (__any_sync(0xffffffffu, !mine)) return false;
+    phase ^= 1u << k;
+    return true;
+  };
+  const RangePlan rp = plan_range(pb);
+
+  // dt loads run up to kDtStages tiles ahead on a cursor of their own
+  TileCursor ahead;
+  bool have_ahead = cursor_first(pb, rp, ahead);
+  int dt_issued = 0;
+  auto issue_dt = [&]() {
+    if (lane == 0) {
+      const int st = dt_issued % kDtStages;
+      const int h0 = (ahead.unit % pairs) * kHeads;
+      mbar_expect_tx(&bars[kBarDt0 + st], kTile * 16);
+      tma_load_2d(smem + L::sdt + st * kTile * 16, tm_dt, h0 & ~3, ahead.tb + ahead.k0, &bars[kBarDt0 + st]);
+    }
+    ++dt_issued;
+    have_ahead = cursor_next(pb, rp, ahead);
+  };
+  for (int k = 0; k < kDtStages && have_ahead; ++k) issue_dt();
+
+  TileCursor cur;
+  bool have = cursor_first(pb, rp, cur);
+  float cs_base[kHeads] = {0.f, 0.f};
+  float a2[kHeads] = {0.f, 0.f}, dsk[kHeads] = {0.f, 0.f};
+  int a_unit = -1, prev_piece = -1;
+  bool ok = true;
+  int t = 0;
+  for (;; ++t) {
+    const int slot = t % kDescSlots;
+    if (t >= kDescSlots && !(ok = wait(kBarDescFree0 + slot))) break;
+    TileDesc& d = descs[slot];
+    if (!have) {
+      if (lane == 0) d.flags = kDescEnd;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kBarDescFull0 + slot]);
+      break;
+    }
+    TileCursor nxt = cur;
+    const bool have_next = cursor_next(pb, rp, nxt);
+    const bool first = cur.piece != prev_piece;
+    const bool last = !have_next || nxt.piece != cur.piece;
+    prev_piece = cur.piece;
+    const int h0 = (cur.unit % pairs) * kHeads;
+    if (cur.unit != a_unit) {
+      a_unit = cur.unit;
+#pragma unroll
+      for (int hh = 0; hh < kHeads; ++hh) {
+        a2[hh] = pb.A[h0 + hh] * 1.4426950408889634f;  // A_h log2(e): cumsums are in log2 units
+        dsk[hh] = pb.D ? pb.D[h0 + hh] : 0.f;
+      }
+    }
+    int flags = 0;
+    if (first) {
+      flags |= kDescFirst;
+      cs_base[0] = cs_base[1] = 0.f;
+      if (cur.flags & kCarryIn) {  // continue from the cumsum the previous CTA reached
+        flags |= kDescCarryIn;
+        bool mine = true;
+        if (lane == 0) {
+          const long long c0 = clock64();
+          while (ld_acquire_gpu(&pb.carry_flag[rp.carry_src]) < kComputeWarps) {
+            if (*abort_flag || clock64() - c0 > kWaitLimit) {
+              *abort_flag = 1;
+              mine = false;
+              break;
+            }
+            __nanosleep(200);
+          }
+        }
+        if (__any_sync(0xffffffffu, !mine)) {
+          ok = false;
+          break;
+        }
+        __threadfence();
+#pragma unroll
+        for (int hh = 0; hh < kHeads; ++hh)
+          cs_base[hh] = __ldcg(pb.carry + (size_t)pb.ranges * kHeads * kHeadDim * NS + rp.carry_src * kHeads + hh);
+      }
+    }
+    if (last && (cur.flags & kUnitEnd) && pb.final_state) flags |= kDescToFinal;
+    if (last && (cur.flags & kCarryOut)) flags |= kDescToCarry;
+    if (cur.k0 % pb.Q == 0) cs_base[0] = cs_base[1] = 0.f;
+
+    // this tile's dt: row 4 lane + j holds the 4 heads' dt of one token; a lane reads its
+    // rows in the order j = (k + rot) & 3, rot = (lane / 2) & 3, so each quarter warp's
+    // 16-byte loads fall in distinct banks
+    if (!(ok = wait(kBarDt0 + t % kDtStages))) break;
+    float dtt[kHeads][4];
+    {
+      const float4* rows = reinterpret_cast<const float4*>(smem + L::sdt + (t % kDtStages) * kTile * 16) + 4 * lane;
+      const int rot = (lane >> 1) & 3, hb = h0 & 3;  // the pair's first head in the 4-head row
+      float v[kHeads][4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) {
+        const float4 q = rows[(k + rot) & 3];
+        v[0][k] = hb == 0 ? q.x : q.z;  // hb is 0 or 2 (h0 is even)
+        v[1][k] = hb == 0 ? q.y : q.w;
+      }
+      const int left = cur.len - cur.k0 - 4 * lane;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {  // token j came in as k = (j - rot) & 3
+        const int k = (j - rot) & 3;
+#pragma unroll
+        for (int hh = 0; hh < kHeads; ++hh) {
+          const float val = k == 0 ? v[hh][0] : k == 1 ? v[hh][1] : k == 2 ? v[hh][2] : v[hh][3];
+          dtt[hh][j] = j < left ? val : 0.f;
+        }
+      }
+    }
+#pragma unroll
+    for (int hh = 0; hh < kHeads; ++hh) {
+      const float Ah2 = a2[hh];
+      float c0 = dtt[hh][0] * Ah2, c1 = c0 + dtt[hh][1] * Ah2, c2 = c1 + dtt[hh][2] * Ah2,
+            c3 = c2 + dtt[hh][3] * Ah2;
+      float v = c3;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const float u = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += u;
+      }
+      const float base = cs_base[hh] + v - c3;  // cumsum before token 4 lane
+      c0 += base, c1 += base, c2 += base, c3 += base;
+      reinterpret_cast<float4*>(d.cs[hh])[lane] = make_float4(c0, c1, c2, c3);
+      reinterpret_cast<float4*>(d.dtv[hh])[lane] = make_float4(dtt[hh][0], dtt[hh][1], dtt[hh][2], dtt[hh][3]);
+      // block ends (tokens 31, 63, 95, 127) live in lanes 7, 15, 23, 31
+      const float ref = __shfl_sync(0xffffffffu, c3, (lane & ~7) | 7);
+      reinterpret_cast<float4*>(d.cc[hh])[lane] =
+          make_float4(ex2(ref - c0) * dtt[hh][0], ex2(ref - c1) * dtt[hh][1], ex2(ref - c2) * dtt[hh][2],
+                      ex2(ref - c3) * dtt[hh][3]);
+      const float cs_end = __shfl_sync(0xffffffffu, c3, 31);  // tokens past the end add 0
+      if (lane == 0) {
+        d.cs_start[hh] = cs_base[hh];
+        d.cs_end[hh] = cs_end;
+        d.decay[hh] = ex2(cs_end - cs_base[hh]);
+        d.dskip[hh] = dsk[hh];
+      }
+      cs_base[hh] = cs_end;
+    }
+    if (lane == 0) {
+      d.t0 = cur.tb + cur.k0;
+      d.rem = min(kTile, cur.len - cur.k0);
+      d.s = cur.unit / pairs;
+      d.h0 = h0;
+      d.flags = flags;
+      d.carry_src = rp.carry_src;
+    }
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars[kBarDescFull0 + slot]);
+    // the dt stage this tile used is read: refill it
+    if (have_ahead) issue_dt();
     cur = nxt;
     have = have_next;
-    stage ^= 1;
+  }
+  if (!ok) {
+    *abort_flag = 1;
+    // dt loads still in flight land before the CTA ends (bounded)
+    if (lane == 0)
+      for (int n = t; n < dt_issued; ++n)
+        mbar_wait_bounded(&bars[kBarDt0 + n % kDtStages], (n / kDtStages) & 1, kWaitLimit);
   }
 }
 
@@ -819,8 +982,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars[kBarP], kComputeWarps);
     mbar_init(&bars[kBarFree], kComputeWarps);
     mbar_init(&bars[kBarXfree], kComputeWarps);
-    mbar_init(&bars[kBarDt0], 1);
-    mbar_init(&bars[kBarDt1], 1);
+    for (int k = 0; k < kDtStages; ++k) mbar_init(&bars[kBarDt0 + k], 1);
+    for (int k = 0; k < kDescSlots; ++k) {
+      mbar_init(&bars[kBarDescFull0 + k], 1);
+      mbar_init(&bars[kBarDescFree0 + k], kComputeWarps);
+    }
+    for (int k = 0; k < kHeads * 4; ++k) mbar_init(&bars[kBarPair0 + k], 1);
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tensormap(&tm_x);
@@ -834,9 +1001,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s_tmem_base;
 
-  if (warp == kComputeThreads / 32) {
-    if ((tid & 31) == 0) issuer_loop<NS>(&tm_x, &tm_b, &tm_c, &tm_dt, pb, smem, tmem, bars, abort_flag);
+  if (warp == kIssuerWarp) {
+    if ((tid & 31) == 0) issuer_loop<NS>(&tm_x, &tm_b, &tm_c, pb, smem, tmem, bars, abort_flag);
     __syncwarp();  // the issuer warp reconverges before the CTA-wide barrier
+  } else if (warp == kHelperWarp) {
+    helper_loop<NS>(&tm_dt, pb, smem, bars, abort_flag);
+    __syncwarp();
   } else {
     compute_loop<NS>(&tm_y32, pb, smem, tmem, bars, abort_flag);
     if ((tid & 31) == 0) bulk_wait_all();  // this warp's y stores complete before the CTA exits
