@@ -5,6 +5,7 @@
 #include <string.h>
 
 #include <atomic>
+#include <vector>
 
 #include "ssd.h"
 #include "ssd_common.cuh"
@@ -35,6 +36,36 @@ unsigned int* status_ptr() {
 }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// The library's stream-ordered pool on the current device: scratch and the host entry
+// point's device buffers come from it, and freed blocks stay cached for the next call
+// (release threshold: never), so repeated calls do not go back to the driver.
+std::atomic<cudaMemPool_t> g_pool[kMaxDevices];
+cudaMemPool_t lib_pool() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  cudaMemPool_t p = g_pool[dev].load();
+  if (p) return p;
+  cudaMemPoolProps props{};
+  props.allocType = cudaMemAllocationTypePinned;
+  props.location.type = cudaMemLocationTypeDevice;
+  props.location.id = dev;
+  if (cudaMemPoolCreate(&p, &props) != cudaSuccess) return nullptr;
+  uint64_t keep = UINT64_MAX;
+  cudaMemPoolSetAttribute(p, cudaMemPoolAttrReleaseThreshold, &keep);
+  cudaMemPool_t expected = nullptr;
+  if (!g_pool[dev].compare_exchange_strong(expected, p)) {
+    cudaMemPoolDestroy(p);
+    p = expected;
+  }
+  return p;
+}
+
+cudaError_t pool_alloc(void** ptr, size_t bytes, cudaStream_t st) {
+  cudaMemPool_t pool = lib_pool();
+  if (!pool) return cudaErrorMemoryAllocation;
+  return cudaMallocFromPoolAsync(ptr, bytes, pool, st);
+}
 
 int64_t nstate_rows(const ssd_shape* s, const int32_t* cu) { return cu ? s->nseq : s->batch; }
 
@@ -161,7 +192,7 @@ int forward_impl(const ssd_shape* s, const void* x, const float* dt, const float
 
   const Scratch w = scratch_layout(s, cu, chunk, path);
   char* ws = nullptr;
-  if (cudaMallocAsync((void**)&ws, w.total, st) != cudaSuccess) return SSD_ERR_CUDA;
+  if (pool_alloc((void**)&ws, w.total, st) != cudaSuccess) return SSD_ERR_CUDA;
   pb.chunks = (ssd::ChunkRec*)(ws + w.table);
   pb.seq_first = (int32_t*)(ws + w.seq_first);
   pb.nchunks = (int32_t*)(ws + w.nchunks);
@@ -208,48 +239,142 @@ int ssd_forward_host(const ssd_shape* s, const void* x, const float* dt, const f
   const int64_t nseq = nstate_rows(s, cu_seqlens);
   const size_t es = s->io_dtype == SSD_BF16 ? 2 : 4;
   const size_t H = (size_t)s->nheads, P = (size_t)s->headdim, N = (size_t)s->dstate, G = (size_t)s->ngroups;
-  const size_t bytes[10] = {
-      (size_t)tokens * H * P * es,                 // x
-      (size_t)tokens * H * 4,                      // dt
-      H * 4,                                       // A
-      (size_t)tokens * G * N * es,                 // B
-      (size_t)tokens * G * N * es,                 // C
-      D ? H * 4 : 0,                               // D
-      init_state ? (size_t)nseq * H * P * N * 4 : 0,  // init
-      cu_seqlens ? (size_t)(nseq + 1) * 4 : 0,     // cu_seqlens
-      (size_t)tokens * H * P * es,                 // y
-      final_state ? (size_t)nseq * H * P * N * 4 : 0,  // final
+  const size_t tok_x = H * P * es, tok_dt = H * 4, tok_bc = G * N * es, seq_state = H * P * N * 4;
+  if (cu_seqlens && s->cu_seqlens_host != cu_seqlens) {  // the host array is the one to check
+    ssd_shape chk = *s;
+    chk.cu_seqlens_host = cu_seqlens;
+    if ((rc = validate(&chk, x, dt, A, B, C, cu_seqlens, chunk, y))) return rc;
+  }
+  auto seq_start = [&](int64_t q) -> int64_t { return cu_seqlens ? cu_seqlens[q] : q * s->seqlen; };
+
+  // Whole sequences in up to kGroups groups of about equal token counts: group g's
+  // inputs are copied in while group g-1 computes and group g-2's outputs go out.
+  constexpr int kGroups = 8;
+  std::vector<int64_t> gs{0};
+  for (int g = 1; g <= kGroups && gs.back() < nseq; ++g) {
+    const int64_t target = tokens * g / kGroups;
+    int64_t q = gs.back() + 1;
+    while (q < nseq && seq_start(q) < target) ++q;
+    gs.push_back(g == kGroups ? nseq : q);
+  }
+  if (gs.back() < nseq) gs.back() = nseq;
+  const int ng = (int)gs.size() - 1;
+
+  // Device buffers for the whole problem.  Each group's slice of a per-token or
+  // per-sequence array starts on a 256-byte boundary (the kernels need 16).
+  auto up = [](size_t v) { return (v + 255) & ~(size_t)255; };
+  std::vector<size_t> seq_off(ng + 1, 0), cu_off(ng + 1, 0);
+  for (int g = 0; g < ng; ++g) {
+    const int64_t q0 = gs[g], q1 = gs[g + 1];
+    seq_off[g + 1] = seq_off[g] + up((size_t)(q1 - q0) * seq_state);
+    cu_off[g + 1] = cu_off[g] + ((size_t)(q1 - q0 + 1 + 63) & ~(size_t)63);  // int32 entries
+  }
+  // per-token arrays: the group's first token index in a padded token space, so that
+  // every slice is aligned for every per-token row size
+  std::vector<int64_t> ptok(ng + 1, 0);
+  for (int g = 0; g < ng; ++g) {
+    const int64_t nt = (gs[g + 1] < nseq ? seq_start(gs[g + 1]) : tokens) - seq_start(gs[g]);
+    ptok[g + 1] = ptok[g] + ((nt + 255) & ~(int64_t)255);
+  }
+  const int64_t ptokens = ptok[ng];
+  const size_t bytes[11] = {
+      (size_t)ptokens * tok_x,                                 // x
+      (size_t)ptokens * tok_dt,                                // dt
+      H * 4,                                                   // A
+      (size_t)ptokens * tok_bc,                                // B
+      (size_t)ptokens * tok_bc,                                // C
+      D ? H * 4 : 0,                                           // D
+      init_state ? seq_off[ng] : 0,                            // init
+      cu_seqlens ? cu_off[ng] * 4 : 0,                         // each group's cu_seqlens from 0
+      (size_t)ptokens * tok_x,                                 // y
+      final_state ? seq_off[ng] : 0,                           // final
+      0,
   };
-  const void* hin[8] = {x, dt, A, B, C, D, init_state, cu_seqlens};
-  void* dev[10] = {};
+  void* dev[11] = {};
+  cudaStream_t sin = nullptr, sout = nullptr;
+  std::vector<cudaEvent_t> ev;
   auto cleanup = [&]() {
+    if (sin) cudaStreamSynchronize(sin);
+    if (sout) cudaStreamSynchronize(sout);
     for (void* p : dev)
       if (p) cudaFreeAsync(p, st);
+    for (cudaEvent_t e : ev) cudaEventDestroy(e);
+    if (sin) cudaStreamDestroy(sin);
+    if (sout) cudaStreamDestroy(sout);
   };
-  for (int i = 0; i < 10; ++i) {
-    if (!bytes[i]) continue;
-    if (cudaMallocAsync(&dev[i], bytes[i], st) != cudaSuccess) {
-      cleanup();
-      return SSD_ERR_CUDA;
-    }
+  auto fail = [&](int code) {
+    cleanup();
+    cudaStreamSynchronize(st);
+    return code;
+  };
+  for (int i = 0; i < 10; ++i)
+    if (bytes[i] && pool_alloc(&dev[i], bytes[i], st) != cudaSuccess) return fail(SSD_ERR_CUDA);
+  if (cudaStreamCreateWithFlags(&sin, cudaStreamNonBlocking) != cudaSuccess ||
+      cudaStreamCreateWithFlags(&sout, cudaStreamNonBlocking) != cudaSuccess)
+    return fail(SSD_ERR_CUDA);
+  ev.resize(2 * ng + 1, nullptr);
+  for (auto& e : ev)
+    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return fail(SSD_ERR_CUDA);
+  // the buffers were taken on `st`: the copy streams start after that
+  if (cudaEventRecord(ev[2 * ng], st) != cudaSuccess || cudaStreamWaitEvent(sin, ev[2 * ng], 0) != cudaSuccess ||
+      cudaStreamWaitEvent(sout, ev[2 * ng], 0) != cudaSuccess)
+    return fail(SSD_ERR_CUDA);
+
+  std::vector<int32_t> cu_groups;  // host copy of each group's cu_seqlens, rebased to 0
+  if (cu_seqlens) {
+    cu_groups.assign(cu_off[ng], 0);
+    for (int g = 0; g < ng; ++g)
+      for (int64_t q = gs[g]; q <= gs[g + 1]; ++q)
+        cu_groups[cu_off[g] + (q - gs[g])] = cu_seqlens[q] - cu_seqlens[gs[g]];
   }
-  for (int i = 0; i < 8; ++i) {
-    if (!bytes[i]) continue;
-    if (cudaMemcpyAsync(dev[i], hin[i], bytes[i], cudaMemcpyHostToDevice, st) != cudaSuccess) {
-      cleanup();
-      return SSD_ERR_CUDA;
+  auto h2d = [&](void* d, const void* h, size_t n) {
+    return n == 0 || cudaMemcpyAsync(d, h, n, cudaMemcpyHostToDevice, sin) == cudaSuccess;
+  };
+  auto d2h = [&](void* h, const void* d, size_t n) {
+    return n == 0 || cudaMemcpyAsync(h, d, n, cudaMemcpyDeviceToHost, sout) == cudaSuccess;
+  };
+  if (!h2d(dev[2], A, bytes[2]) || !h2d(dev[5], D, bytes[5]) ||
+      (cu_seqlens && !h2d(dev[7], cu_groups.data(), bytes[7])))
+    return fail(SSD_ERR_CUDA);
+  if (cu_seqlens && cudaStreamSynchronize(sin) != cudaSuccess) return fail(SSD_ERR_CUDA);  // pageable source
+
+  auto at = [](void* base, size_t off) { return base ? (void*)((char*)base + off) : nullptr; };
+  for (int g = 0; g < ng && rc == SSD_OK; ++g) {
+    const int64_t q0 = gs[g], q1 = gs[g + 1];
+    const int64_t t0 = seq_start(q0), t1 = q1 < nseq ? seq_start(q1) : tokens, nt = t1 - t0;
+    const size_t p0 = (size_t)ptok[g];  // first token of the group in the device buffers
+    const char* hx = (const char*)x;
+    if (!h2d(at(dev[0], p0 * tok_x), hx + t0 * tok_x, nt * tok_x) ||
+        !h2d(at(dev[1], p0 * tok_dt), (const char*)dt + t0 * tok_dt, nt * tok_dt) ||
+        !h2d(at(dev[3], p0 * tok_bc), (const char*)B + t0 * tok_bc, nt * tok_bc) ||
+        !h2d(at(dev[4], p0 * tok_bc), (const char*)C + t0 * tok_bc, nt * tok_bc) ||
+        (init_state && !h2d(at(dev[6], seq_off[g]), (const char*)init_state + q0 * seq_state,
+                            (q1 - q0) * seq_state)) ||
+        cudaEventRecord(ev[2 * g], sin) != cudaSuccess || cudaStreamWaitEvent(st, ev[2 * g], 0) != cudaSuccess) {
+      rc = SSD_ERR_CUDA;
+      break;
     }
+    ssd_shape sg = *s;
+    if (cu_seqlens) {
+      sg.batch = 1;
+      sg.seqlen = nt;
+      sg.nseq = q1 - q0;
+      sg.cu_seqlens_host = nullptr;  // validated above
+    } else {
+      sg.batch = q1 - q0;
+      sg.cu_seqlens_host = nullptr;
+    }
+    rc = forward_impl(&sg, at(dev[0], p0 * tok_x), (const float*)at(dev[1], p0 * tok_dt), (const float*)dev[2],
+                      at(dev[3], p0 * tok_bc), at(dev[4], p0 * tok_bc), (const float*)dev[5],
+                      (const float*)at(dev[6], seq_off[g]),
+                      cu_seqlens ? (const int32_t*)dev[7] + cu_off[g] : nullptr, chunk, at(dev[8], p0 * tok_x),
+                      (float*)at(dev[9], seq_off[g]), st);
+    if (rc != SSD_OK) break;
+    if (cudaEventRecord(ev[2 * g + 1], st) != cudaSuccess || cudaStreamWaitEvent(sout, ev[2 * g + 1], 0) != cudaSuccess ||
+        !d2h((char*)y + t0 * tok_x, at(dev[8], p0 * tok_x), nt * tok_x) ||
+        (final_state && !d2h((char*)final_state + q0 * seq_state, at(dev[9], seq_off[g]), (q1 - q0) * seq_state)))
+      rc = SSD_ERR_CUDA;
   }
-  ssd_shape sd = *s;
-  sd.cu_seqlens_host = nullptr;  // validated above
-  rc = forward_impl(&sd, dev[0], (const float*)dev[1], (const float*)dev[2], dev[3], dev[4],
-                    (const float*)dev[5], (const float*)dev[6], (const int32_t*)dev[7], chunk, dev[8],
-                    (float*)dev[9], st);
-  if (rc == SSD_OK && bytes[8] && cudaMemcpyAsync(y, dev[8], bytes[8], cudaMemcpyDeviceToHost, st) != cudaSuccess)
-    rc = SSD_ERR_CUDA;
-  if (rc == SSD_OK && bytes[9] &&
-      cudaMemcpyAsync(final_state, dev[9], bytes[9], cudaMemcpyDeviceToHost, st) != cudaSuccess)
-    rc = SSD_ERR_CUDA;
   cleanup();
   if (cudaStreamSynchronize(st) != cudaSuccess) return SSD_ERR_CUDA;
   if (rc != SSD_OK) return rc;

@@ -85,7 +85,6 @@ constexpr uint32_t kTmemCols = 512;
 // decay in place and the right-factor MMA accumulates B^T (w o x) onto it.
 constexpr uint32_t kColS = 0, kColP = 128, kColY = 256, kColSt = 384;
 constexpr long long kWaitLimit = 4ll << 30;  // SM cycles (about 2 s) before a wait gives up
-constexpr uint32_t kSuspendHintNs = 1000;    // a waiting thread sleeps until the phase completes, at most 1 us per try
 constexpr uint32_t kAtom = kTile * 128;      // one 128-row x 128-byte swizzled operand column
 
 // mbarriers.  Issuer -> compute: tile loads (tx bytes) and UMMA commits.
@@ -274,7 +273,7 @@ __device__ __forceinline__ void warp_arrive(uint64_t* bar) {
 __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
-  while (!mbar_try_wait_sleep(bar, parity, kSuspendHintNs)) {
+  while (!mbar_try_wait(bar, parity)) {
     if (*abort_flag) return false;
     if (clock64() - t0 > kWaitLimit) {
       *abort_flag = 1;

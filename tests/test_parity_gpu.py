@@ -138,6 +138,23 @@ def test_host_entry_point_matches_device():
     assert torch.equal(yh, y.cpu()) and torch.equal(fh, fin.cpu())
 
 
+@pytest.mark.parametrize("lengths", [None, [700, 0, 1, 300, 129, 2048, 64, 5, 900, 33]], ids=["dense", "packed"])
+def test_host_entry_point_groups_match_device(lengths):
+    """The host entry point copies in, computes and copies out by groups of whole sequences;
+    every sequence's outputs equal the single device call's bit for bit."""
+    if lengths is None:
+        wl = workloads.custom(6, 500, H=8, P=64, N=128, G=2, chunk=256, dtype="bf16", init=True)
+        prob = workloads.generate(wl, seed=11)
+    else:
+        wl = workloads.custom(1, 0, H=8, P=64, N=64, G=1, chunk=128, dtype="bf16", init=True, lengths=lengths)
+        prob = workloads.generate(wl, seed=11, lengths=lengths)
+    y, fin = run(prob, chunk=wl.chunk)
+    pin = lambda t: None if t is None else t.pin_memory()
+    yh, fh = ssd.ssd_forward_host(pin(prob.x), pin(prob.dt), pin(prob.A), pin(prob.B), pin(prob.C), pin(prob.D),
+                                  pin(prob.init_state), pin(prob.cu_seqlens), chunk=wl.chunk)
+    assert torch.equal(yh, y.cpu()) and torch.equal(fh, fin.cpu())
+
+
 def test_bad_device_seqlens_sets_status_and_writes_nothing():
     wl = workloads.custom(1, 300, H=4, P=64, N=64, G=1, chunk=128, dtype="bf16", lengths=[100, 200])
     prob = workloads.generate(wl, seed=8, lengths=[100, 200])
