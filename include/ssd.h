@@ -22,8 +22,10 @@
  *    must be 16-byte aligned.  The caller owns every buffer; the library keeps
  *    no pointer after the call returns.
  *  - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
- *    stream) unless stated otherwise.  Scratch memory, when needed, comes from
- *    the stream-ordered allocator (cudaMallocAsync / cudaFreeAsync on `stream`).
+ *    stream) unless stated otherwise.  Scratch memory, when needed, comes from a
+ *    stream-ordered pool the library creates per device (cudaMallocFromPoolAsync
+ *    / cudaFreeAsync on `stream`); freed blocks stay in that pool for later calls
+ *    and are returned to the driver when the process exits.
  *  - The return value is an ssd_status.  On any host-detected error nothing is
  *    launched and no output is written.  Errors found on the device (bad
  *    cu_seqlens values, a bounded wait that ran out) are recorded in a per-device
@@ -96,11 +98,15 @@ int ssd_forward(const ssd_shape* shape, const void* x, const float* dt, const fl
 
 /*
  * ssd_forward_host -- the same computation on HOST buffers (pinned memory gives full
- * copy bandwidth).  Device buffers are taken from the stream-ordered allocator, the
- * inputs are copied in, ssd_forward runs, the outputs are copied back, and the call
- * synchronises `stream` before returning.  Same layouts and errors as ssd_forward;
- * cu_seqlens is a host pointer here.  Returns SSD_ERR_DEVICE_TIMEOUT or
- * SSD_ERR_BAD_SEQLENS when the device reported one during this call.
+ * copy bandwidth; pageable memory works but its copies do not overlap).  The
+ * sequences are split into up to 8 groups of whole sequences with about equal token
+ * counts; device buffers come from the library's pool; group g's inputs are copied in
+ * on one library stream while group g-1 runs ssd_forward on `stream` and group g-2's
+ * outputs are copied back on another, and the call synchronises all of them before
+ * returning.  Every sequence's outputs are the ones a single ssd_forward call gives.
+ * Same layouts and errors as ssd_forward; cu_seqlens is a host pointer here and is
+ * checked on the host (SSD_ERR_BAD_SEQLENS).  Returns SSD_ERR_DEVICE_TIMEOUT when the
+ * device reported one during this call.
  */
 int ssd_forward_host(const ssd_shape* shape, const void* x, const float* dt, const float* A, const void* B,
                      const void* C, const float* D, const float* init_state, const int32_t* cu_seqlens, int chunk,
