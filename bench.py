@@ -341,9 +341,50 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": int(launches),
         "clocks": clocks,
     }
+    if world == 1 and not args.no_decode:
+        out["next"] = {"decode_step": decode_measurement(dev, stream, flush)}
     if world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(prob, budget_s=args.cpu_budget)
     return out
+
+
+# ------------------------------------------------------- decode step (next row)
+DECODE = workloads.custom(64, 1, H=80, P=64, N=128, G=1, chunk=64, dtype="bf16", init=True,
+                          name="decode_step_b64_H80_P64_N128_bf16")
+
+
+def decode_measurement(dev, stream, flush, reps: int = 20):
+    """One recurrent decode step for 64 sequences at the Mamba-2-2.7B layer shape: the fp32
+    state (168 MB, larger than L2) is read and written once.  Median of ``reps`` launches,
+    CUDA events on the launching stream, L2 flushed between launches."""
+    import ssd_sequence_mixing_b200 as ssd
+
+    wl = DECODE
+    prob = workloads.generate(wl, seed=0)
+    x, dt, B, C = (getattr(prob, k)[:, 0].contiguous().to(dev) for k in ("x", "dt", "B", "C"))
+    A, D = prob.A.to(dev), prob.D.to(dev)
+    state = prob.init_state.to(dev)
+    y = torch.empty_like(x)
+    for _ in range(3):
+        ssd.ssd_decode_step(x, dt, A, B, C, D, state, y=y, stream=stream)
+    ms = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        ssd.ssd_decode_step(x, dt, A, B, C, D, state, y=y, stream=stream)
+        b.record(stream)
+        ms.append((a, b))
+    torch.cuda.synchronize()
+    t = statistics.median(a.elapsed_time(b) for a, b in ms) / 1e3
+    rows, H, P, N, G = wl.batch, wl.nheads, wl.headdim, wl.dstate, wl.ngroups
+    nbytes = rows * H * P * N * 4 * 2 + rows * H * P * 2 * 2 + rows * G * N * 2 * 2 + rows * H * 4
+    peaks, kind = load_peaks()
+    gbs = nbytes / t / 1e9
+    return {"workload": wl.name, "us": t * 1e6, "tokens_per_s": rows / t, "algorithmic_bytes": nbytes,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "peak_source": f"{kind} (GB/s)"},
+            "l2": "flushed between launches; the state alone exceeds L2"}
 
 
 # ------------------------------------------------------------ reference arm
@@ -385,6 +426,7 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-decode", action="store_true", help="skip the decode-step measurement")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--ref-heads", type=int, default=16)
     args = ap.parse_args()

@@ -97,6 +97,29 @@ int ssd_forward(const ssd_shape* shape, const void* x, const float* dt, const fl
                 void* y, float* final_state, ssd_stream_t stream);
 
 /*
+ * ssd_forward_dt -- ssd_forward with the step size made inside the kernels from the raw
+ * per-head projection, as the pages' discretisation does it (the wikillm.com card: the
+ * Mamba-2 block sketch of sec. 7.1, Method note 7 "Discretisation", "Paper vs code" 7:
+ * dt = softplus(dt_raw + dt_bias)).  Every kernel that reads dt applies, per token t
+ * and head h,
+ *     v  = dt_raw[t,h] + (dt_bias ? dt_bias[h] : 0)
+ *     dt = softplus ? log(1 + exp(v)) : v,   then clamped to [dt_min, dt_max]
+ * so no separate pass over dt precedes the call.  `dt_raw` has dt's layout (batch,
+ * seqlen, H) fp32; dt_bias is (H) fp32 on the device or NULL; use dt_min = 0 and
+ * dt_max = INFINITY for no clamp.  prologue == NULL is ssd_forward.  Errors as
+ * ssd_forward, plus SSD_ERR_INVALID_ARG for dt_min < 0, dt_max < dt_min or a NaN bound
+ * and SSD_ERR_MISALIGNED for a dt_bias not 16-byte aligned.
+ */
+typedef struct {
+  const float* dt_bias;  /* (H) fp32 device pointer, or NULL (= 0) */
+  int softplus;          /* 1: dt = softplus(dt_raw + dt_bias); 0: dt = dt_raw + dt_bias */
+  float dt_min, dt_max;  /* clamp after softplus */
+} ssd_dt_prologue;
+int ssd_forward_dt(const ssd_shape* shape, const ssd_dt_prologue* prologue, const void* x, const float* dt_raw,
+                   const float* A, const void* B, const void* C, const float* D, const float* init_state,
+                   const int32_t* cu_seqlens, int chunk, void* y, float* final_state, ssd_stream_t stream);
+
+/*
  * ssd_forward_host -- the same computation on HOST buffers (pinned memory gives full
  * copy bandwidth; pageable memory works but its copies do not overlap).  The
  * sequences are split into up to 8 groups of whole sequences with about equal token
@@ -142,6 +165,31 @@ int ssd_forward_host(const ssd_shape* shape, const void* x, const float* dt, con
 int ssd_forward_noalloc(const ssd_shape* shape, const void* x, const float* dt, const float* A, const void* B,
                         const void* C, const float* D, const float* init_state, const int32_t* cu_seqlens,
                         int chunk, void* y, float* final_state, ssd_stream_t stream);
+
+/*
+ * ssd_decode_step -- one recurrent generation step for a batch of sequences (the
+ * wikillm.com card, Method step 8 and sec. 6.3: in generation the layer runs as its
+ * linear recurrence, N^2 work per token and head).  For every row b and head h, with
+ * g = h / (H/G) and the fp32 state S = state[b,h] (P x N, N contiguous), in place:
+ *   a = exp(dt[b,h] A[h]);  S <- a S + dt[b,h] x[b,h,:] B[b,g,:]^T;
+ *   y[b,h,:] = S C[b,g,:] + D[h] x[b,h,:]
+ * This is the same recurrence ssd_forward evaluates in chunks, one token at a time:
+ * T steps from init_state give ssd_forward's y rows and final_state.
+ *
+ *   shape       batch = rows, seqlen = 1, nheads H, headdim P, dstate N (N % 4 == 0,
+ *               N <= 256), ngroups G; io_dtype for x, B, C, y; nseq and
+ *               cu_seqlens_host unused
+ *   x, y        (batch, H, P)       io_dtype
+ *   dt          (batch, H)          fp32, > 0
+ *   A, D        (H)                 fp32 (D may be NULL = 0)
+ *   B, C        (batch, G, N)       io_dtype
+ *   state       (batch, H, P, N)    fp32, read and overwritten
+ * Device pointers, 16-byte aligned; no scratch; asynchronous on `stream`.  Errors:
+ * SSD_ERR_INVALID_ARG (null pointer, seqlen != 1), SSD_ERR_UNSUPPORTED (N % 4, N > 256,
+ * H % G), SSD_ERR_MISALIGNED, SSD_ERR_CUDA; nothing is launched on an error.
+ */
+int ssd_decode_step(const ssd_shape* shape, const void* x, const float* dt, const float* A, const void* B,
+                    const void* C, const float* D, float* state, void* y, ssd_stream_t stream);
 
 /* Bytes of stream-ordered scratch ssd_forward takes for this shape (informational). */
 size_t ssd_workspace_bytes(const ssd_shape* shape, int chunk);

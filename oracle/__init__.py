@@ -11,6 +11,8 @@ leg may import this package.  It shares no code with the CUDA path.
 * ``chunked.ssd_chunked``: the pages' chunked algorithm restated in numpy
   (Method step 5, sec. 6), used to pin the recurrence.
 * ``decode_step``: one recurrent generation step (Method step 8, sec. 6.3).
+* ``dt_prologue``: the step size from the raw projection, dt = softplus(raw + bias)
+  (the Mamba-2 block sketch of sec. 7.1 and Method note 7 "Discretisation").
 
 Parity status of every function here is recorded in the tests that pin it.
 """
@@ -161,6 +163,15 @@ def ssd_forward_problem(prob, pairs: Optional[Iterable[Tuple[int, int]]] = None,
             y[offs[s]:offs[s + 1], h] = ys[sub_offs[si]:sub_offs[si + 1], hi]
             fin[s, h] = fs[si, hi]
     return y, fin
+
+
+def dt_prologue(dt_raw, dt_bias=None, softplus: bool = True, dt_min: float = 0.0, dt_max: float = np.inf):
+    """The pages' discretisation of the step size, in fp64: v = dt_raw + dt_bias (bias per head,
+    the last axis), dt = log(1 + exp(v)) when ``softplus``, then clamped to [dt_min, dt_max]."""
+    v = _f64(dt_raw) + (0.0 if dt_bias is None else _f64(dt_bias))
+    if softplus:
+        v = np.logaddexp(0.0, v)  # log(exp(0) + exp(v)) = log(1 + exp(v))
+    return np.clip(v, dt_min, dt_max)
 
 
 def decode_step(x, dt, A, B, C, D, state):

@@ -43,7 +43,18 @@ EXPORTS = (
     "ssd_profile_dominant",
     "ssd_kernel_launch_count",
     "ssd_forward_noalloc",
+    "ssd_decode_step",
+    "ssd_forward_dt",
 )
+
+
+class SsdDtPrologue(ctypes.Structure):
+    _fields_ = [
+        ("dt_bias", ctypes.c_void_p),
+        ("softplus", ctypes.c_int),
+        ("dt_min", ctypes.c_float),
+        ("dt_max", ctypes.c_float),
+    ]
 
 
 class SsdShape(ctypes.Structure):
@@ -89,6 +100,10 @@ def _open() -> ctypes.CDLL:
     lib.ssd_profile_dominant.restype = I
     lib.ssd_kernel_launch_count.argtypes = []
     lib.ssd_kernel_launch_count.restype = ctypes.c_uint64
+    lib.ssd_decode_step.argtypes = [SP, V, V, V, V, V, V, V, V, V]
+    lib.ssd_decode_step.restype = I
+    lib.ssd_forward_dt.argtypes = [SP, ctypes.POINTER(SsdDtPrologue)] + fwd[1:]
+    lib.ssd_forward_dt.restype = I
     return lib
 
 
@@ -218,6 +233,68 @@ def ssd_forward_noalloc(x, dt, A, B, C, D=None, init_state=None, cu_seqlens=None
     if rc:
         raise SsdError(rc, "ssd_forward_noalloc")
     return y, final_state
+
+
+def ssd_forward_dt(x, dt_raw, A, B, C, D=None, init_state=None, cu_seqlens=None, chunk: int = 256,
+                   dt_bias: Optional[torch.Tensor] = None, softplus: bool = True, dt_min: float = 0.0,
+                   dt_max: float = float("inf"), y: Optional[torch.Tensor] = None,
+                   final_state: Optional[torch.Tensor] = None, return_final: bool = True, stream=None):
+    """ssd_forward with the step size made inside the kernels: dt = clamp(softplus(dt_raw +
+    dt_bias), dt_min, dt_max) per token and head (softplus=False skips the softplus)."""
+    device = x.device
+    if device.type != "cuda":
+        raise ValueError("ssd_forward_dt takes CUDA tensors")
+    y, final_state = _prepare(x, dt_raw, A, B, C, D, init_state, cu_seqlens, y, final_state, return_final, device)
+    _check("dt_bias", dt_bias, device, torch.float32, (x.shape[2],))
+    pro = SsdDtPrologue(None if dt_bias is None else dt_bias.data_ptr(), int(bool(softplus)), float(dt_min),
+                        float(dt_max))
+    shape = make_shape(x, B, cu_seqlens)
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    with torch.cuda.device(device):
+        rc = _lib.ssd_forward_dt(ctypes.byref(shape), ctypes.byref(pro), _ptr(x), _ptr(dt_raw), _ptr(A), _ptr(B),
+                                 _ptr(C), _ptr(D), _ptr(init_state), _ptr(cu_seqlens), int(chunk), _ptr(y),
+                                 _ptr(final_state), ctypes.c_void_p(handle))
+    if rc:
+        raise SsdError(rc, "ssd_forward_dt")
+    return y, final_state
+
+
+def ssd_decode_step(x, dt, A, B, C, D, state, y: Optional[torch.Tensor] = None, stream=None):
+    """One recurrent generation step for a batch of sequences, state updated in place.
+
+    x (batch, H, P) and B, C (batch, G, N) in float32 or bfloat16; dt (batch, H), A and D (H,)
+    float32 (D may be None); state (batch, H, P, N) float32 on the same device.  Returns y
+    (batch, H, P) in x's dtype.
+    """
+    device = x.device
+    if device.type != "cuda":
+        raise ValueError("ssd_decode_step takes CUDA tensors")
+    if x.dim() != 3 or B.dim() != 3:
+        raise ValueError("x must be (batch, H, P) and B, C (batch, G, N)")
+    batch, H, P = x.shape
+    G, N = B.shape[1], B.shape[2]
+    _check("x", x, device)
+    _check("dt", dt, device, torch.float32, (batch, H))
+    _check("A", A, device, torch.float32, (H,))
+    _check("B", B, device, x.dtype, (batch, G, N))
+    _check("C", C, device, x.dtype, (batch, G, N))
+    _check("D", D, device, torch.float32, (H,))
+    _check("state", state, device, torch.float32, (batch, H, P, N))
+    if y is None:
+        y = torch.empty_like(x)
+    _check("y", y, device, x.dtype, (batch, H, P))
+    shape = SsdShape(batch, 1, H, P, N, G, 0, _io_code(x.dtype), None)
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    with torch.cuda.device(device):
+        rc = _lib.ssd_decode_step(ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), _ptr(C), _ptr(D),
+                                  _ptr(state), _ptr(y), ctypes.c_void_p(handle))
+    if rc:
+        raise SsdError(rc, "ssd_decode_step")
+    return y
 
 
 def ssd_forward_host(x, dt, A, B, C, D=None, init_state=None, cu_seqlens=None, chunk: int = 256, y=None,

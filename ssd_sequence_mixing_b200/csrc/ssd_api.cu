@@ -149,10 +149,11 @@ int select_path(const ssd_shape* s, int chunk) {
 
 int forward_impl(const ssd_shape* s, const void* x, const float* dt, const float* A, const void* B, const void* C,
                  const float* D, const float* init, const int32_t* cu, int chunk, void* y, float* fin,
-                 cudaStream_t st) {
+                 cudaStream_t st, const ssd_dt_prologue* pro = nullptr) {
   int rc = validate(s, x, dt, A, B, C, cu, chunk, y);
   if (rc) return rc;
-  const void* ptrs[] = {x, dt, A, B, C, D, init, cu, y, fin};
+  if (pro && !(pro->dt_min >= 0.f && pro->dt_max >= pro->dt_min)) return SSD_ERR_INVALID_ARG;  // NaN fails too
+  const void* ptrs[] = {x, dt, A, B, C, D, init, cu, y, fin, pro ? pro->dt_bias : nullptr};
   for (const void* p : ptrs)
     if (p && !aligned16(p)) return SSD_ERR_MISALIGNED;
   const int path = select_path(s, chunk);
@@ -186,6 +187,13 @@ int forward_impl(const ssd_shape* s, const void* x, const float* dt, const float
   pb.final_state = fin;
   pb.status = status;
   pb.Cmax = ssd::max_chunks(tokens, (int)nseq, chunk);
+  if (pro) {
+    pb.dt_prologue = 1;
+    pb.dt_softplus = pro->softplus != 0;
+    pb.dt_bias = pro->dt_bias;
+    pb.dt_min = pro->dt_min;
+    pb.dt_max = pro->dt_max;
+  }
   pb.prof_start = g_prof_start.load();
   pb.prof_stop = g_prof_stop.load();
   if (!pb.prof_start || !pb.prof_stop) pb.prof_start = pb.prof_stop = nullptr;
@@ -227,6 +235,13 @@ int ssd_forward(const ssd_shape* shape, const void* x, const float* dt, const fl
                 void* y, float* final_state, ssd_stream_t stream) {
   return forward_impl(shape, x, dt, A, B, C, D, init_state, cu_seqlens, chunk, y, final_state,
                       (cudaStream_t)stream);
+}
+
+int ssd_forward_dt(const ssd_shape* shape, const ssd_dt_prologue* prologue, const void* x, const float* dt_raw,
+                   const float* A, const void* B, const void* C, const float* D, const float* init_state,
+                   const int32_t* cu_seqlens, int chunk, void* y, float* final_state, ssd_stream_t stream) {
+  return forward_impl(shape, x, dt_raw, A, B, C, D, init_state, cu_seqlens, chunk, y, final_state,
+                      (cudaStream_t)stream, prologue);
 }
 
 int ssd_forward_host(const ssd_shape* s, const void* x, const float* dt, const float* A, const void* B,

@@ -50,7 +50,21 @@ struct Problem {
   int ranges;          // CTAs of the tensor-core launch
   // host-side measurement hooks (events around the dominant kernel, or null)
   cudaEvent_t prof_start, prof_stop;
+  // fused dt prologue (ssd_forward_dt): dt holds the raw values, see dt_value()
+  int dt_prologue, dt_softplus;
+  const float* dt_bias;  // (H) or null
+  float dt_min, dt_max;
 };
+
+// The step size of head h from the stored value v: v itself, or with the fused prologue
+// of the pages' discretisation clamp(softplus(v + dt_bias[h]), dt_min, dt_max)
+// (softplus(v) = log(1 + exp(v)), evaluated as max(v, 0) + log1p(exp(-|v|))).
+__device__ __forceinline__ float dt_value(const Problem& pb, float v, int h) {
+  if (!pb.dt_prologue) return v;
+  if (pb.dt_bias) v += pb.dt_bias[h];
+  if (pb.dt_softplus) v = fmaxf(v, 0.f) + log1pf(expf(-fabsf(v)));
+  return fminf(fmaxf(v, pb.dt_min), pb.dt_max);
+}
 
 __device__ __forceinline__ int64_t seq_off(const Problem& pb, int s) {
   return pb.cu ? (int64_t)pb.cu[s] : (int64_t)s * pb.seqlen;

@@ -25,14 +25,13 @@ namespace ssd {
 // One block: validates cu_seqlens (0 = c0 <= ... <= c_nseq = tokens), then lays
 // out every sequence's chunks in sequence order.  On invalid input it records
 // kStatusBadSeqlens and sets nchunks = -1, and every later kernel does nothing.
+// The tensor-core path (seq_tiles set) needs only the prefix over 128-token tiles
+// and the validity flag; the SIMT path needs the chunk prefix and chunk records.
 __global__ void __launch_bounds__(1024) chunk_table_kernel(Problem pb) {
-  __shared__ int s_bad, s_carry;
-  __shared__ int s_scan[1024];
-  const int tid = threadIdx.x;
-  if (tid == 0) {
-    s_bad = 0;
-    s_carry = 0;
-  }
+  __shared__ int s_bad;
+  __shared__ int s_warp[32];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  if (tid == 0) s_bad = 0;
   __syncthreads();
   if (pb.cu) {
     for (int s = tid; s <= pb.nseq; s += blockDim.x) {
@@ -49,39 +48,45 @@ __global__ void __launch_bounds__(1024) chunk_table_kernel(Problem pb) {
     }
     return;
   }
-  // Two prefix sums over sequences: chunks of Q tokens (SIMT path) and, when the
-  // tensor-core path asked for it, tiles of kTcTile tokens.
-  for (int pass = 0; pass < (pb.seq_tiles ? 2 : 1); ++pass) {
-    const int unit = pass == 0 ? pb.Q : kTcTile;
-    int32_t* out = pass == 0 ? pb.seq_first : pb.seq_tiles;
-    if (tid == 0) s_carry = 0;
-    __syncthreads();
-    for (int base = 0; base < pb.nseq; base += blockDim.x) {
-      const int s = base + tid;
-      int n = 0;
-      if (s < pb.nseq) {
-        const int64_t len = seq_off(pb, s + 1) - seq_off(pb, s);
-        n = (int)((len + unit - 1) / unit);
-      }
-      s_scan[tid] = n;
-      __syncthreads();
-      for (int off = 1; off < (int)blockDim.x; off <<= 1) {
-        const int v = tid >= off ? s_scan[tid - off] : 0;
-        __syncthreads();
-        s_scan[tid] += v;
-        __syncthreads();
-      }
-      if (s < pb.nseq) out[s] = s_carry + s_scan[tid] - n;
-      __syncthreads();
-      if (tid == blockDim.x - 1) s_carry += s_scan[tid];
-      __syncthreads();
+  const bool tc = pb.seq_tiles != nullptr;
+  const int unit = tc ? kTcTile : pb.Q;
+  int32_t* out = tc ? pb.seq_tiles : pb.seq_first;
+  // exclusive prefix over sequences of ceil(len / unit), 1024 sequences at a time
+  int carry = 0;  // the same in every thread
+  for (int base = 0; base < pb.nseq; base += blockDim.x) {
+    const int s = base + tid;
+    int n = 0;
+    if (s < pb.nseq) {
+      const int64_t len = seq_off(pb, s + 1) - seq_off(pb, s);
+      n = (int)((len + unit - 1) / unit);
     }
-    if (tid == 0) {
-      out[pb.nseq] = s_carry;
-      if (pass == 0) *pb.nchunks = s_carry;
+    int v = n;  // inclusive scan within the warp
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, v, off);
+      if (lane >= off) v += u;
+    }
+    if (lane == 31) s_warp[warp] = v;
+    __syncthreads();
+    if (warp == 0) {
+      int w = lane < (int)(blockDim.x >> 5) ? s_warp[lane] : 0;
+#pragma unroll
+      for (int off = 1; off < 32; off <<= 1) {
+        const int u = __shfl_up_sync(0xffffffffu, w, off);
+        if (lane >= off) w += u;
+      }
+      s_warp[lane] = w;  // inclusive over warps
     }
     __syncthreads();
+    if (s < pb.nseq) out[s] = carry + (warp > 0 ? s_warp[warp - 1] : 0) + v - n;
+    carry += s_warp[31];
+    __syncthreads();  // s_warp is rewritten by the next round
   }
+  if (tid == 0) {
+    out[pb.nseq] = carry;
+    *pb.nchunks = tc ? 0 : carry;  // the tensor-core path reads only the validity flag
+  }
+  if (tc) return;
   for (int s = tid; s < pb.nseq; s += blockDim.x) {
     const int64_t off = seq_off(pb, s), len = seq_off(pb, s + 1) - off;
     const int first = pb.seq_first[s];  // written above by this same thread
@@ -119,7 +124,7 @@ __global__ void __launch_bounds__(256) chunk_cumsum_kernel(Problem pb) {
   for (int i = 0; i < 8; ++i) {
     const int q = lane * per + i;
     float l = 0.f;
-    if (i < per && q < r.len) l = pb.dt[((int64_t)r.t0 + q) * pb.H + h] * Ah;
+    if (i < per && q < r.len) l = dt_value(pb, pb.dt[((int64_t)r.t0 + q) * pb.H + h], h) * Ah;
     run += l;
     v[i] = run;
   }
@@ -166,7 +171,7 @@ __global__ void __launch_bounds__(256) chunk_states_kernel(Problem pb) {
       if (q < r.len) {
         const int64_t t = (int64_t)r.t0 + q;
         if (p0 + col < pb.P) {
-          const float w = expf(cs_end - cs[q]) * pb.dt[t * pb.H + h];
+          const float w = expf(cs_end - cs[q]) * dt_value(pb, pb.dt[t * pb.H + h], h);
           xv = w * to_f(x[(t * pb.H + h) * pb.P + p0 + col]);
         }
         if (n0 + col < pb.N) bv = to_f(Bm[(t * pb.G + g) * pb.N + n0 + col]);
@@ -295,7 +300,7 @@ __global__ void __launch_bounds__(256) chunk_output_kernel(Problem pb) {
     if (threadIdx.x < 64) {
       const int j = threadIdx.x;
       cs_col[j] = j < cols ? cs[col0 + j] : 0.f;
-      dt_col[j] = j < cols ? pb.dt[((int64_t)r.t0 + col0 + j) * pb.H + h] : 0.f;
+      dt_col[j] = j < cols ? dt_value(pb, pb.dt[((int64_t)r.t0 + col0 + j) * pb.H + h], h) : 0.f;
     }
     // scores S[t][j] = C_t . B_j, 4 x 4 per thread at (ty + 16 i, tx + 16 j)
     float sacc[4][4] = {};

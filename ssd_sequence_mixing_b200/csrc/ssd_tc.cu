@@ -893,7 +893,7 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t
 #pragma unroll
         for (int hh = 0; hh < kHeads; ++hh) {
           const float val = k == 0 ? v[hh][0] : k == 1 ? v[hh][1] : k == 2 ? v[hh][2] : v[hh][3];
-          dtt[hh][j] = j < left ? val : 0.f;
+          dtt[hh][j] = j < left ? dt_value(pb, val, h0 + hh) : 0.f;
         }
       }
     }

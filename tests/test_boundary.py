@@ -116,3 +116,48 @@ def test_workspace_bytes_grows_with_problem():
     assert 0 < small < big
     # the SIMT path keeps one fp32 P x N state per chunk and head
     assert big >= 2 * 16 * 4 * 64 * 128 * 4
+
+
+# ------------------------------------------------------------------ decode step
+def call_decode(s, **ptrs):
+    p = {k: FAKE for k in ("x", "dt", "A", "B", "C", "state", "y")}
+    p.update(ptrs)
+    v = lambda k: None if p.get(k) is None else ctypes.c_void_p(p[k])
+    return ssd.library().ssd_decode_step(ctypes.byref(s), v("x"), v("dt"), v("A"), v("B"), v("C"), v("D"),
+                                         v("state"), v("y"), None)
+
+
+def test_decode_rejects_before_launch():
+    assert call_decode(shape(seqlen=2)) == 1  # one token per row
+    assert call_decode(shape(seqlen=1, nheads=0)) == 1
+    assert call_decode(shape(seqlen=1, io_dtype=7)) == 1
+    assert call_decode(shape(seqlen=1, dstate=6)) == 2  # N % 4
+    assert call_decode(shape(seqlen=1, dstate=260)) == 2  # N > 256
+    assert call_decode(shape(seqlen=1, nheads=6, ngroups=4)) == 2  # H % G
+    for k in ("x", "dt", "A", "B", "C", "state", "y"):
+        assert call_decode(shape(seqlen=1), **{k: None}) == 1, k
+        assert call_decode(shape(seqlen=1), **{k: FAKE + 8}) == 3, k
+    assert call_decode(shape(seqlen=1), D=FAKE + 4) == 3
+    assert ssd.library().ssd_decode_step(None, *([None] * 8), None) == 1
+
+
+def test_decode_empty_batch_is_a_no_op():
+    assert call_decode(shape(seqlen=1, batch=0)) == 0
+
+
+# ------------------------------------------------------------------ dt prologue
+@pytest.mark.parametrize("bounds", [(-1.0, 1.0), (0.5, 0.1), (float("nan"), 1.0), (0.0, float("nan"))])
+def test_dt_prologue_bad_bounds(bounds):
+    pro = ssd.SsdDtPrologue(None, 1, bounds[0], bounds[1])
+    p = {k: ctypes.c_void_p(FAKE) for k in ("x", "dt", "A", "B", "C", "y")}
+    rc = ssd.library().ssd_forward_dt(ctypes.byref(shape()), ctypes.byref(pro), p["x"], p["dt"], p["A"], p["B"],
+                                      p["C"], None, None, None, 256, p["y"], None, None)
+    assert rc == 1
+
+
+def test_dt_prologue_misaligned_bias():
+    pro = ssd.SsdDtPrologue(FAKE + 4, 1, 0.0, float("inf"))
+    p = {k: ctypes.c_void_p(FAKE) for k in ("x", "dt", "A", "B", "C", "y")}
+    rc = ssd.library().ssd_forward_dt(ctypes.byref(shape()), ctypes.byref(pro), p["x"], p["dt"], p["A"], p["B"],
+                                      p["C"], None, None, None, 256, p["y"], None, None)
+    assert rc == 3

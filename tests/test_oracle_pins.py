@@ -233,6 +233,38 @@ def test_decode_steps_equal_dense_matrix():
         assert rel(ys[:, h], M @ x[:, h] + D[h] * x[:, h]) < 1e-12
 
 
+# ------------------------------------------------- step-size prologue (NEXT-1)
+def test_dt_prologue_closed_forms():
+    """softplus(0) = ln 2; softplus(ln(e - 1)) = 1; softplus(v) -> v for large v and
+    -> exp(v) for very negative v; the bias is per head (last axis); the clamp bounds."""
+    dt = oracle.dt_prologue(np.array([[0.0, math.log(math.e - 1.0), 40.0, -40.0]]))
+    assert dt[0, 0] == pytest.approx(math.log(2.0), rel=1e-15)
+    assert dt[0, 1] == pytest.approx(1.0, rel=1e-15)
+    assert dt[0, 2] == pytest.approx(40.0, rel=1e-15)
+    assert dt[0, 3] == pytest.approx(math.exp(-40.0), rel=1e-12)
+    raw = np.zeros((3, 2))
+    got = oracle.dt_prologue(raw, dt_bias=np.array([0.0, math.log(math.e ** 2 - 1.0)]))
+    assert np.allclose(got[:, 0], math.log(2.0)) and np.allclose(got[:, 1], 2.0)
+    assert np.array_equal(oracle.dt_prologue(raw + 0.3, softplus=False), raw + 0.3)
+    assert np.all(oracle.dt_prologue(raw, dt_min=0.9) == 0.9)
+    assert np.all(oracle.dt_prologue(raw, dt_max=0.25) == 0.25)
+
+
+def test_dt_prologue_forward_equals_forward_on_inverse_softplus():
+    """Raw values built with the inverse softplus ln(e^d - 1) of a chosen dt give the
+    forward pass on that dt (and a clamp gives the forward pass on the clamped dt)."""
+    rng = np.random.default_rng(31)
+    x, dt, A, B, C, D = rand_problem(rng, 40, 3, 5, 6, 1)
+    bias = rng.uniform(-0.5, 0.5, 3)
+    raw = np.log(np.expm1(dt)) - bias
+    y0, f0 = oracle.ssd_forward(x, dt, A, B, C, D)
+    y1, f1 = oracle.ssd_forward(x, oracle.dt_prologue(raw, bias), A, B, C, D)
+    assert np.allclose(y1, y0, rtol=1e-12, atol=1e-12) and np.allclose(f1, f0, rtol=1e-12, atol=1e-12)
+    y2, f2 = oracle.ssd_forward(x, np.full_like(dt, 0.2), A, B, C, D)
+    y3, f3 = oracle.ssd_forward(x, oracle.dt_prologue(raw, bias, dt_min=0.2, dt_max=0.2), A, B, C, D)
+    assert np.array_equal(y3, y2) and np.array_equal(f3, f2)
+
+
 # ------------------------------------------------------- workload generator
 def test_sampled_problem_matches_full():
     """The sampled-pairs harness returns exactly the full oracle's rows."""

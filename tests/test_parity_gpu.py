@@ -107,6 +107,37 @@ def test_tiny_dt_and_strong_decay():
             check(prob, y, fin)
 
 
+@pytest.mark.parametrize("case", [(2, 700, 4, 64, 128, 2, 256, "bf16", True, 1e-3, 0.3),
+                                  (1, 300, 3, 32, 16, 1, 64, "f32", True, 0.0, float("inf")),
+                                  (2, 260, 8, 64, 64, 2, 128, "bf16", False, 0.0, float("inf"))],
+                         ids=["bf16_softplus_clamp", "f32_softplus", "bf16_bias_only"])
+def test_fused_dt_prologue(case):
+    """ssd_forward_dt makes dt = clamp(softplus(dt_raw + dt_bias)) inside the kernels; the
+    oracle runs on the same raw values through its own fp64 prologue."""
+    b, T, H, P, N, G, Q, dtype, softplus, lo, hi = case
+    wl = workloads.custom(b, T, H, P, N, G, chunk=Q, dtype=dtype, init=True)
+    prob = workloads.generate(wl, seed=12)
+    rng = np.random.default_rng(12)
+    mean = -3.0 if softplus else 0.05
+    raw = torch.from_numpy(rng.normal(mean, 1.0 if softplus else 0.01, tuple(prob.dt.shape)).astype(np.float32))
+    bias = torch.from_numpy(rng.uniform(-1, 1, H).astype(np.float32) * (1.0 if softplus else 0.01))
+    if not softplus:
+        raw = raw.abs()
+    ref_dt = oracle.dt_prologue(raw.double().numpy(), bias.double().numpy(), softplus, lo, hi)
+    prob.dt = torch.from_numpy(ref_dt)  # the oracle reads dt from the problem (fp64 here)
+    dev = to_device(prob)
+    raw_d, bias_d = raw.cuda(), bias.cuda()
+    for name, path in paths_for(prob, Q):
+        old = ssd.set_path(path)
+        try:
+            y, fin = ssd.ssd_forward_dt(dev["x"], raw_d, dev["A"], dev["B"], dev["C"], dev["D"], dev["init_state"],
+                                        None, Q, dt_bias=bias_d, softplus=softplus, dt_min=lo, dt_max=hi)
+        finally:
+            ssd.set_path(old)
+        torch.cuda.synchronize()
+        check(prob, y, fin)
+
+
 def test_no_skip_no_init_no_final():
     wl = workloads.custom(1, 300, H=4, P=64, N=64, G=1, chunk=128, dtype="bf16")
     prob = workloads.generate(wl, seed=5)
