@@ -74,7 +74,8 @@ constexpr int kHeads = 2;           // heads of one B/C group processed together
 constexpr int kHalves = 2;          // each head's Y and state columns split over two warpgroups
 constexpr int kComputeThreads = kHeads * kHalves * kWGThreads;
 constexpr int kComputeWarps = kComputeThreads / 32;
-constexpr int kThreads = kComputeThreads + 64;  // + the issuer warp (TMA and UMMA) and the helper warp
+constexpr int kHelperWarps = kHeads;  // one helper warp per head of the pair
+constexpr int kThreads = kComputeThreads + 32 + 32 * kHelperWarps;  // + the issuer warp (TMA and UMMA), helpers
 constexpr int kIssuerWarp = kComputeWarps, kHelperWarp = kComputeWarps + 1;
 constexpr int kDescSlots = 2;  // tile descriptors the helper warp may run ahead
 constexpr int kDtStages = 4;   // dt tiles in flight
@@ -102,8 +103,8 @@ enum {
   kBarP,          // P written and Y rows scaled
   kBarFree,       // Y read (the next left factor may overwrite it)
   kBarXfree,      // a stage's x buffer (which held that tile's y for the TMA stores) is reusable
-  kBarDt0,        // kDtStages barriers: dt of a tile (4 heads x 128 tokens) in that stage
-  kBarDescFull0 = kBarDt0 + kDtStages,  // kDescSlots barriers: descriptor written
+  kBarDt0,        // kHelperWarps x kDtStages barriers: dt of a tile (4 heads x 128 tokens) in a helper's stage
+  kBarDescFull0 = kBarDt0 + kHelperWarps * kDtStages,  // kDescSlots barriers: descriptor written (both helpers)
   kBarDescFree0 = kBarDescFull0 + kDescSlots,  // kDescSlots barriers: descriptor used up
   kBarPair0 = kBarDescFree0 + kDescSlots,  // 8 barriers: the column-half-1 warp of a row quarter staged its y
   kNumBars = kBarPair0 + kHeads * 4
@@ -145,8 +146,8 @@ struct Layout {
   static constexpr uint32_t xw = c + (NS / 64) * kAtom;     // [head] [128 tok][64 p]
   static constexpr uint32_t ht = xw + kHeads * kAtom;       // [head] [NS n][64 p]
   static constexpr uint32_t desc = ht + kHeads * NS * 128;           // TileDesc[kDescSlots]
-  static constexpr uint32_t sdt = desc + kDescSlots * kDescBytes;    // float[stage][128 tok][4 heads]
-  static constexpr uint32_t bars = sdt + kDtStages * kTile * 16;     // uint64[kNumBars]
+  static constexpr uint32_t sdt = desc + kDescSlots * kDescBytes;    // float[helper][stage][128 tok][4 heads]
+  static constexpr uint32_t bars = sdt + kHelperWarps * kDtStages * kTile * 16;  // uint64[kNumBars]
   static constexpr uint32_t flag = bars + kNumBars * 8;     // int: a wait gave up
   static constexpr uint32_t bytes = flag + 16;
 };
@@ -697,7 +698,9 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
         if (lane == 0) red_add_release_gpu(&pb.carry_flag[blockIdx.x], 1);
         __syncwarp();
       }
+      TRACE_MARK(10);
       if (!wait(kBarDescFull0 + nslot)) return;
+      TRACE_MARK(11);
       const TileDesc& dn = descs[nslot];
       more = !(dn.flags & kDescEnd);
       if (more) {
@@ -717,6 +720,7 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
     tc_fence_after();
     {
       const float Dh = d.dskip[hw];
+      const uint64_t d2 = f2(Dh, Dh);
       const bool full = rem >= 32 * wq + 32;  // all 32 rows of this quarter are in the sequence
       uint8_t* ystage = const_cast<uint8_t*>(sxh);  // each thread overwrites the x chunks it reads
       __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(pb.y) + ((int64_t)(t0 + i) * pb.H + h) * kHeadDim;
@@ -731,10 +735,9 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
         const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
         uint32_t out[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const float x0 = __uint_as_float(xu[q] << 16), x1 = __uint_as_float(xu[q] & 0xFFFF0000u);
-          out[q] = pack_bf16(fmaf(Dh, x0, __uint_as_float(ry[8 * cc + 2 * q])),
-                             fmaf(Dh, x1, __uint_as_float(ry[8 * cc + 2 * q + 1])));
+        for (int q = 0; q < 4; ++q) {  // bf16 pair -> fp32 pair (exact), then D x + Y as one f32x2 fma
+          const uint64_t x2 = f2u(xu[q] << 16, xu[q] & 0xFFFF0000u);
+          out[q] = bf16x2_of(fma2(d2, x2, f2u(ry[8 * cc + 2 * q], ry[8 * cc + 2 * q + 1])));
         }
         const uint4 ov = make_uint4(out[0], out[1], out[2], out[3]);
         if (full)
@@ -769,18 +772,22 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
   }
 }
 
-// ------------------------------------------------------------------ helper warp
-// Walks the CTA's tile sequence a few tiles ahead of the compute warps: loads each tile's
-// dt by TMA (kDtStages tiles in flight) and writes the tile's descriptor into a ring of
-// kDescSlots: where the tile is, what happens to the state around it, and per head of the
-// pair the in-chunk cumsum of dt A in log2 units (restarted at every chunk boundary, and
-// continued from the handing-on CTA's value at a hand-on), the column factors
-// exp2(cs(end of 32-block) - cs_j) dt_j, dt (0 past the sequence end) and D.
+// ------------------------------------------------------------------ helper warps
+// Helper warp hh walks the CTA's tile sequence a few tiles ahead of the compute warps,
+// loads each tile's dt by TMA into a ring of its own (kDtStages tiles in flight) and
+// writes head hh's part of the tile's descriptor into a ring of kDescSlots: the in-chunk
+// cumsum of dt A in log2 units (restarted at every chunk boundary, and continued from the
+// handing-on CTA's value at a hand-on), the column factors exp2(cs(end of 32-block) -
+// cs_j) dt_j, dt (0 past the sequence end), the decay and D.  Helper 0 also writes where
+// the tile is and what happens to the state around it.  The descriptor is complete when
+// both helpers have arrived.
 template <int NS>
 __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t* smem, uint64_t* bars,
-                            volatile int* abort_flag) {
+                            volatile int* abort_flag, int hh) {
   using L = Layout<NS>;
   const int lane = threadIdx.x & 31;
+  uint8_t* my_dt = smem + L::sdt + hh * kDtStages * kTile * 16;
+  uint64_t* my_bar = bars + kBarDt0 + hh * kDtStages;
   const int pairs = pb.H / kHeads;
   TileDesc* descs = reinterpret_cast<TileDesc*>(smem + L::desc);
   uint32_t phase = 0;
@@ -800,8 +807,8 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t
     if (lane == 0) {
       const int st = dt_issued % kDtStages;
       const int h0 = (ahead.unit % pairs) * kHeads;
-      mbar_expect_tx(&bars[kBarDt0 + st], kTile * 16);
-      tma_load_2d(smem + L::sdt + st * kTile * 16, tm_dt, h0 & ~3, ahead.tb + ahead.k0, &bars[kBarDt0 + st]);
+      mbar_expect_tx(&my_bar[st], kTile * 16);
+      tma_load_2d(my_dt + st * kTile * 16, tm_dt, h0 & ~3, ahead.tb + ahead.k0, &my_bar[st]);
     }
     ++dt_issued;
     have_ahead = cursor_next(pb, rp, ahead);
@@ -810,8 +817,7 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t
 
   TileCursor cur;
   bool have = cursor_first(pb, rp, cur);
-  float cs_base[kHeads] = {0.f, 0.f};
-  float a2[kHeads] = {0.f, 0.f}, dsk[kHeads] = {0.f, 0.f};
+  float cs_base = 0.f, a2 = 0.f, dsk = 0.f;
   int a_unit = -1, prev_piece = -1;
   bool ok = true;
   int t = 0;
@@ -820,7 +826,7 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t
     if (t >= kDescSlots && !(ok = wait(kBarDescFree0 + slot))) break;
     TileDesc& d = descs[slot];
     if (!have) {
-      if (lane == 0) d.flags = kDescEnd;
+      if (hh == 0 && lane == 0) d.flags = kDescEnd;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kBarDescFull0 + slot]);
       break;
@@ -833,16 +839,13 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t
     const int h0 = (cur.unit % pairs) * kHeads;
     if (cur.unit != a_unit) {
       a_unit = cur.unit;
-#pragma unroll
-      for (int hh = 0; hh < kHeads; ++hh) {
-        a2[hh] = pb.A[h0 + hh] * 1.4426950408889634f;  // A_h log2(e): cumsums are in log2 units
-        dsk[hh] = pb.D ? pb.D[h0 + hh] : 0.f;
-      }
+      a2 = pb.A[h0 + hh] * 1.4426950408889634f;  // A_h log2(e): cumsums are in log2 units
+      dsk = pb.D ? pb.D[h0 + hh] : 0.f;
     }
     int flags = 0;
     if (first) {
       flags |= kDescFirst;
-      cs_base[0] = cs_base[1] = 0.f;
+      cs_base = 0.f;
       if (cur.flags & kCarryIn) {  // continue from the cumsum the previous CTA reached
         flags |= kDescCarryIn;
         bool mine = true;
@@ -862,71 +865,61 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t
           break;
         }
         __threadfence();
-#pragma unroll
-        for (int hh = 0; hh < kHeads; ++hh)
-          cs_base[hh] = __ldcg(pb.carry + (size_t)pb.ranges * kHeads * kHeadDim * NS + rp.carry_src * kHeads + hh);
+        cs_base = __ldcg(pb.carry + (size_t)pb.ranges * kHeads * kHeadDim * NS + rp.carry_src * kHeads + hh);
       }
     }
     if (last && (cur.flags & kUnitEnd) && pb.final_state) flags |= kDescToFinal;
     if (last && (cur.flags & kCarryOut)) flags |= kDescToCarry;
-    if (cur.k0 % pb.Q == 0) cs_base[0] = cs_base[1] = 0.f;
+    if (cur.k0 % pb.Q == 0) cs_base = 0.f;
 
     // this tile's dt: row 4 lane + j holds the 4 heads' dt of one token; a lane reads its
     // rows in the order j = (k + rot) & 3, rot = (lane / 2) & 3, so each quarter warp's
     // 16-byte loads fall in distinct banks
-    if (!(ok = wait(kBarDt0 + t % kDtStages))) break;
-    float dtt[kHeads][4];
+    if (!(ok = wait(kBarDt0 + hh * kDtStages + t % kDtStages))) break;
+    float dtt[4];
     {
-      const float4* rows = reinterpret_cast<const float4*>(smem + L::sdt + (t % kDtStages) * kTile * 16) + 4 * lane;
-      const int rot = (lane >> 1) & 3, hb = h0 & 3;  // the pair's first head in the 4-head row
-      float v[kHeads][4];
+      const float4* rows = reinterpret_cast<const float4*>(my_dt + (t % kDtStages) * kTile * 16) + 4 * lane;
+      const int rot = (lane >> 1) & 3, c = (h0 & 3) + hh;  // this head's column in the 4-head row
+      float v[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
         const float4 q = rows[(k + rot) & 3];
-        v[0][k] = hb == 0 ? q.x : q.z;  // hb is 0 or 2 (h0 is even)
-        v[1][k] = hb == 0 ? q.y : q.w;
+        v[k] = c == 0 ? q.x : c == 1 ? q.y : c == 2 ? q.z : q.w;
       }
       const int left = cur.len - cur.k0 - 4 * lane;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {  // token j came in as k = (j - rot) & 3
         const int k = (j - rot) & 3;
-#pragma unroll
-        for (int hh = 0; hh < kHeads; ++hh) {
-          const float val = k == 0 ? v[hh][0] : k == 1 ? v[hh][1] : k == 2 ? v[hh][2] : v[hh][3];
-          dtt[hh][j] = j < left ? dt_value(pb, val, h0 + hh) : 0.f;
-        }
+        const float val = k == 0 ? v[0] : k == 1 ? v[1] : k == 2 ? v[2] : v[3];
+        dtt[j] = j < left ? dt_value(pb, val, h0 + hh) : 0.f;
       }
     }
-#pragma unroll
-    for (int hh = 0; hh < kHeads; ++hh) {
-      const float Ah2 = a2[hh];
-      float c0 = dtt[hh][0] * Ah2, c1 = c0 + dtt[hh][1] * Ah2, c2 = c1 + dtt[hh][2] * Ah2,
-            c3 = c2 + dtt[hh][3] * Ah2;
+    {
+      float c0 = dtt[0] * a2, c1 = c0 + dtt[1] * a2, c2 = c1 + dtt[2] * a2, c3 = c2 + dtt[3] * a2;
       float v = c3;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const float u = __shfl_up_sync(0xffffffffu, v, o);
         if (lane >= o) v += u;
       }
-      const float base = cs_base[hh] + v - c3;  // cumsum before token 4 lane
+      const float base = cs_base + v - c3;  // cumsum before token 4 lane
       c0 += base, c1 += base, c2 += base, c3 += base;
       reinterpret_cast<float4*>(d.cs[hh])[lane] = make_float4(c0, c1, c2, c3);
-      reinterpret_cast<float4*>(d.dtv[hh])[lane] = make_float4(dtt[hh][0], dtt[hh][1], dtt[hh][2], dtt[hh][3]);
+      reinterpret_cast<float4*>(d.dtv[hh])[lane] = make_float4(dtt[0], dtt[1], dtt[2], dtt[3]);
       // block ends (tokens 31, 63, 95, 127) live in lanes 7, 15, 23, 31
       const float ref = __shfl_sync(0xffffffffu, c3, (lane & ~7) | 7);
-      reinterpret_cast<float4*>(d.cc[hh])[lane] =
-          make_float4(ex2(ref - c0) * dtt[hh][0], ex2(ref - c1) * dtt[hh][1], ex2(ref - c2) * dtt[hh][2],
-                      ex2(ref - c3) * dtt[hh][3]);
+      reinterpret_cast<float4*>(d.cc[hh])[lane] = make_float4(ex2(ref - c0) * dtt[0], ex2(ref - c1) * dtt[1],
+                                                              ex2(ref - c2) * dtt[2], ex2(ref - c3) * dtt[3]);
       const float cs_end = __shfl_sync(0xffffffffu, c3, 31);  // tokens past the end add 0
       if (lane == 0) {
-        d.cs_start[hh] = cs_base[hh];
+        d.cs_start[hh] = cs_base;
         d.cs_end[hh] = cs_end;
-        d.decay[hh] = ex2(cs_end - cs_base[hh]);
-        d.dskip[hh] = dsk[hh];
+        d.decay[hh] = ex2(cs_end - cs_base);
+        d.dskip[hh] = dsk;
       }
-      cs_base[hh] = cs_end;
+      cs_base = cs_end;
     }
-    if (lane == 0) {
+    if (hh == 0 && lane == 0) {
       d.t0 = cur.tb + cur.k0;
       d.rem = min(kTile, cur.len - cur.k0);
       d.s = cur.unit / pairs;
@@ -946,7 +939,7 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t
     // dt loads still in flight land before the CTA ends (bounded)
     if (lane == 0)
       for (int n = t; n < dt_issued; ++n)
-        mbar_wait_bounded(&bars[kBarDt0 + n % kDtStages], (n / kDtStages) & 1, kWaitLimit);
+        mbar_wait_bounded(&my_bar[n % kDtStages], (n / kDtStages) & 1, kWaitLimit);
   }
 }
 
@@ -981,9 +974,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars[kBarP], kComputeWarps);
     mbar_init(&bars[kBarFree], kComputeWarps);
     mbar_init(&bars[kBarXfree], kComputeWarps);
-    for (int k = 0; k < kDtStages; ++k) mbar_init(&bars[kBarDt0 + k], 1);
+    for (int k = 0; k < kHelperWarps * kDtStages; ++k) mbar_init(&bars[kBarDt0 + k], 1);
     for (int k = 0; k < kDescSlots; ++k) {
-      mbar_init(&bars[kBarDescFull0 + k], 1);
+      mbar_init(&bars[kBarDescFull0 + k], kHelperWarps);
       mbar_init(&bars[kBarDescFree0 + k], kComputeWarps);
     }
     for (int k = 0; k < kHeads * 4; ++k) mbar_init(&bars[kBarPair0 + k], 1);
@@ -1003,8 +996,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == kIssuerWarp) {
     if ((tid & 31) == 0) issuer_loop<NS>(&tm_x, &tm_b, &tm_c, pb, smem, tmem, bars, abort_flag);
     __syncwarp();  // the issuer warp reconverges before the CTA-wide barrier
-  } else if (warp == kHelperWarp) {
-    helper_loop<NS>(&tm_dt, pb, smem, bars, abort_flag);
+  } else if (warp >= kHelperWarp) {
+    helper_loop<NS>(&tm_dt, pb, smem, bars, abort_flag, warp - kHelperWarp);
     __syncwarp();
   } else {
     compute_loop<NS>(&tm_y32, pb, smem, tmem, bars, abort_flag);
