@@ -343,6 +343,7 @@ def run_ours(args, rank, world, local_rank):
     }
     if world == 1 and not args.no_decode:
         out["next"] = {"decode_step": decode_measurement(dev, stream, flush)}
+        out["next"].update(block_measurements(dev, stream, flush))
     if world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(prob, budget_s=args.cpu_budget)
     return out
@@ -387,6 +388,56 @@ def decode_measurement(dev, stream, flush, reps: int = 20):
             "l2": "flushed between launches; the state alone exceeds L2"}
 
 
+def _median_us(fn, stream, flush, reps: int = 20) -> float:
+    for _ in range(3):
+        fn()
+    ev = []
+    for _ in range(reps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fn()
+        b.record(stream)
+        ev.append((a, b))
+    torch.cuda.synchronize()
+    return statistics.median(a.elapsed_time(b) for a, b in ev) * 1e3
+
+
+def block_measurements(dev, stream, flush):
+    """The Mamba-2 block's steps either side of the SSD at the 2.7B layer shape (batch 8 x
+    2048 tokens, d_inner 5120, one B/C group of N = 128, bf16): the causal conv1d + SiLU
+    over the 5376 x/B/C channels and the gated RMSNorm over 5120 features.  Both read
+    each input once and write each output once; seeded synthetic inputs and weights."""
+    import ssd_sequence_mixing_b200 as ssd
+
+    peaks, kind = load_peaks()
+    g = torch.Generator(device=dev).manual_seed(0)
+    tokens, ch, dim = 8 * 2048, 5120 + 2 * 128, 5120
+    xbc = torch.randn((8, 2048, ch), generator=g, device=dev).to(torch.bfloat16)
+    w = torch.randn((ch, 4), generator=g, device=dev) * 0.5
+    b = torch.randn((ch,), generator=g, device=dev) * 0.1
+    out = torch.empty_like(xbc)
+    t_conv = _median_us(lambda: ssd.causal_conv1d_silu(xbc, w, b, out=out, stream=stream), stream, flush)
+    conv_bytes = tokens * ch * 2 * 2 + ch * 5 * 4
+    del xbc, out
+    y = torch.randn((tokens, dim), generator=g, device=dev).to(torch.bfloat16)
+    z = torch.randn((tokens, dim), generator=g, device=dev).to(torch.bfloat16)
+    wn = 1.0 + 0.1 * torch.randn((dim,), generator=g, device=dev)
+    o = torch.empty_like(y)
+    t_norm = _median_us(lambda: ssd.gated_rmsnorm(y, z, wn, out=o, stream=stream), stream, flush)
+    norm_bytes = tokens * dim * 2 * 3 + dim * 4
+
+    def line(name, t_us, nbytes):
+        gbs = nbytes / (t_us * 1e-6) / 1e9
+        return {"workload": name, "us": t_us, "algorithmic_bytes": nbytes,
+                "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                             "frac": gbs / peaks["hbm_gbs"], "peak_source": f"{kind} (GB/s)"},
+                "l2": "flushed between launches"}
+
+    return {"causal_conv1d_silu": line("conv1d_k4_silu_b8_L2048_ch5376_bf16", t_conv, conv_bytes),
+            "gated_rmsnorm": line("gated_rmsnorm_tokens16384_dim5120_bf16", t_norm, norm_bytes)}
+
+
 # ------------------------------------------------------------ reference arm
 def run_reference(args):
     """The fp64 CPU oracle on this workload: each step is a bounded sample (one sequence x
@@ -426,7 +477,8 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--e2e-steps", type=int, default=3)
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-decode", action="store_true", help="skip the decode-step measurement")
+    ap.add_argument("--no-decode", action="store_true",
+                    help="skip the measurements of the decode step and the block steps around the SSD")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--ref-heads", type=int, default=16)
     args = ap.parse_args()

@@ -191,6 +191,35 @@ int ssd_forward_noalloc(const ssd_shape* shape, const void* x, const float* dt, 
 int ssd_decode_step(const ssd_shape* shape, const void* x, const float* dt, const float* A, const void* B,
                     const void* C, const float* D, float* state, void* y, ssd_stream_t stream);
 
+/*
+ * ssd_causal_conv1d_silu -- the step before the SSD in the Mamba-2 block (the wikillm.com
+ * card: the Mamba-2 block sketch of sec. 7.1, "Paper vs code" 1 and 2): a depthwise causal
+ * convolution of kernel 4 over the concatenated x, B, C channels, then SiLU,
+ *     out[t,c] = silu(bias[c] + sum_{k=0..3} weight[c,k] in[t-3+k, c]),  silu(v) = v / (1 + e^-v)
+ * with in[] = 0 before each sequence's first token (the window restarts at every sequence).
+ *   xbc, out    (batch, seqlen, channels)  io_dtype (out may not alias xbc)
+ *   weight      (channels, 4)              fp32;  bias (channels) fp32 or NULL (= 0)
+ *   cu_seqlens  (nseq + 1) int32 on the device, or NULL for a dense batch; it must be a
+ *               valid offset list (0 = c_0 <= ... <= c_nseq = seqlen, batch = 1): this
+ *               call does not check its values.
+ * channels % 8 == 0 (SSD_ERR_UNSUPPORTED otherwise).  Device pointers, 16-byte aligned;
+ * no scratch; asynchronous on `stream`.
+ */
+int ssd_causal_conv1d_silu(int64_t batch, int64_t seqlen, int64_t channels, ssd_dtype io_dtype, const void* xbc,
+                           const float* weight, const float* bias, const int32_t* cu_seqlens, int64_t nseq,
+                           void* out, ssd_stream_t stream);
+
+/*
+ * ssd_gated_rmsnorm -- the step after the SSD in the Mamba-2 block (the wikillm.com card:
+ * the Mamba-2 block sketch of sec. 7.1 and "Paper vs code" 9: gated RMSNorm, gate before
+ * the norm, eps 1e-5 there), per token over its `dim` features:
+ *     g = y * silu(z);   out = g / sqrt(mean(g^2) + eps) * weight
+ *   y, z, out   (tokens, dim)  io_dtype;   weight (dim) fp32
+ * dim % 8 == 0 and dim <= 8192.  Device pointers, 16-byte aligned; asynchronous on `stream`.
+ */
+int ssd_gated_rmsnorm(int64_t tokens, int64_t dim, ssd_dtype io_dtype, const void* y, const void* z,
+                      const float* weight, float eps, void* out, ssd_stream_t stream);
+
 /* Bytes of stream-ordered scratch ssd_forward takes for this shape (informational). */
 size_t ssd_workspace_bytes(const ssd_shape* shape, int chunk);
 

@@ -13,6 +13,8 @@ leg may import this package.  It shares no code with the CUDA path.
 * ``decode_step``: one recurrent generation step (Method step 8, sec. 6.3).
 * ``dt_prologue``: the step size from the raw projection, dt = softplus(raw + bias)
   (the Mamba-2 block sketch of sec. 7.1 and Method note 7 "Discretisation").
+* ``causal_conv1d_silu`` and ``gated_rmsnorm``: the block's steps before and after the
+  SSD (the Mamba-2 block sketch of sec. 7.1; "Paper vs code" 1, 2 and 9).
 
 Parity status of every function here is recorded in the tests that pin it.
 """
@@ -172,6 +174,36 @@ def dt_prologue(dt_raw, dt_bias=None, softplus: bool = True, dt_min: float = 0.0
     if softplus:
         v = np.logaddexp(0.0, v)  # log(exp(0) + exp(v)) = log(1 + exp(v))
     return np.clip(v, dt_min, dt_max)
+
+
+def causal_conv1d_silu(x, weight, bias=None, seq_offsets=None):
+    """Depthwise causal convolution of kernel K = weight.shape[1] along time, then SiLU, in
+    fp64: out[t, c] = silu(bias[c] + sum_k weight[c, k] x[t - (K-1) + k, c]) with x = 0
+    before each sequence's first token; silu(v) = v / (1 + exp(-v)).
+    x (T, channels); seq_offsets (nseq + 1) token offsets (default: one sequence)."""
+    x, w = _f64(x), _f64(weight)
+    T, ch = x.shape
+    K = w.shape[1]
+    offs = [0, T] if seq_offsets is None else list(seq_offsets)
+    out = np.zeros((T, ch))
+    for s in range(len(offs) - 1):
+        a, e = int(offs[s]), int(offs[s + 1])
+        for t in range(a, e):
+            acc = np.zeros(ch) if bias is None else _f64(bias).copy()
+            for k in range(K):
+                src = t - (K - 1) + k
+                if src >= a:
+                    acc += w[:, k] * x[src]
+            out[t] = acc / (1.0 + np.exp(-acc))
+    return out
+
+
+def gated_rmsnorm(y, z, weight, eps: float = 1e-5):
+    """Gate first, then RMSNorm over the last axis, in fp64: g = y * silu(z),
+    out = g / sqrt(mean(g^2) + eps) * weight."""
+    y, z, w = _f64(y), _f64(z), _f64(weight)
+    g = y * (z / (1.0 + np.exp(-z)))
+    return g / np.sqrt(np.mean(g * g, axis=-1, keepdims=True) + eps) * w
 
 
 def decode_step(x, dt, A, B, C, D, state):

@@ -45,6 +45,8 @@ EXPORTS = (
     "ssd_forward_noalloc",
     "ssd_decode_step",
     "ssd_forward_dt",
+    "ssd_causal_conv1d_silu",
+    "ssd_gated_rmsnorm",
 )
 
 
@@ -104,6 +106,11 @@ def _open() -> ctypes.CDLL:
     lib.ssd_decode_step.restype = I
     lib.ssd_forward_dt.argtypes = [SP, ctypes.POINTER(SsdDtPrologue)] + fwd[1:]
     lib.ssd_forward_dt.restype = I
+    L = ctypes.c_int64
+    lib.ssd_causal_conv1d_silu.argtypes = [L, L, L, I, V, V, V, V, L, V, V]
+    lib.ssd_causal_conv1d_silu.restype = I
+    lib.ssd_gated_rmsnorm.argtypes = [L, L, I, V, V, V, ctypes.c_float, V, V]
+    lib.ssd_gated_rmsnorm.restype = I
     return lib
 
 
@@ -259,6 +266,59 @@ def ssd_forward_dt(x, dt_raw, A, B, C, D=None, init_state=None, cu_seqlens=None,
     if rc:
         raise SsdError(rc, "ssd_forward_dt")
     return y, final_state
+
+
+def causal_conv1d_silu(xbc, weight, bias=None, cu_seqlens=None, out: Optional[torch.Tensor] = None, stream=None):
+    """Depthwise causal conv1d (kernel 4) + SiLU over the channels of xbc (batch, seqlen,
+    channels); weight (channels, 4) and bias (channels,) float32; the window restarts at
+    every sequence (rows of a dense batch, or cu_seqlens ranges)."""
+    device = xbc.device
+    if device.type != "cuda":
+        raise ValueError("causal_conv1d_silu takes CUDA tensors")
+    if xbc.dim() != 3:
+        raise ValueError("xbc must be (batch, seqlen, channels)")
+    batch, T, ch = xbc.shape
+    _check("xbc", xbc, device)
+    _check("weight", weight, device, torch.float32, (ch, 4))
+    _check("bias", bias, device, torch.float32, (ch,))
+    _check("cu_seqlens", cu_seqlens, device, torch.int32)
+    if out is None:
+        out = torch.empty_like(xbc)
+    _check("out", out, device, xbc.dtype, tuple(xbc.shape))
+    nseq = 0 if cu_seqlens is None else cu_seqlens.numel() - 1
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    with torch.cuda.device(device):
+        rc = _lib.ssd_causal_conv1d_silu(batch, T, ch, _io_code(xbc.dtype), _ptr(xbc), _ptr(weight), _ptr(bias),
+                                         _ptr(cu_seqlens), nseq, _ptr(out), ctypes.c_void_p(handle))
+    if rc:
+        raise SsdError(rc, "ssd_causal_conv1d_silu")
+    return out
+
+
+def gated_rmsnorm(y, z, weight, eps: float = 1e-5, out: Optional[torch.Tensor] = None, stream=None):
+    """Gate first, then RMSNorm over the last dimension: g = y silu(z), out = g / rms(g) * weight."""
+    device = y.device
+    if device.type != "cuda":
+        raise ValueError("gated_rmsnorm takes CUDA tensors")
+    dim = y.shape[-1]
+    tokens = y.numel() // dim if dim else 0
+    _check("y", y, device)
+    _check("z", z, device, y.dtype, tuple(y.shape))
+    _check("weight", weight, device, torch.float32, (dim,))
+    if out is None:
+        out = torch.empty_like(y)
+    _check("out", out, device, y.dtype, tuple(y.shape))
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    with torch.cuda.device(device):
+        rc = _lib.ssd_gated_rmsnorm(tokens, dim, _io_code(y.dtype), _ptr(y), _ptr(z), _ptr(weight), float(eps),
+                                    _ptr(out), ctypes.c_void_p(handle))
+    if rc:
+        raise SsdError(rc, "ssd_gated_rmsnorm")
+    return out
 
 
 def ssd_decode_step(x, dt, A, B, C, D, state, y: Optional[torch.Tensor] = None, stream=None):

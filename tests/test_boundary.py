@@ -161,3 +161,23 @@ def test_dt_prologue_misaligned_bias():
     rc = ssd.library().ssd_forward_dt(ctypes.byref(shape()), ctypes.byref(pro), p["x"], p["dt"], p["A"], p["B"],
                                       p["C"], None, None, None, 256, p["y"], None, None)
     assert rc == 3
+
+
+# ------------------------------------------------- block steps around the SSD
+def test_conv_and_norm_reject_before_launch():
+    lib = ssd.library()
+    F = ctypes.c_void_p(FAKE)
+    conv = lambda *a, **k: lib.ssd_causal_conv1d_silu(*a)
+    assert conv(2, 10, 12, ssd.SSD_BF16, F, F, None, None, 0, F, None) == 2  # channels % 8
+    assert conv(2, 10, 16, 9, F, F, None, None, 0, F, None) == 1
+    assert conv(2, 10, 16, ssd.SSD_BF16, F, F, None, F, 3, F, None) == 1  # packed needs batch 1
+    assert conv(1, 10, 16, ssd.SSD_BF16, None, F, None, None, 0, F, None) == 1
+    assert conv(1, 10, 16, ssd.SSD_BF16, ctypes.c_void_p(FAKE + 4), F, None, None, 0, F, None) == 3
+    assert conv(0, 10, 16, ssd.SSD_BF16, None, None, None, None, 0, None, None) == 0  # nothing to do
+    norm = lib.ssd_gated_rmsnorm
+    assert norm(4, 12, ssd.SSD_BF16, F, F, F, 1e-5, F, None) == 2  # dim % 8
+    assert norm(4, 8200, ssd.SSD_BF16, F, F, F, 1e-5, F, None) == 2  # dim > 8192
+    assert norm(4, 16, ssd.SSD_BF16, F, F, F, -1.0, F, None) == 1
+    assert norm(4, 16, ssd.SSD_BF16, F, None, F, 1e-5, F, None) == 1
+    assert norm(4, 16, ssd.SSD_BF16, F, F, ctypes.c_void_p(FAKE + 8), 1e-5, F, None) == 3
+    assert norm(0, 16, ssd.SSD_BF16, None, None, None, 1e-5, None, None) == 0

@@ -265,6 +265,60 @@ def test_dt_prologue_forward_equals_forward_on_inverse_softplus():
     assert np.array_equal(y3, y2) and np.array_equal(f3, f2)
 
 
+# ------------------------------------------ block steps around the SSD (NEXT-3)
+def silu_ref(v):
+    return v / (1.0 + np.exp(-v))
+
+
+def test_conv_impulse_response_and_sequence_reset():
+    """A unit impulse at token t0 of channel c gives pre-activations w[c, 3 - j] at
+    t0 + j (j < 4) and 0 elsewhere; an impulse on a sequence's last token does not
+    reach the next sequence."""
+    rng = np.random.default_rng(41)
+    w = rng.standard_normal((3, 4))
+    x = np.zeros((12, 3))
+    x[5, 1] = 1.0
+    out = oracle.causal_conv1d_silu(x, w)
+    expect = np.zeros((12, 3))
+    for j in range(4):
+        expect[5 + j, 1] = silu_ref(w[1, 3 - j])
+    assert np.allclose(out, expect, rtol=1e-15, atol=1e-300)
+    x2 = np.zeros((12, 3))
+    x2[6, 0] = 1.0  # last token of the first sequence [0, 7)
+    bias = np.array([0.25, -0.5, 0.0])
+    out2 = oracle.causal_conv1d_silu(x2, w, bias, seq_offsets=[0, 7, 7, 12])
+    assert np.allclose(out2[7:], silu_ref(bias)[None, :].repeat(5, 0))
+    assert out2[6, 0] == pytest.approx(silu_ref(w[0, 3] + 0.25))
+
+
+def test_conv_equals_library_convolution():
+    rng = np.random.default_rng(42)
+    T, ch = 50, 4
+    x = rng.standard_normal((T, ch))
+    w = rng.standard_normal((ch, 4))
+    b = rng.standard_normal(ch)
+    out = oracle.causal_conv1d_silu(x, w, b)
+    for c in range(ch):
+        pre = np.convolve(x[:, c], w[c, ::-1])[:T] + b[c]  # causal: out[t] = sum_k w[k] x[t-3+k]
+        assert np.allclose(out[:, c], silu_ref(pre), rtol=1e-13, atol=1e-13)
+
+
+def test_gated_rmsnorm_closed_forms():
+    rng = np.random.default_rng(43)
+    y = rng.standard_normal((5, 16))
+    w = rng.uniform(0.5, 2.0, 16)
+    # z = 0 gates everything off: g = 0, out = 0
+    assert np.array_equal(oracle.gated_rmsnorm(y, np.zeros_like(y), w), np.zeros_like(y))
+    # a constant gate cancels in the norm: out = y / sqrt(mean(y^2) + eps / s^2) * w, s = silu(z)
+    s = silu_ref(3.0)
+    got = oracle.gated_rmsnorm(y, np.full_like(y, 3.0), w, eps=1e-5)
+    expect = y / np.sqrt(np.mean(y * y, axis=1, keepdims=True) + 1e-5 / s ** 2) * w
+    assert np.allclose(got, expect, rtol=1e-13)
+    # eps = 0, unit weight: every token's output has RMS 1
+    out = oracle.gated_rmsnorm(y, rng.standard_normal(y.shape), np.ones(16), eps=0.0)
+    assert np.allclose(np.sqrt(np.mean(out * out, axis=1)), 1.0, rtol=1e-13)
+
+
 # ------------------------------------------------------- workload generator
 def test_sampled_problem_matches_full():
     """The sampled-pairs harness returns exactly the full oracle's rows."""
