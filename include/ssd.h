@@ -220,6 +220,26 @@ int ssd_causal_conv1d_silu(int64_t batch, int64_t seqlen, int64_t channels, ssd_
 int ssd_gated_rmsnorm(int64_t tokens, int64_t dim, ssd_dtype io_dtype, const void* y, const void* z,
                       const float* weight, float eps, void* out, ssd_stream_t stream);
 
+/*
+ * Sequence-parallel SSD (one sequence split into contiguous segments, one per GPU): the
+ * state passes from segment to segment exactly as from chunk to chunk (the wikillm.com
+ * card, Method step 5, the centre factor).  Each rank r runs ssd_forward on its segment
+ * from a zero state, giving its end state s_r, and ssd_segment_logdecay gives
+ * lambda_r[h] = A[h] * sum_t dt[t,h] over the segment.  After an all-gather of (s, lambda),
+ * ssd_state_prefix gives the segment's true start state
+ *     h_0 = init,  h_{q+1} = exp(lambda_q) h_q + s_q   (q < rank),
+ * and the rank runs ssd_forward again from it.  See sequence_parallel.py in the package.
+ *
+ * ssd_segment_logdecay: dt (tokens, H) fp32, A (H) fp32 -> out (H) fp32.
+ * ssd_state_prefix: states (>= rank, H, P, N) and logdecay (>= rank, H) of the
+ *   preceding segments, init_state (H, P, N) or NULL (= 0) -> out (H, P, N); all fp32.
+ * Device pointers; asynchronous on `stream`; SSD_ERR_INVALID_ARG for bad sizes or nulls.
+ */
+int ssd_segment_logdecay(int64_t tokens, int64_t nheads, const float* dt, const float* A, float* out,
+                         ssd_stream_t stream);
+int ssd_state_prefix(int rank, int64_t nheads, int64_t headdim, int64_t dstate, const float* states,
+                     const float* logdecay, const float* init_state, float* out, ssd_stream_t stream);
+
 /* Bytes of stream-ordered scratch ssd_forward takes for this shape (informational). */
 size_t ssd_workspace_bytes(const ssd_shape* shape, int chunk);
 

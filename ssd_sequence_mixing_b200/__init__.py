@@ -47,6 +47,8 @@ EXPORTS = (
     "ssd_forward_dt",
     "ssd_causal_conv1d_silu",
     "ssd_gated_rmsnorm",
+    "ssd_segment_logdecay",
+    "ssd_state_prefix",
 )
 
 
@@ -111,6 +113,10 @@ def _open() -> ctypes.CDLL:
     lib.ssd_causal_conv1d_silu.restype = I
     lib.ssd_gated_rmsnorm.argtypes = [L, L, I, V, V, V, ctypes.c_float, V, V]
     lib.ssd_gated_rmsnorm.restype = I
+    lib.ssd_segment_logdecay.argtypes = [L, L, V, V, V, V]
+    lib.ssd_segment_logdecay.restype = I
+    lib.ssd_state_prefix.argtypes = [I, L, L, L, V, V, V, V, V]
+    lib.ssd_state_prefix.restype = I
     return lib
 
 
@@ -318,6 +324,46 @@ def gated_rmsnorm(y, z, weight, eps: float = 1e-5, out: Optional[torch.Tensor] =
                                     _ptr(out), ctypes.c_void_p(handle))
     if rc:
         raise SsdError(rc, "ssd_gated_rmsnorm")
+    return out
+
+
+def segment_logdecay(dt, A, stream=None):
+    """lambda[h] = A[h] * sum_t dt[t, h] over a segment; dt (tokens, H) or (1, tokens, H)."""
+    device = dt.device
+    H = dt.shape[-1]
+    tokens = dt.numel() // H
+    _check("dt", dt, device, torch.float32)
+    _check("A", A, device, torch.float32, (H,))
+    out = torch.empty(H, dtype=torch.float32, device=device)
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    with torch.cuda.device(device):
+        rc = _lib.ssd_segment_logdecay(tokens, H, _ptr(dt), _ptr(A), _ptr(out), ctypes.c_void_p(handle))
+    if rc:
+        raise SsdError(rc, "ssd_segment_logdecay")
+    return out
+
+
+def state_prefix(rank: int, states, logdecay, init_state=None, stream=None):
+    """Start state of segment ``rank`` from the preceding segments' zero-start end states
+    (>= rank, H, P, N) and log-decays (>= rank, H): h_{q+1} = exp(lambda_q) h_q + s_q."""
+    device = states.device
+    _, H, P, N = states.shape
+    _check("states", states, device, torch.float32)
+    _check("logdecay", logdecay, device, torch.float32)
+    _check("init_state", init_state, device, torch.float32, (H, P, N))
+    if states.shape[0] < rank or logdecay.shape[0] < rank or logdecay.shape[1] != H:
+        raise ValueError("states and logdecay must cover the preceding segments")
+    out = torch.empty((H, P, N), dtype=torch.float32, device=device)
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    with torch.cuda.device(device):
+        rc = _lib.ssd_state_prefix(int(rank), H, P, N, _ptr(states), _ptr(logdecay), _ptr(init_state), _ptr(out),
+                                   ctypes.c_void_p(handle))
+    if rc:
+        raise SsdError(rc, "ssd_state_prefix")
     return out
 
 

@@ -17,7 +17,10 @@
 namespace ssd {
 namespace {
 
-__device__ __forceinline__ float silu(float v) { return v / (1.f + expf(-v)); }
+// v sigmoid(v) with the hardware exponential and the approximate division (relative error
+// a few ulp, far below bf16 rounding; 0 where e^-v overflows); both kernels are bound by
+// instruction issue with the IEEE forms.
+__device__ __forceinline__ float silu(float v) { return __fdividef(v, 1.f + __expf(-v)); }
 
 // 8 consecutive channels of one token: one 16-byte (bf16) or two (fp32) loads.
 struct Vec8 {
@@ -38,6 +41,32 @@ __device__ __forceinline__ Vec8 load8(const float* p) {
   const float4 a = *reinterpret_cast<const float4*>(p), b = *reinterpret_cast<const float4*>(p + 4);
   return Vec8{{a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w}};
 }
+// The raw 16 (bf16) or 32 (fp32) bytes of 8 channels, unpacked when used.
+template <typename T>
+struct Raw8;
+template <>
+struct Raw8<__nv_bfloat16> {
+  uint4 q;
+  __device__ __forceinline__ void load(const __nv_bfloat16* p) { q = *reinterpret_cast<const uint4*>(p); }
+  __device__ __forceinline__ float at(int i) const {
+    const uint32_t word = (i >> 1) == 0 ? q.x : (i >> 1) == 1 ? q.y : (i >> 1) == 2 ? q.z : q.w;
+    return __uint_as_float((i & 1) ? (word & 0xFFFF0000u) : (word << 16));
+  }
+};
+template <>
+struct Raw8<float> {
+  float4 a, b;
+  __device__ __forceinline__ void load(const float* p) {
+    a = *reinterpret_cast<const float4*>(p);
+    b = *reinterpret_cast<const float4*>(p + 4);
+  }
+  __device__ __forceinline__ float at(int i) const {
+    const float4& h = i < 4 ? a : b;
+    const int j = i & 3;
+    return j == 0 ? h.x : j == 1 ? h.y : j == 2 ? h.z : h.w;
+  }
+};
+
 __device__ __forceinline__ void store8(__nv_bfloat16* p, const float (&v)[8]) {
   uint4 q;
   uint32_t* w = reinterpret_cast<uint32_t*>(&q);
@@ -63,25 +92,33 @@ struct ConvArgs {
   const int32_t* cu;  // (nseq + 1) or null
   void* out;
 };
-constexpr int kConvTok = 64;     // tokens one thread walks
-constexpr int kConvBatch = 8;    // tokens whose loads are in flight together
+constexpr int kConvTok = 8;  // tokens per thread: their inputs and the 3-token halo load at once
 constexpr int kConvThreads = 128;
 
 __device__ __forceinline__ int64_t seq_start_of(const ConvArgs& a, int64_t s) {
   return a.cu ? (int64_t)a.cu[s] : s * a.seqlen;
 }
 
-// Grid (ceil(channels / 8 / 128), ceil(tokens / 64)).  Thread: 8 channels x 64 tokens,
-// walking the tokens in order with the previous three inputs in registers; the window
-// is zero before each sequence start.
+// Grid: ceil(channels / 8 / 128) channel blocks x ceil(tokens / 8) token blocks, flattened
+// (channel block fastest).  A thread computes 8 channels of 8
+// consecutive tokens: it loads those tokens and the three before them (the halo, an L2 hit
+// after the neighbouring thread block's load) in one go, then walks them in order.  Inputs
+// before the start of a token's sequence count as zero.
 template <typename T>
 __global__ void __launch_bounds__(kConvThreads) conv1d_silu_kernel(ConvArgs a) {
-  const int64_t c0 = ((int64_t)blockIdx.x * kConvThreads + threadIdx.x) * 8;
+  const int64_t cblocks = (a.channels / 8 + kConvThreads - 1) / kConvThreads;
+  const int64_t c0 = ((int64_t)(blockIdx.x % cblocks) * kConvThreads + threadIdx.x) * 8;
   if (c0 >= a.channels) return;
-  const int64_t t0 = (int64_t)blockIdx.y * kConvTok;
+  const int64_t t0 = (int64_t)(blockIdx.x / cblocks) * kConvTok;
   const int64_t t1 = min(t0 + (int64_t)kConvTok, a.tokens);
   const T* in = static_cast<const T*>(a.in);
   T* out = static_cast<T*>(a.out);
+  Raw8<T> raw[kConvTok + 3];  // tokens t0 - 3 .. t0 + 7
+#pragma unroll
+  for (int k = 0; k < kConvTok + 3; ++k) {
+    const int64_t t = t0 - 3 + k;
+    if (t >= 0 && t < t1) raw[k].load(in + t * a.channels + c0);
+  }
   float w[8][4], b[8];
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
@@ -89,7 +126,7 @@ __global__ void __launch_bounds__(kConvThreads) conv1d_silu_kernel(ConvArgs a) {
     w[i][0] = q.x, w[i][1] = q.y, w[i][2] = q.z, w[i][3] = q.w;
     b[i] = a.bias ? a.bias[c0 + i] : 0.f;
   }
-  // the sequence holding t0, and where the next one starts
+  // the sequence holding t0: its start, and where the next one starts
   int64_t s;
   if (a.cu) {
     int lo = 0, hi = a.nseq;  // cu[lo] <= t0 < cu[hi]
@@ -102,58 +139,46 @@ __global__ void __launch_bounds__(kConvThreads) conv1d_silu_kernel(ConvArgs a) {
   } else {
     s = t0 / a.seqlen;
   }
-  int64_t start = seq_start_of(a, s), next = s + 1 <= a.nseq ? seq_start_of(a, s + 1) : a.tokens;
-  while (next <= t0 && s + 1 < a.nseq) {  // empty sequences end where the next begins
-    ++s;
-    start = next;
-    next = seq_start_of(a, s + 1);
-  }
-  float win[3][8];  // inputs at t - 3, t - 2, t - 1
+  int64_t start = seq_start_of(a, s), next = seq_start_of(a, s + 1);
+  if (start <= t0 - 3 && next >= t1) {  // no sequence start in the window: every tap is live
 #pragma unroll
-  for (int j = 0; j < 3; ++j) {
-    const int64_t t = t0 - 3 + j;
-    if (t >= start && t >= 0) {
-      const Vec8 v = load8(in + t * a.channels + c0);
-#pragma unroll
-      for (int i = 0; i < 8; ++i) win[j][i] = v.v[i];
-    } else {
-#pragma unroll
-      for (int i = 0; i < 8; ++i) win[j][i] = 0.f;
-    }
-  }
-  for (int64_t tb = t0; tb < t1; tb += kConvBatch) {
-    Vec8 cur[kConvBatch];
-#pragma unroll
-    for (int k = 0; k < kConvBatch; ++k)
-      if (tb + k < t1) cur[k] = load8(in + (tb + k) * a.channels + c0);
-#pragma unroll
-    for (int k = 0; k < kConvBatch; ++k) {
-      const int64_t t = tb + k;
+    for (int k = 0; k < kConvTok; ++k) {
+      const int64_t t = t0 + k;
       if (t >= t1) break;
-      while (t >= next && s + 1 < a.nseq) {  // a new sequence starts: the window restarts at zero
-        ++s;
-        start = next;
-        next = seq_start_of(a, s + 1);
-#pragma unroll
-        for (int j = 0; j < 3; ++j)
-#pragma unroll
-          for (int i = 0; i < 8; ++i) win[j][i] = 0.f;
-      }
       float o[8];
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         float acc = b[i];
-        acc = fmaf(w[i][0], win[0][i], acc);
-        acc = fmaf(w[i][1], win[1][i], acc);
-        acc = fmaf(w[i][2], win[2][i], acc);
-        acc = fmaf(w[i][3], cur[k].v[i], acc);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) acc = fmaf(w[i][j], raw[k + j].at(i), acc);  // input t - 3 + j
         o[i] = silu(acc);
-        win[0][i] = win[1][i];
-        win[1][i] = win[2][i];
-        win[2][i] = cur[k].v[i];
       }
       store8(out + t * a.channels + c0, o);
     }
+    return;
+  }
+#pragma unroll
+  for (int k = 0; k < kConvTok; ++k) {
+    const int64_t t = t0 + k;
+    if (t >= t1) break;
+    while (t >= next && s + 1 < a.nseq) {  // empty sequences end where the next begins
+      ++s;
+      start = next;
+      next = seq_start_of(a, s + 1);
+    }
+    bool live[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) live[j] = t - 3 + j >= start;
+    float o[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float acc = b[i];
+#pragma unroll
+      for (int j = 0; j < 4; ++j)  // input t - 3 + j sits in raw[k + j]
+        if (live[j]) acc = fmaf(w[i][j], raw[k + j].at(i), acc);
+      o[i] = silu(acc);
+    }
+    store8(out + t * a.channels + c0, o);
   }
 }
 
@@ -166,11 +191,11 @@ struct NormArgs {
   float eps;
   void* out;
 };
-constexpr int kNormThreads = 128;
-constexpr int kNormVecs = 8;  // 8-channel vectors per thread: dim <= 8 * 128 * 8 = 8192
+constexpr int kNormThreads = 256;
+constexpr int kNormVecs = 4;  // 8-feature vectors per thread held in registers: dim <= 8192
 
-// One block per token: g = y silu(z) in fp32 registers, a block sum of g^2, then
-// out = g * rsqrt(mean(g^2) + eps) * w.
+// One block per token: g = y silu(z) in fp32 registers (with the weights loaded alongside),
+// a block sum of g^2, then out = g * rsqrt(mean(g^2) + eps) * w.
 template <typename T>
 __global__ void __launch_bounds__(kNormThreads) gated_rmsnorm_kernel(NormArgs a) {
   __shared__ float s_part[kNormThreads / 32];
@@ -179,16 +204,17 @@ __global__ void __launch_bounds__(kNormThreads) gated_rmsnorm_kernel(NormArgs a)
   const T* z = static_cast<const T*>(a.z) + tok * a.dim;
   T* out = static_cast<T*>(a.out) + tok * a.dim;
   const int nv = (int)(a.dim / 8);
-  float g[kNormVecs][8];
+  float g[kNormVecs][8], wr[kNormVecs][8];
   float ss = 0.f;
 #pragma unroll
   for (int k = 0; k < kNormVecs; ++k) {
     const int v = threadIdx.x + k * kNormThreads;
     if (v < nv) {
-      const Vec8 yv = load8(y + v * 8), zv = load8(z + v * 8);
+      const Vec8 yv = load8(y + v * 8), zv = load8(z + v * 8), wv = load8(a.w + v * 8);
 #pragma unroll
       for (int i = 0; i < 8; ++i) {
         g[k][i] = yv.v[i] * silu(zv.v[i]);
+        wr[k][i] = wv.v[i];
         ss = fmaf(g[k][i], g[k][i], ss);
       }
     }
@@ -205,10 +231,9 @@ __global__ void __launch_bounds__(kNormThreads) gated_rmsnorm_kernel(NormArgs a)
   for (int k = 0; k < kNormVecs; ++k) {
     const int v = threadIdx.x + k * kNormThreads;
     if (v < nv) {
-      const Vec8 wv = load8(a.w + v * 8);
       float o[8];
 #pragma unroll
-      for (int i = 0; i < 8; ++i) o[i] = g[k][i] * r * wv.v[i];
+      for (int i = 0; i < 8; ++i) o[i] = g[k][i] * r * wr[k][i];
       store8(out + v * 8, o);
     }
   }
@@ -239,9 +264,10 @@ extern "C" int ssd_causal_conv1d_silu(int64_t batch, int64_t seqlen, int64_t cha
   a.seqlen = cu_seqlens ? tokens : seqlen;
   a.nseq = (int)(cu_seqlens ? nseq : batch);
   a.in = xbc, a.w = weight, a.bias = bias, a.cu = cu_seqlens, a.out = out;
-  const dim3 grid((unsigned)((channels / 8 + ssd::kConvThreads - 1) / ssd::kConvThreads),
-                  (unsigned)((tokens + ssd::kConvTok - 1) / ssd::kConvTok));
-  if (grid.y > 65535u * 1024u) return SSD_ERR_UNSUPPORTED;
+  const int64_t nblocks = (channels / 8 + ssd::kConvThreads - 1) / ssd::kConvThreads *
+                          ((tokens + ssd::kConvTok - 1) / ssd::kConvTok);
+  if (nblocks > ((int64_t)1 << 31) - 1) return SSD_ERR_UNSUPPORTED;
+  const dim3 grid((unsigned)nblocks);
   cudaStream_t st = (cudaStream_t)stream;
   if (io_dtype == SSD_BF16)
     ssd::conv1d_silu_kernel<__nv_bfloat16><<<grid, ssd::kConvThreads, 0, st>>>(a);

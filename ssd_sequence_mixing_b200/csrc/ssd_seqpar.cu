@@ -1,0 +1,74 @@
+// ssd_seqpar.cu -- the two small steps of the sequence-parallel SSD ("Transformers are
+// SSMs", the wikillm.com card: Method step 5, the centre factor that passes the state from
+// one chunk to the next, applied here between segments of one sequence held by different
+// GPUs).  A rank runs its segment from a zero state and publishes its end state s_r and
+// its segment log-decay lambda_r = sum_t dt_t A_h; the start state of segment r is then
+//     h_0 = init,   h_{q+1} = exp(lambda_q) h_q + s_q,
+// after which the rank runs its segment again from h_r.
+#include <cuda_runtime.h>
+#include <math.h>
+#include <stdint.h>
+
+#include "ssd.h"
+#include "ssd_common.cuh"
+
+namespace ssd {
+namespace {
+
+constexpr int kHeadsPerBlock = 32, kTokLanes = 8;
+
+// Grid ceil(H / 32); block (32 heads x 8 token lanes): coalesced reads of dt rows.
+__global__ void __launch_bounds__(kHeadsPerBlock * kTokLanes)
+    segment_logdecay_kernel(int64_t tokens, int H, const float* dt, const float* A, float* out) {
+  __shared__ float part[kTokLanes][kHeadsPerBlock];
+  const int hl = threadIdx.x % kHeadsPerBlock, tl = threadIdx.x / kHeadsPerBlock;
+  const int h = blockIdx.x * kHeadsPerBlock + hl;
+  float acc = 0.f;
+  if (h < H)
+    for (int64_t t = tl; t < tokens; t += kTokLanes) acc += dt[t * H + h];
+  part[tl][hl] = acc;
+  __syncthreads();
+  if (tl == 0 && h < H) {
+    float s = 0.f;
+#pragma unroll
+    for (int k = 0; k < kTokLanes; ++k) s += part[k][hl];
+    out[h] = s * A[h];
+  }
+}
+
+// One thread per state element (h, p, n): the recurrence over the preceding segments.
+__global__ void __launch_bounds__(256) state_prefix_kernel(int rank, int64_t H, int64_t PN, const float* states,
+                                                           const float* logdecay, const float* init, float* out) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= H * PN) return;
+  const int64_t h = e / PN;
+  float acc = init ? init[e] : 0.f;
+  for (int q = 0; q < rank; ++q) acc = fmaf(expf(logdecay[q * H + h]), acc, states[q * H * PN + e]);
+  out[e] = acc;
+}
+
+}  // namespace
+}  // namespace ssd
+
+extern "C" int ssd_segment_logdecay(int64_t tokens, int64_t nheads, const float* dt, const float* A, float* out,
+                                    ssd_stream_t stream) {
+  if (tokens < 0 || nheads <= 0 || nheads > (1 << 24)) return SSD_ERR_INVALID_ARG;
+  if (!dt || !A || !out) return SSD_ERR_INVALID_ARG;
+  const unsigned blocks = (unsigned)((nheads + ssd::kHeadsPerBlock - 1) / ssd::kHeadsPerBlock);
+  ssd::segment_logdecay_kernel<<<blocks, ssd::kHeadsPerBlock * ssd::kTokLanes, 0, (cudaStream_t)stream>>>(
+      tokens, (int)nheads, dt, A, out);
+  ssd::count_launches(1);
+  return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
+
+extern "C" int ssd_state_prefix(int rank, int64_t nheads, int64_t headdim, int64_t dstate, const float* states,
+                                const float* logdecay, const float* init_state, float* out, ssd_stream_t stream) {
+  if (rank < 0 || nheads <= 0 || headdim <= 0 || dstate <= 0) return SSD_ERR_INVALID_ARG;
+  if (!out || (rank > 0 && (!states || !logdecay))) return SSD_ERR_INVALID_ARG;
+  const int64_t n = nheads * headdim * dstate;
+  if (n > ((int64_t)1 << 40)) return SSD_ERR_UNSUPPORTED;
+  ssd::state_prefix_kernel<<<(unsigned)((n + 255) / 256), 256, 0, (cudaStream_t)stream>>>(
+      rank, nheads, headdim * dstate, states, logdecay, init_state, out);
+  ssd::count_launches(1);
+  return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
+}
