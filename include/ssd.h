@@ -90,6 +90,8 @@ typedef struct {
  *   chunk       Q in {64, 128, 256}: length of the chunks of the block decomposition
  *   y           (batch, seqlen, H, P)  io_dtype   output (may not alias an input)
  *   final_state (nseq_or_batch, H, P, N) fp32     state after each sequence, or NULL
+ * When the shape has no tokens (every sequence empty), x, dt, B, C and y may be NULL and
+ * final_state gets init_state (or zeros).
  * Returns SSD_OK or an error code (see ssd_status).  Asynchronous on `stream`.
  */
 int ssd_forward(const ssd_shape* shape, const void* x, const float* dt, const float* A, const void* B,

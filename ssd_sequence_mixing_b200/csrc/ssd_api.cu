@@ -84,8 +84,8 @@ int validate(const ssd_shape* s, const void* x, const float* dt, const float* A,
   const int64_t tokens = s->batch * s->seqlen;
   if (tokens > ((int64_t)1 << 30) || tokens * s->nheads * s->headdim > ((int64_t)1 << 40))
     return SSD_ERR_UNSUPPORTED;
-  if (!A || !dt) return SSD_ERR_INVALID_ARG;
-  if (tokens > 0 && (!x || !B || !C || !y)) return SSD_ERR_INVALID_ARG;
+  if (!A) return SSD_ERR_INVALID_ARG;
+  if (tokens > 0 && (!x || !dt || !B || !C || !y)) return SSD_ERR_INVALID_ARG;  // empty inputs may be NULL
   if (s->cu_seqlens_host) {
     const int32_t* c = s->cu_seqlens_host;
     if (c[0] != 0 || (int64_t)c[s->nseq] != tokens) return SSD_ERR_BAD_SEQLENS;

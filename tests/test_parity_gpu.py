@@ -214,3 +214,61 @@ def test_full_size_sampled(wl):
     pairs = sample_pairs(prob, k=6)
     check(prob, y, fin, pairs=pairs)
     assert torch.isfinite(y.float()).all()
+
+
+# ------------------------------------------------------------------ edge cases
+def test_all_sequences_empty_gives_init_as_final():
+    """Packed sequences that are all empty: no y rows; every final state equals its init."""
+    lens = [0, 0, 0]
+    wl = workloads.custom(1, 0, H=4, P=64, N=64, G=1, chunk=128, dtype="bf16", init=True, lengths=lens)
+    prob = workloads.generate(wl, seed=13, lengths=lens)
+    dev = to_device(prob)
+    for name, path in [("simt", ssd.PATH_SIMT), ("auto", ssd.PATH_AUTO)]:
+        old = ssd.set_path(path)
+        try:
+            y, fin = ssd.ssd_forward(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init_state"],
+                                     dev["cu_seqlens"], 128)
+        finally:
+            ssd.set_path(old)
+        torch.cuda.synchronize()
+        assert y.numel() == 0 and ssd.query_status() == 0
+        assert torch.equal(fin, dev["init_state"]), name
+
+
+def test_largest_head_and_state_sizes():
+    """P = N = 256 (the largest the boundary takes) on the SIMT path, fp32 and bf16."""
+    for dtype in ("f32", "bf16"):
+        wl = workloads.custom(1, 200, H=2, P=256, N=256, G=1, chunk=64, dtype=dtype, init=True)
+        prob = workloads.generate(wl, seed=14)
+        y, fin = run(prob)
+        check(prob, y, fin)
+
+
+SWEEP = np.random.default_rng(2024)
+
+
+def _sweep_cases(n=10):
+    cases = []
+    for k in range(n):
+        G = int(SWEEP.choice([1, 2]))
+        H = G * int(SWEEP.choice([2, 4]))
+        P = int(SWEEP.choice([16, 32, 64]))
+        N = int(SWEEP.choice([16, 64, 128]))
+        Q = int(SWEEP.choice([64, 128, 256]))
+        dtype = str(SWEEP.choice(["bf16", "f32"]))
+        lens = [int(v) for v in SWEEP.integers(0, 600, int(SWEEP.integers(1, 5)))]
+        cases.append((k, H, P, N, G, Q, dtype, lens))
+    return cases
+
+
+@pytest.mark.parametrize("case", _sweep_cases(), ids=lambda c: "sweep{}_H{}_P{}_N{}_G{}_Q{}_{}".format(*c[:7]))
+def test_seeded_shape_sweep(case):
+    """Seeded random shapes, chunk lengths, dtypes and packed length mixes, every path."""
+    k, H, P, N, G, Q, dtype, lens = case
+    if sum(lens) == 0:
+        lens = lens + [1]
+    wl = workloads.custom(1, 0, H=H, P=P, N=N, G=G, chunk=Q, dtype=dtype, init=bool(k % 2), lengths=lens)
+    prob = workloads.generate(wl, seed=100 + k, lengths=lens)
+    for name, path in paths_for(prob, Q):
+        y, fin = run(prob, path=path)
+        check(prob, y, fin)
