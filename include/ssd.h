@@ -144,8 +144,9 @@ int ssd_forward_host(const ssd_shape* shape, const void* x, const float* dt, con
  * Who needs it: a caller that reserves the GPU's memory up front and hands it out
  * itself (an inference server that gives nearly all HBM to weights and KV caches, or
  * a runtime that accounts for every byte through its own pool) cannot let a library
- * call cudaMallocAsync: the allocation can fail once the pool is spent, and it can
- * stall a latency-critical loop while the driver grows or trims the pool.
+ * allocate device memory (cudaMallocAsync or a pool of its own): the allocation can
+ * fail once the memory is spent, and it can stall a latency-critical loop while the
+ * driver grows or trims a pool.
  *
  * Same arguments, layouts and results as ssd_forward.  It always runs the SIMT
  * kernels, and their scratch (chunk table, cumsums, chunk states) lives in one

@@ -1,24 +1,30 @@
 // ssd_tc.cu -- the tensor-core path: one fused sm_100a kernel for the whole chunked
 // SSD forward pass ("Transformers are SSMs", wikillm.com card, Method step 5, sec. 6).
 //
-// A CTA owns one (sequence, head) at a time and walks the sequence in 128-token
-// tiles (the tcgen05 M).  The P x N state never leaves the chip: each of the 128
-// threads keeps one column n of the fp32 state in registers.  Per tile:
+// One persistent CTA per SM walks an equal share of the flat list of 128-token tiles
+// (the tcgen05 M) of all units (sequence, pair of heads sharing a B/C group), handing
+// the state on through global memory where its share starts or ends inside a unit.
+// The P x N state of each head never leaves the chip: it stays in fp32 in tensor
+// memory, with a bf16 copy in shared memory as an MMA operand.  Per tile:
 //
-//   cumsum   cs_j = running in-chunk cumsum of dt_j A_h (restarted at each chunk
-//            start, so a 256-token chunk spans two tiles)
-//   MMA  S   = C B^T                                   (128 x 128, K = N)
+//   cumsum   cs_j = running in-chunk cumsum of dt_j A_h in log2 units (restarted at
+//            each chunk start, so a 256-token chunk spans two tiles)   [helper warps]
+//   MMA  S   = C B^T                                   (128 x 128, K = N, once per pair)
+//   MMA  Yo  = C [h0 h1]^T        left factor           (128 x 128, K = N)
+//   MMA  h^T += B^T [w0 o x0 | w1 o x1]   right factor  (N x 128, K = 128),
+//            w_j = exp(cs_end - cs_j) dt_j, onto the decay-scaled state
 //   mask     P_ij = S_ij exp(cs_i - cs_j) dt_j for j <= i, else 0 (mask before exp),
-//            written as bf16 to shared memory
-//   MMA  Y   = P X                 diagonal block      (128 x 64, K = 128)
-//   MMA  Yo  = C h^T               left factor         (128 x 64, K = N)
-//   MMA  s^T = B^T (w o X)         right factor        (N x 64, K = 128), w_j = exp(cs_end - cs_j) dt_j
-//   epilogue y_i = Y_i + exp(cs_i - cs_start) Yo_i + D x_i  (bf16 store)
-//            h  <- exp(cs_end - cs_start) h + s          (centre factor, in registers)
+//            written as bf16 pairs to tensor memory
+//   scale    Y_i = exp(cs_i - cs_start) Yo_i
+//   MMA  Y  += P_h x_h            diagonal block, A from tensor memory  (128 x 64, K = 128)
+//   state    h <- exp(cs_end' - cs_start') h for the next tile (centre factor), its bf16
+//            copy, or the final state / hand-on at the end of a piece
+//   epilogue y_i = Y_i + D x_i    (bf16, staged over the x tile, TMA store)
 //
-// Operands come from shared memory: x, B, C by TMA with 128-byte swizzle; P, w o X
-// and the bf16 copy of h are written by the threads in the same swizzled layouts.
-// Accumulators live in tensor memory (S 128 cols, Y 64, Yo 64, s^T 64).
+// Roles: 16 compute warps (per head, two column halves x four lane quarters), one
+// issuer warp (every TMA load of x, B, C and every tcgen05.mma) and two helper warps
+// (dt loads and the per-tile descriptors: cumsums, column factors, decays, flags).
+// Tensor memory: S 128 columns, P 2 x 64, Y 2 x 64, h^T 2 x 64.
 // Every wait is bounded; a wait that gives up records SSD_ERR_DEVICE_TIMEOUT in the
 // status word, drains what is in flight (bounded), frees tensor memory and exits.
 #include <cuda.h>
