@@ -12,6 +12,10 @@ the max over ranks.  Rank 0 prints one JSON line.
 
 ``--impl reference`` times the fp64 CPU oracle instead (rank 0 only) on bounded
 samples of the same workload.
+
+On one GPU the line also carries ``next``: the decode step, the causal conv1d +
+SiLU and the gated RMSNorm timed at the same layer's shapes (``--no-decode``
+skips them).
 """
 from __future__ import annotations
 

@@ -5,6 +5,13 @@ module only marshals arguments: shapes are read off torch tensors, outputs are
 allocated with torch when the caller does not pass them, and every step of the
 computation runs in the library's CUDA kernels.  There is no CPU fallback:
 without the built library, importing this package raises.
+
+Entry points: ``ssd_forward`` (device buffers), ``ssd_forward_host`` (host
+buffers, copies pipelined with the compute), ``ssd_forward_noalloc`` (no device
+allocation), ``ssd_forward_dt`` (step size from the raw projection inside the
+kernels), ``ssd_decode_step`` (one generation step), ``causal_conv1d_silu`` and
+``gated_rmsnorm`` (the block's steps around the SSD), ``segment_logdecay`` and
+``state_prefix`` (sequence parallelism, see ``sequence_parallel``).
 """
 from __future__ import annotations
 
