@@ -92,15 +92,15 @@ struct ConvArgs {
   const int32_t* cu;  // (nseq + 1) or null
   void* out;
 };
-constexpr int kConvTok = 8;  // tokens per thread: their inputs and the 3-token halo load at once
+constexpr int kConvTok = 16;  // tokens per thread: their inputs and the 3-token halo load at once
 constexpr int kConvThreads = 128;
 
 __device__ __forceinline__ int64_t seq_start_of(const ConvArgs& a, int64_t s) {
   return a.cu ? (int64_t)a.cu[s] : s * a.seqlen;
 }
 
-// Grid: ceil(channels / 8 / 128) channel blocks x ceil(tokens / 8) token blocks, flattened
-// (channel block fastest).  A thread computes 8 channels of 8
+// Grid: ceil(channels / 8 / 128) channel blocks x ceil(tokens / 16) token blocks, flattened
+// (channel block fastest).  A thread computes 8 channels of 16
 // consecutive tokens: it loads those tokens and the three before them (the halo, an L2 hit
 // after the neighbouring thread block's load) in one go, then walks them in order.  Inputs
 // before the start of a token's sequence count as zero.
