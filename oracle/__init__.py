@@ -16,7 +16,13 @@ leg may import this package.  It shares no code with the CUDA path.
 * ``causal_conv1d_silu`` and ``gated_rmsnorm``: the block's steps before and after the
   SSD (the Mamba-2 block sketch of sec. 7.1; "Paper vs code" 1, 2 and 9).
 
-Parity status of every function here is recorded in the tests that pin it.
+Pins (``tests/test_oracle_pins.py``): ``ssd_forward`` against a dense semiseparable
+brute force, textbook special cases, closed forms, hand-worked values and the
+chunked restatement; ``decode_step`` against the dense matrix; ``dt_prologue``
+against softplus closed forms and the inverse softplus; ``causal_conv1d_silu``
+against an impulse response, a sequence reset and numpy's convolution;
+``gated_rmsnorm`` against closed forms (gate off, constant gate, unit RMS).  No
+function here is unpinned.
 """
 from __future__ import annotations
 
