@@ -51,11 +51,13 @@ def problem(seed, T=90, H=3, P=4, N=5, G=1):
     return [torch.from_numpy(v) for v in (x, dt, A, B, C, D, init)]
 
 
-def _rank(rank, world, port, cuts, out):
+def _rank(rank, world, port, cuts, variant, out):
     os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
-        x, dt, A, B, C, D, init = problem(7)
+        x, dt, A, B, C, D, init = problem(7, **variant)
+        if variant.get("G") == 2:
+            init, D = None, None  # no initial state, no skip
         a, e = cuts[rank], cuts[rank + 1]
         seg = lambda v: v[:, a:e].contiguous()
         y, fin = forward_sequence_parallel(seg(x), seg(dt), A, seg(B), seg(C), D, init, steps=oracle_steps())
@@ -64,14 +66,18 @@ def _rank(rank, world, port, cuts, out):
         dist.destroy_process_group()
 
 
-@pytest.mark.parametrize("cuts", [[0, 40, 90], [0, 1, 60, 90], [0, 30, 30, 90]], ids=["two", "three", "empty_middle"])
-def test_sequence_parallel_equals_one_pass(cuts):
+@pytest.mark.parametrize("cuts,variant", [([0, 40, 90], {}), ([0, 1, 60, 90], {}), ([0, 30, 30, 90], {}),
+                                          ([0, 45, 90], {"H": 4, "G": 2})],
+                         ids=["two", "three", "empty_middle", "two_groups_no_init_no_skip"])
+def test_sequence_parallel_equals_one_pass(cuts, variant):
     world = len(cuts) - 1
     out = mp.Manager().dict()
-    mp.spawn(_rank, args=(world, _free_port(), cuts, out), nprocs=world, join=True)
-    x, dt, A, B, C, D, init = problem(7)
+    mp.spawn(_rank, args=(world, _free_port(), cuts, variant, out), nprocs=world, join=True)
+    x, dt, A, B, C, D, init = problem(7, **variant)
+    if variant.get("G") == 2:
+        init, D = None, None
     y_ref, fin_ref = oracle.ssd_forward(x[0].numpy(), dt[0].numpy(), A.numpy(), B[0].numpy(), C[0].numpy(),
-                                        D.numpy(), init.numpy())
+                                        None if D is None else D.numpy(), None if init is None else init.numpy())
     y = np.concatenate([out[r][0][0] for r in range(world)], 0)
     assert np.allclose(y, y_ref, rtol=1e-10, atol=1e-12)
     assert np.allclose(out[world - 1][1], fin_ref, rtol=1e-10, atol=1e-12)
