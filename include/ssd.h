@@ -29,7 +29,8 @@
  *  - The return value is an ssd_status.  On any host-detected error nothing is
  *    launched and no output is written.  Errors found on the device (bad
  *    cu_seqlens values, a bounded wait that ran out) are recorded in a per-device
- *    status word, read with ssd_query_status().
+ *    status word, read with ssd_query_status().  With SSD_DEBUG set in the
+ *    environment, a failed tensor-core launch also prints its CUDA error to stderr.
  */
 #ifndef SSD_H_
 #define SSD_H_
