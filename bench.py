@@ -13,9 +13,12 @@ the max over ranks.  Rank 0 prints one JSON line.
 ``--impl reference`` times the fp64 CPU oracle instead (rank 0 only) on bounded
 samples of the same workload.
 
-On one GPU the line also carries ``next``: the decode step, the causal conv1d +
-SiLU and the gated RMSNorm timed at the same layer's shapes (``--no-decode``
-skips them).
+On one GPU the line also carries ``workloads``: every workload of the table
+(the layer, the state-size sweep, the length sweep and the packed batch), each
+with tokens/s, the dominant kernel's time, its roofline fraction and the path it
+took (``--no-workloads`` skips them); and ``next``: the decode step, the causal
+conv1d + SiLU and the gated RMSNorm timed at the same layer's shapes
+(``--no-decode`` skips them).
 """
 from __future__ import annotations
 
@@ -298,6 +301,7 @@ def run_ours(args, rank, world, local_rank):
         b.synchronize()
         e2e_ms.append(a.elapsed_time(b))
     e2e_value = weak_scaling_value(wl.tokens, args.e2e_steps, world, aggregate_max(sum(e2e_ms) / 1e3, world, dev))
+    link = host_link_gbs(dev) if rank == 0 else None
 
     if rank != 0:
         return None
@@ -341,15 +345,127 @@ def run_ours(args, rank, world, local_rank):
                      "step_roofline_us": roof_s * 1e6, "step_frac": roof_s / step_s},
         "e2e": {"value": e2e_value, "unit": "tokens/s", "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "steps": args.e2e_steps, "ms_per_step": statistics.mean(e2e_ms),
-                "api": "ssd_forward_host (pinned host buffers)"},
+                "api": "ssd_forward_host (pinned host buffers)",
+                # the host link measured on this machine, and the copy time it allows per step
+                "link": link,
+                "link_bound_ms": 1e3 * max(h2d / (link["h2d_gbs"] * 1e9), d2h / (link["d2h_gbs"] * 1e9),
+                                           (h2d + d2h) / (link["bidir_gbs"] * 1e9)),
+                "link_frac": 1e3 * max(h2d / (link["h2d_gbs"] * 1e9), d2h / (link["d2h_gbs"] * 1e9),
+                                       (h2d + d2h) / (link["bidir_gbs"] * 1e9)) / statistics.mean(e2e_ms)},
         "gpu_launches": int(launches),
         "clocks": clocks,
     }
+    if world == 1 and not args.no_workloads:
+        # configs 1-4 of the workload table (the tiny parity case is launch-bound)
+        out["workloads"] = [workload_measurement(w, dev, stream, flush) for w in workloads.ALL
+                            if w is not workloads.TINY]
     if world == 1 and not args.no_decode:
         out["next"] = {"decode_step": decode_measurement(dev, stream, flush)}
         out["next"].update(block_measurements(dev, stream, flush))
     if world == 1 and not args.no_cpu_baseline:
         out["cpu_baseline"] = cpu_baseline(prob, budget_s=args.cpu_budget)
+    return out
+
+
+# ------------------------------------------------------------- the host link
+def host_link_gbs(dev, nbytes: int = 256 << 20, reps: int = 5):
+    """Pinned host <-> device copy bandwidth of this machine (GB/s, best of ``reps``): host to
+    device alone, device to host alone, and both directions at once on two streams."""
+    h_src = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    h_dst = torch.empty(nbytes, dtype=torch.uint8).pin_memory()
+    d_a = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    d_b = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    s_in, s_out = torch.cuda.Stream(dev), torch.cuda.Stream(dev)
+
+    def once(h2d: bool, d2h: bool) -> float:
+        start = torch.cuda.Event(enable_timing=True)
+        ends = []
+        start.record(s_in)
+        s_out.wait_event(start)
+        if h2d:
+            with torch.cuda.stream(s_in):
+                d_a.copy_(h_src, non_blocking=True)
+                e = torch.cuda.Event(enable_timing=True)
+                e.record(s_in)
+                ends.append(e)
+        if d2h:
+            with torch.cuda.stream(s_out):
+                h_dst.copy_(d_b, non_blocking=True)
+                e = torch.cuda.Event(enable_timing=True)
+                e.record(s_out)
+                ends.append(e)
+        torch.cuda.synchronize(dev)
+        return max(start.elapsed_time(e) for e in ends) / 1e3
+
+    out = {}
+    for name, h2d, d2h in (("h2d_gbs", True, False), ("d2h_gbs", False, True), ("bidir_gbs", True, True)):
+        t = min(once(h2d, d2h) for _ in range(reps))
+        out[name] = (int(h2d) + int(d2h)) * nbytes / t / 1e9
+    return out
+
+
+# ------------------------------------------------- every workload of the table
+def roofline_line(wl, prob, dom_s, peaks, peak_kind):
+    """Roofline of one ssd_forward workload: max(bytes / HBM peak, FLOPs / bf16 peak)."""
+    nbytes = algorithmic_bytes(wl, prob.init_state is not None, prob.nseq)
+    lens = [prob.seq_offsets[i + 1] - prob.seq_offsets[i] for i in range(prob.nseq)]
+    flops = algorithmic_flops(wl, lens)
+    t_mem = nbytes / (peaks["hbm_gbs"] * 1e9)
+    t_flop = flops / (peaks["bf16_tflops"] * 1e12)
+    if t_mem >= t_flop:
+        bound, achieved, peak, unit = "hbm", nbytes / dom_s / 1e9, peaks["hbm_gbs"], "GB/s"
+    else:
+        bound, achieved, peak, unit = "tensor", flops / dom_s / 1e12, peaks["bf16_tflops"], "TFLOP/s"
+    return {"bound": bound, "achieved": achieved, "peak": peak, "unit": unit, "frac": achieved / peak,
+            "peak_source": f"{peak_kind} ({unit})", "algorithmic_bytes": nbytes, "algorithmic_flops": flops,
+            "roofline_us": max(t_mem, t_flop) * 1e6}
+
+
+def workload_measurement(wl, dev, stream, flush, steps=10, warmup=3):
+    """Time one ssd_forward call on workload ``wl`` (seeded synthetic inputs resident in
+    HBM, L2 flushed between steps): step time and the dominant kernel's time from the
+    library's events, median over ``steps``."""
+    import ssd_sequence_mixing_b200 as ssd
+
+    prob = workloads.generate(wl, seed=0)
+    d = {k: (None if getattr(prob, k) is None else getattr(prob, k).to(dev))
+         for k in ("x", "dt", "A", "B", "C", "D", "init_state", "cu_seqlens")}
+    y = torch.empty_like(d["x"])
+    fin = torch.empty((prob.nseq, wl.nheads, wl.headdim, wl.dstate), dtype=torch.float32, device=dev)
+    shape = ssd.make_shape(d["x"], d["B"], d["cu_seqlens"])
+    path = {ssd.PATH_SIMT: "simt", ssd.PATH_TC: "tc"}.get(ssd.select_path(shape, wl.chunk), "?")
+
+    def step():
+        ssd.ssd_forward(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["init_state"], d["cu_seqlens"], wl.chunk,
+                        y=y, final_state=fin, stream=stream)
+
+    for _ in range(warmup):
+        flush.zero_()
+        step()
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    dom = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
+    for a, b in dom:
+        a.record(stream)
+        b.record(stream)
+    torch.cuda.synchronize()
+    for k in range(steps):
+        flush.zero_()
+        ssd.profile_dominant(*dom[k])
+        ev[k][0].record(stream)
+        step()
+        ev[k][1].record(stream)
+    torch.cuda.synchronize()
+    ssd.profile_dominant(None, None)
+    assert ssd.query_status() == 0
+    step_s = statistics.median(a.elapsed_time(b) for a, b in ev) / 1e3
+    dom_s = statistics.median(a.elapsed_time(b) for a, b in dom) / 1e3
+    peaks, kind = load_peaks()
+    roof = roofline_line(wl, prob, dom_s, peaks, kind)
+    out = {"workload": wl.name, "path": path, "tokens": wl.tokens, "tokens_per_s": wl.tokens / step_s,
+           "step_us": step_s * 1e6, "dominant_us": dom_s * 1e6, "roofline": roof,
+           "step_frac": roof["roofline_us"] / (step_s * 1e6)}
+    del d, y, fin
+    torch.cuda.empty_cache()
     return out
 
 
@@ -483,6 +599,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true",
                     help="skip the measurements of the decode step and the block steps around the SSD")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the per-workload measurements (state-size and length sweeps, packed batch)")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
     ap.add_argument("--ref-heads", type=int, default=16)
     args = ap.parse_args()

@@ -92,7 +92,9 @@ typedef struct {
  *   y           (batch, seqlen, H, P)  io_dtype   output (may not alias an input)
  *   final_state (nseq_or_batch, H, P, N) fp32     state after each sequence, or NULL
  * When the shape has no tokens (every sequence empty), x, dt, B, C and y may be NULL and
- * final_state gets init_state (or zeros).
+ * final_state gets init_state (or zeros).  With y == NULL and final_state given, only the
+ * final states are computed: C and D are not read (either may be NULL), and the
+ * tensor-core kernel loads only x, dt and B (the first pass of sequence parallelism).
  * Returns SSD_OK or an error code (see ssd_status).  Asynchronous on `stream`.
  */
 int ssd_forward(const ssd_shape* shape, const void* x, const float* dt, const float* A, const void* B,
@@ -132,7 +134,9 @@ int ssd_forward_dt(const ssd_shape* shape, const ssd_dt_prologue* prologue, cons
  * returning.  Every sequence's outputs are the ones a single ssd_forward call gives.
  * Same layouts and errors as ssd_forward; cu_seqlens is a host pointer here and is
  * checked on the host (SSD_ERR_BAD_SEQLENS).  Returns SSD_ERR_DEVICE_TIMEOUT when the
- * device reported one during this call.
+ * device reported one during this call.  The two copy streams and their events are
+ * created on a device's first call and kept; calls on one device from several host
+ * threads take turns (a per-device lock).
  */
 int ssd_forward_host(const ssd_shape* shape, const void* x, const float* dt, const float* A, const void* B,
                      const void* C, const float* D, const float* init_state, const int32_t* cu_seqlens, int chunk,
@@ -157,9 +161,10 @@ int ssd_forward_host(const ssd_shape* shape, const void* x, const float* dt, con
  *  - Shapes whose scratch exceeds SSD_NOALLOC_SCRATCH_BYTES (ssd_workspace_bytes with
  *    ssd_set_path(SSD_PATH_SIMT) gives the need) return SSD_ERR_SCRATCH_LIMIT and
  *    launch nothing.
- *  - The first call on a device looks up the array's device address on that device
- *    (cudaGetSymbolAddress, with that device current); make that first call before any
- *    stream capture.
+ *  - Every call looks up the array's device address on the current device
+ *    (cudaGetSymbolAddress, which allocates nothing), so a context recreated after a
+ *    device reset gets its own copy of the array.  The first call on a device loads
+ *    the module there; make that first call before any stream capture.
  *  - All calls share the one array and it keeps the last call's contents; each call
  *    first resets the word that marks the chunk table as not yet built.  Calls whose
  *    work overlaps on the GPU (different streams, or different host threads, without
@@ -284,6 +289,19 @@ typedef struct CUevent_st* ssd_event_t;
  */
 int ssd_profile_dominant(ssd_event_t start, ssd_event_t stop);
 uint64_t ssd_kernel_launch_count(void);
+
+/*
+ * Test hooks for the failure path of the tensor-core kernel (process-wide, not
+ * thread-safe; meant for tests).  Every device-side wait of that kernel is bounded:
+ * after `wait_limit_cycles` SM clock cycles (0 = the default, 2^32, about 2 s) it gives
+ * up, the kernel drains its in-flight copies and tensor-core work, frees tensor memory
+ * and returns, and ssd_query_status() reports SSD_ERR_DEVICE_TIMEOUT; the outputs of
+ * that call are then undefined.  withhold_carry = 1 makes every CTA keep back the flag
+ * that hands its state on to the next CTA (the state itself is still written), so the
+ * CTAs that wait for it run out of time: the only way a test makes a wait fail.
+ * Returns SSD_OK, or SSD_ERR_INVALID_ARG for a negative limit.
+ */
+int ssd_set_test_hooks(int64_t wait_limit_cycles, int withhold_carry);
 
 #ifdef __cplusplus
 }

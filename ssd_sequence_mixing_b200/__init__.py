@@ -56,6 +56,7 @@ EXPORTS = (
     "ssd_gated_rmsnorm",
     "ssd_segment_logdecay",
     "ssd_state_prefix",
+    "ssd_set_test_hooks",
 )
 
 
@@ -124,6 +125,8 @@ def _open() -> ctypes.CDLL:
     lib.ssd_segment_logdecay.restype = I
     lib.ssd_state_prefix.argtypes = [I, L, L, L, V, V, V, V, V]
     lib.ssd_state_prefix.restype = I
+    lib.ssd_set_test_hooks.argtypes = [L, I]
+    lib.ssd_set_test_hooks.restype = I
     return lib
 
 
@@ -223,6 +226,40 @@ def ssd_forward(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Ten
     if rc:
         raise SsdError(rc, "ssd_forward")
     return y, final_state
+
+
+def ssd_final_state(x: torch.Tensor, dt: torch.Tensor, A: torch.Tensor, B: torch.Tensor,
+                    init_state: Optional[torch.Tensor] = None, cu_seqlens: Optional[torch.Tensor] = None,
+                    chunk: int = 256, final_state: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+    """Only the state after each sequence: ssd_forward with y = NULL, which reads neither C
+    nor D (the tensor-core kernel then loads x, dt and B alone).  Returns final_state
+    (rows, H, P, N) fp32."""
+    device = x.device
+    if device.type != "cuda":
+        raise ValueError("ssd_final_state takes CUDA tensors")
+    batch, T, H, P = x.shape
+    G, N = B.shape[2], B.shape[3]
+    rows = cu_seqlens.numel() - 1 if cu_seqlens is not None else batch
+    _check("x", x, device)
+    _check("dt", dt, device, torch.float32, (batch, T, H))
+    _check("A", A, device, torch.float32, (H,))
+    _check("B", B, device, x.dtype, (batch, T, G, N))
+    _check("init_state", init_state, device, torch.float32, (rows, H, P, N))
+    _check("cu_seqlens", cu_seqlens, device, torch.int32)
+    if final_state is None:
+        final_state = torch.empty((rows, H, P, N), dtype=torch.float32, device=device)
+    _check("final_state", final_state, device, torch.float32, (rows, H, P, N))
+    shape = make_shape(x, B, cu_seqlens)
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    handle = stream.cuda_stream if hasattr(stream, "cuda_stream") else int(stream)
+    with torch.cuda.device(device):
+        rc = _lib.ssd_forward(ctypes.byref(shape), _ptr(x), _ptr(dt), _ptr(A), _ptr(B), None, None,
+                              _ptr(init_state), _ptr(cu_seqlens), int(chunk), None, _ptr(final_state),
+                              ctypes.c_void_p(handle))
+    if rc:
+        raise SsdError(rc, "ssd_forward (final state only)")
+    return final_state
 
 
 def ssd_forward_noalloc(x, dt, A, B, C, D=None, init_state=None, cu_seqlens=None, chunk: int = 256,
@@ -464,3 +501,13 @@ def profile_dominant(start=None, stop=None) -> None:
 def kernel_launch_count() -> int:
     """Kernels launched by the library so far in this process."""
     return int(_lib.ssd_kernel_launch_count())
+
+
+def set_test_hooks(wait_limit_cycles: int = 0, withhold_carry: bool = False) -> None:
+    """Test hooks of the tensor-core kernel's failure path: the cycle limit of every
+    device-side wait (0 = the default, about 2 s) and whether CTAs withhold the flag that
+    hands their state on (so that the CTAs waiting for it time out).  Defaults restore
+    normal operation."""
+    rc = _lib.ssd_set_test_hooks(int(wait_limit_cycles), 1 if withhold_carry else 0)
+    if rc:
+        raise SsdError(rc, "ssd_set_test_hooks")

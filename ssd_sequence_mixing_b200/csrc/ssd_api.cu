@@ -5,6 +5,8 @@
 #include <string.h>
 
 #include <atomic>
+#include <chrono>
+#include <mutex>
 #include <vector>
 
 #include "ssd.h"
@@ -21,6 +23,10 @@ std::atomic<unsigned int*> g_status_ptr[kMaxDevices];
 std::atomic<int> g_path{SSD_PATH_AUTO};
 std::atomic<uint64_t> g_launches{0};
 std::atomic<cudaEvent_t> g_prof_start{nullptr}, g_prof_stop{nullptr};
+// Device-side waits give up after this many SM cycles (about 2 s at the B200's clock).
+constexpr long long kDefaultWaitLimit = 4ll << 30;
+std::atomic<long long> g_wait_limit{kDefaultWaitLimit};
+std::atomic<int> g_withhold_carry{0};
 
 unsigned int* status_ptr() {
   int dev = 0;
@@ -36,6 +42,22 @@ unsigned int* status_ptr() {
 }
 
 bool aligned16(const void* p) { return ((uintptr_t)p & 15u) == 0; }
+
+// A value no earlier launch of this process used: the tensor-core kernel's carry flags
+// are set to it, so flags left over in reused scratch never look published.  The high
+// half is drawn from the address of a stack variable and the clock once per process.
+uint64_t next_epoch() {
+  static std::atomic<uint64_t> counter{0};
+  static const uint64_t salt = [] {
+    int probe = 0;
+    uint64_t v = (uint64_t)(uintptr_t)&probe ^ (uint64_t)std::chrono::steady_clock::now().time_since_epoch().count();
+    v ^= v >> 29;
+    v *= 0xbf58476d1ce4e5b9ull;
+    v ^= v >> 32;
+    return v << 32;
+  }();
+  return salt | ((counter.fetch_add(1) + 1) & 0xffffffffull);
+}
 
 // The library's stream-ordered pool on the current device: scratch and the host entry
 // point's device buffers come from it, and freed blocks stay cached for the next call
@@ -72,7 +94,7 @@ int64_t nstate_rows(const ssd_shape* s, const int32_t* cu) { return cu ? s->nseq
 // Host-side validation shared by every entry point.  `cu` is the (device or host)
 // cu_seqlens pointer as passed by the caller; only its nullness is used here.
 int validate(const ssd_shape* s, const void* x, const float* dt, const float* A, const void* B, const void* C,
-             const int32_t* cu, int chunk, const void* y) {
+             const int32_t* cu, int chunk, const void* y, bool state_only = false) {
   if (!s) return SSD_ERR_INVALID_ARG;
   if (s->batch < 0 || s->seqlen < 0 || s->nheads <= 0 || s->headdim <= 0 || s->dstate <= 0 || s->ngroups <= 0)
     return SSD_ERR_INVALID_ARG;
@@ -85,7 +107,7 @@ int validate(const ssd_shape* s, const void* x, const float* dt, const float* A,
   if (tokens > ((int64_t)1 << 30) || tokens * s->nheads * s->headdim > ((int64_t)1 << 40))
     return SSD_ERR_UNSUPPORTED;
   if (!A) return SSD_ERR_INVALID_ARG;
-  if (tokens > 0 && (!x || !dt || !B || !C || !y)) return SSD_ERR_INVALID_ARG;  // empty inputs may be NULL
+  if (tokens > 0 && (!x || !dt || !B || (!state_only && (!C || !y)))) return SSD_ERR_INVALID_ARG;  // empty inputs may be NULL
   if (s->cu_seqlens_host) {
     const int32_t* c = s->cu_seqlens_host;
     if (c[0] != 0 || (int64_t)c[s->nseq] != tokens) return SSD_ERR_BAD_SEQLENS;
@@ -130,13 +152,39 @@ Scratch scratch_layout(const ssd_shape* s, const int32_t* cu, int chunk, int pat
   w.total = w.seq_tiles;
   w.ranges = 0;
   if (path == SSD_PATH_TC) {
-    // one CTA per SM; each may hand a (2 heads x P x N) fp32 state and two cumsums on
+    // one CTA per SM; each may hand a (2 heads x P x N) fp32 state on, with one flag per
+    // compute warp (16)
     w.ranges = device_sms();
     w.carry = w.seq_tiles + up(sizeof(int32_t) * (size_t)(nseq + 1));
-    w.carry_flag = w.carry + up(sizeof(float) * (size_t)w.ranges * 2 * (s->headdim * s->dstate + 1));
-    w.total = w.carry_flag + up(sizeof(int32_t) * (size_t)w.ranges);
+    w.carry_flag = w.carry + up(sizeof(float) * (size_t)w.ranges * 2 * s->headdim * s->dstate);
+    w.total = w.carry_flag + up(sizeof(uint64_t) * 16 * (size_t)w.ranges);
   }
   return w;
+}
+
+// ssd_forward_host's two copy streams (in, out) and its events, one set per device,
+// created on first use and kept for the life of the process.
+constexpr int kHostGroups = 8;
+struct HostCopies {
+  std::mutex mu;
+  bool ready = false;
+  cudaStream_t sin = nullptr, sout = nullptr;
+  cudaEvent_t ev[2 * kHostGroups + 1] = {};
+  bool create() {
+    if (cudaStreamCreateWithFlags(&sin, cudaStreamNonBlocking) != cudaSuccess ||
+        cudaStreamCreateWithFlags(&sout, cudaStreamNonBlocking) != cudaSuccess)
+      return false;
+    for (auto& e : ev)
+      if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return false;
+    ready = true;
+    return true;
+  }
+};
+HostCopies g_host_copies[kMaxDevices];
+HostCopies* host_copies() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  return &g_host_copies[dev];
 }
 
 int select_path(const ssd_shape* s, int chunk) {
@@ -149,9 +197,73 @@ int select_path(const ssd_shape* s, int chunk) {
 
 int forward_impl(const ssd_shape* s, const void* x, const float* dt, const float* A, const void* B, const void* C,
                  const float* D, const float* init, const int32_t* cu, int chunk, void* y, float* fin,
-                 cudaStream_t st, const ssd_dt_prologue* pro = nullptr) {
-  int rc = validate(s, x, dt, A, B, C, cu, chunk, y);
+                 cudaStream_t st, const ssd_dt_prologue* pro = nullptr);
+
+// Segments per sequence for a dense batch on the tensor-core path.  Its CTAs cut the flat
+// tile list into equal ranges; a unit (sequence, head pair) much longer than a range is
+// processed range after range, each CTA waiting for the state of the one before (at the
+// (2, 65536) length-sweep point a unit is 2.3 ranges long and the kernel takes the time of
+// a whole unit).  Cutting each sequence into k segments of at most a range's length and
+// passing the state between segments as the chunked algorithm passes it between chunks
+// costs one final-state-only pass (x, dt and B again) and removes the wait.
+int segments_for(const ssd_shape* s, int path, const int32_t* cu, const ssd_dt_prologue* pro) {
+  if (path != SSD_PATH_TC || cu || pro || s->batch < 1 || s->seqlen <= 0) return 1;
+  const int64_t tiles = (s->seqlen + ssd::kTcTile - 1) / ssd::kTcTile;
+  const int64_t units = s->batch * (s->nheads / 2);
+  const double share = (double)(units * tiles) / device_sms();  // tiles per CTA
+  if (tiles <= 1.5 * share) return 1;
+  int64_t k = (int64_t)((tiles + share - 1) / share);
+  if (k < 2) return 1;
+  if (s->batch * k > (1 << 20)) return 1;
+  return (int)k;
+}
+
+int forward_segmented(const ssd_shape* s, int k, const void* x, const float* dt, const float* A, const void* B,
+                      const void* C, const float* D, const float* init, int chunk, void* y, float* fin,
+                      cudaStream_t st) {
+  const int64_t L = s->seqlen, tiles = (L + ssd::kTcTile - 1) / ssd::kTcTile;
+  const int64_t seg = (tiles + k - 1) / k * ssd::kTcTile;  // tokens per segment, whole tiles
+  k = (int)((L + seg - 1) / seg);
+  const int nseq = (int)s->batch, nseg = nseq * k;
+  const int64_t H = s->nheads, PN = s->headdim * s->dstate, HPN = H * PN;
+  auto up = [](size_t v) { return (v + 255) & ~(size_t)255; };
+  const size_t o_cu = 0, o_st = up(sizeof(int32_t) * (nseg + 1)), o_lam = o_st + up(sizeof(float) * nseg * HPN),
+               o_h = o_lam + up(sizeof(float) * nseg * H), o_fin = o_h + up(sizeof(float) * nseg * HPN),
+               total = o_fin + (fin ? up(sizeof(float) * nseg * HPN) : 0);
+  char* ws = nullptr;
+  if (pool_alloc((void**)&ws, total, st) != cudaSuccess) return SSD_ERR_CUDA;
+  int32_t* cu = (int32_t*)(ws + o_cu);
+  float *states = (float*)(ws + o_st), *lam = (float*)(ws + o_lam), *h_in = (float*)(ws + o_h);
+  float* seg_fin = fin ? (float*)(ws + o_fin) : nullptr;
+  ssd_shape sg = *s;
+  sg.batch = 1;
+  sg.seqlen = s->batch * L;
+  sg.nseq = nseg;
+  sg.cu_seqlens_host = nullptr;
+  int rc = SSD_OK;
+  if (ssd::launch_segment_offsets(nseq, L, k, seg, cu, st) != cudaSuccess) rc = SSD_ERR_CUDA;
+  // 1. every segment's end state from a zero state (x, dt, B only)
+  if (rc == SSD_OK) rc = forward_impl(&sg, x, dt, A, B, nullptr, nullptr, nullptr, cu, chunk, nullptr, states, st);
+  // 2. the segments' decays and true start states
+  if (rc == SSD_OK && (ssd::launch_segments_logdecay(cu, nseg, (int)H, dt, A, lam, st) != cudaSuccess ||
+                       ssd::launch_segments_prefix(nseq, k, H, PN, states, lam, init, h_in, st) != cudaSuccess))
+    rc = SSD_ERR_CUDA;
+  // 3. the full pass on the segments from their start states
+  if (rc == SSD_OK) rc = forward_impl(&sg, x, dt, A, B, C, D, h_in, cu, chunk, y, seg_fin, st);
+  if (rc == SSD_OK && fin && ssd::launch_segments_final(nseq, k, HPN, seg_fin, fin, st) != cudaSuccess)
+    rc = SSD_ERR_CUDA;
+  if (cudaFreeAsync(ws, st) != cudaSuccess && rc == SSD_OK) rc = SSD_ERR_CUDA;
+  return rc;
+}
+
+int forward_impl(const ssd_shape* s, const void* x, const float* dt, const float* A, const void* B, const void* C,
+                 const float* D, const float* init, const int32_t* cu, int chunk, void* y, float* fin,
+                 cudaStream_t st, const ssd_dt_prologue* pro) {
+  // y == NULL: only the final states are computed (C and D are not read)
+  const bool state_only = y == nullptr && fin != nullptr;
+  int rc = validate(s, x, dt, A, B, C, cu, chunk, y, state_only);
   if (rc) return rc;
+  if (state_only) C = nullptr, D = nullptr;
   if (pro && !(pro->dt_min >= 0.f && pro->dt_max >= pro->dt_min)) return SSD_ERR_INVALID_ARG;  // NaN fails too
   const void* ptrs[] = {x, dt, A, B, C, D, init, cu, y, fin, pro ? pro->dt_bias : nullptr};
   for (const void* p : ptrs)
@@ -163,6 +275,10 @@ int forward_impl(const ssd_shape* s, const void* x, const float* dt, const float
   if (nseq == 0) return SSD_OK;
   unsigned int* status = status_ptr();
   if (!status) return SSD_ERR_CUDA;
+  if (!state_only) {
+    const int k = segments_for(s, path, cu, pro);
+    if (k > 1) return forward_segmented(s, k, x, dt, A, B, C, D, init, chunk, y, fin, st);
+  }
 
   ssd::Problem pb{};
   pb.tokens = tokens;
@@ -207,11 +323,26 @@ int forward_impl(const ssd_shape* s, const void* x, const float* dt, const float
   pb.cs = (float*)(ws + w.cs);
   pb.states = (float*)(ws + w.states);
   pb.seq_tiles = path == SSD_PATH_TC ? (int32_t*)(ws + w.seq_tiles) : nullptr;
+  pb.dense_tiles = (int)((s->seqlen + ssd::kTcTile - 1) / ssd::kTcTile);
   pb.carry = (float*)(ws + w.carry);
-  pb.carry_flag = (int32_t*)(ws + w.carry_flag);
+  pb.carry_flag = (uint64_t*)(ws + w.carry_flag);
+  pb.epoch = next_epoch();
   pb.ranges = w.ranges;
+  pb.wait_limit = g_wait_limit.load();
+  if (path == SSD_PATH_TC && pb.wait_limit == kDefaultWaitLimit) {
+    // A CTA whose range lies inside one unit waits for the CTA before it to finish its
+    // range, and every role of the CTA waits behind it; along a chain of such CTAs the
+    // wait grows with the work ahead.  Allow 16K cycles (about 8 us, several times the
+    // measured cost) per tile of the whole problem on top of the default.
+    const int64_t tiles = (tokens / ssd::kTcTile + nseq) * ((s->nheads + 1) / 2);
+    pb.wait_limit += (long long)tiles * 16384;
+  }
+  pb.withhold_carry = g_withhold_carry.load();
 
-  cudaError_t e = ssd::launch_chunk_table(pb, st);
+  // The chunk table: the SIMT path's chunk records, or the tensor-core path's tile
+  // prefix over packed sequences (a dense batch needs none).
+  cudaError_t e = cudaSuccess;
+  if (path == SSD_PATH_SIMT || cu) e = ssd::launch_chunk_table(pb, st);
   if (e == cudaSuccess) e = path == SSD_PATH_TC ? ssd::launch_tc(pb, st) : ssd::launch_simt(pb, st);
   const cudaError_t e2 = cudaFreeAsync(ws, st);
   return (e != cudaSuccess || e2 != cudaSuccess) ? SSD_ERR_CUDA : SSD_OK;
@@ -264,7 +395,7 @@ int ssd_forward_host(const ssd_shape* s, const void* x, const float* dt, const f
 
   // Whole sequences in up to kGroups groups of about equal token counts: group g's
   // inputs are copied in while group g-1 computes and group g-2's outputs go out.
-  constexpr int kGroups = 8;
+  constexpr int kGroups = kHostGroups;
   std::vector<int64_t> gs{0};
   for (int g = 1; g <= kGroups && gs.back() < nseq; ++g) {
     const int64_t target = tokens * g / kGroups;
@@ -306,16 +437,18 @@ int ssd_forward_host(const ssd_shape* s, const void* x, const float* dt, const f
       0,
   };
   void* dev[11] = {};
-  cudaStream_t sin = nullptr, sout = nullptr;
-  std::vector<cudaEvent_t> ev;
+  // the device's copy streams and events, created once; calls on one device take turns
+  HostCopies* hc = host_copies();
+  if (!hc) return SSD_ERR_CUDA;
+  std::lock_guard<std::mutex> lock(hc->mu);
+  if (!hc->ready && !hc->create()) return SSD_ERR_CUDA;
+  cudaStream_t sin = hc->sin, sout = hc->sout;
+  cudaEvent_t* ev = hc->ev;
   auto cleanup = [&]() {
-    if (sin) cudaStreamSynchronize(sin);
-    if (sout) cudaStreamSynchronize(sout);
+    cudaStreamSynchronize(sin);
+    cudaStreamSynchronize(sout);
     for (void* p : dev)
       if (p) cudaFreeAsync(p, st);
-    for (cudaEvent_t e : ev) cudaEventDestroy(e);
-    if (sin) cudaStreamDestroy(sin);
-    if (sout) cudaStreamDestroy(sout);
   };
   auto fail = [&](int code) {
     cleanup();
@@ -324,12 +457,6 @@ int ssd_forward_host(const ssd_shape* s, const void* x, const float* dt, const f
   };
   for (int i = 0; i < 10; ++i)
     if (bytes[i] && pool_alloc(&dev[i], bytes[i], st) != cudaSuccess) return fail(SSD_ERR_CUDA);
-  if (cudaStreamCreateWithFlags(&sin, cudaStreamNonBlocking) != cudaSuccess ||
-      cudaStreamCreateWithFlags(&sout, cudaStreamNonBlocking) != cudaSuccess)
-    return fail(SSD_ERR_CUDA);
-  ev.resize(2 * ng + 1, nullptr);
-  for (auto& e : ev)
-    if (cudaEventCreateWithFlags(&e, cudaEventDisableTiming) != cudaSuccess) return fail(SSD_ERR_CUDA);
   // the buffers were taken on `st`: the copy streams start after that
   if (cudaEventRecord(ev[2 * ng], st) != cudaSuccess || cudaStreamWaitEvent(sin, ev[2 * ng], 0) != cudaSuccess ||
       cudaStreamWaitEvent(sout, ev[2 * ng], 0) != cudaSuccess)
@@ -447,6 +574,13 @@ int ssd_profile_dominant(ssd_event_t start, ssd_event_t stop) {
 }
 
 uint64_t ssd_kernel_launch_count(void) { return g_launches.load(); }
+
+int ssd_set_test_hooks(int64_t wait_limit_cycles, int withhold_carry) {
+  if (wait_limit_cycles < 0) return SSD_ERR_INVALID_ARG;
+  g_wait_limit.store(wait_limit_cycles ? (long long)wait_limit_cycles : kDefaultWaitLimit);
+  g_withhold_carry.store(withhold_carry ? 1 : 0);
+  return SSD_OK;
+}
 
 int ssd_select_path(const ssd_shape* shape, int chunk) {
   const int rc = validate(shape, (const void*)16, (const float*)16, (const float*)16, (const void*)16,

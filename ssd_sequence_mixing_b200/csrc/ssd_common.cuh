@@ -44,10 +44,14 @@ struct Problem {
   float* states;       // (Cmax, H, P, N) chunk states, then chunk start states
   int Cmax;
   // tensor-core path scratch
-  int32_t* seq_tiles;  // nseq + 1: prefix over sequences of ceil(len / kTcTile)
-  float* carry;        // (ranges, 2, P, N) states handed between CTAs, then (ranges, 2) cumsums
-  int32_t* carry_flag; // (ranges) 1 once a CTA has published its carry
-  int ranges;          // CTAs of the tensor-core launch
+  int32_t* seq_tiles;    // nseq + 1: prefix over sequences of ceil(len / kTcTile) (packed batches)
+  int dense_tiles;       // tiles per sequence of a dense batch
+  float* carry;          // (ranges, 2, P, N) states handed between CTAs
+  uint64_t* carry_flag;  // (ranges, 16): `epoch` once a compute warp has published its part
+  uint64_t epoch;        // unique per launch, so flags left in reused scratch never match
+  int ranges;            // CTAs of the tensor-core launch
+  long long wait_limit;  // SM cycles a device-side wait may take before it gives up
+  int withhold_carry;    // test hook: CTAs never publish the state they hand on
   // host-side measurement hooks (events around the dominant kernel, or null)
   cudaEvent_t prof_start, prof_stop;
   // fused dt prologue (ssd_forward_dt): dt holds the raw values, see dt_value()
@@ -102,5 +106,16 @@ int check_shape(const ssd_shape* s, bool packed, int chunk);
 // Launchers implemented in the kernel files.
 cudaError_t launch_chunk_table(const Problem& pb, cudaStream_t st);
 cudaError_t launch_simt(const Problem& pb, cudaStream_t st);
+// Long sequences in segments (ssd_seqpar.cu): segment offsets of a dense batch of nseq
+// sequences of L tokens cut into k segments of `seg` tokens (the last of each shorter);
+// per-segment log-decays; every segment's start state; each sequence's final state from
+// its last segment's.
+cudaError_t launch_segment_offsets(int nseq, int64_t L, int k, int64_t seg, int32_t* cu, cudaStream_t st);
+cudaError_t launch_segments_logdecay(const int32_t* cu, int nseg, int H, const float* dt, const float* A,
+                                     float* lam, cudaStream_t st);
+cudaError_t launch_segments_prefix(int nseq, int k, int64_t H, int64_t PN, const float* states, const float* lam,
+                                   const float* init, float* out, cudaStream_t st);
+cudaError_t launch_segments_final(int nseq, int k, int64_t HPN, const float* seg_final, float* fin,
+                                  cudaStream_t st);
 
 }  // namespace ssd

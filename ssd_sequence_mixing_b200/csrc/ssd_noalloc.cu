@@ -6,8 +6,6 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
-#include <atomic>
-
 #include "ssd.h"
 #include "ssd_common.cuh"
 
@@ -19,22 +17,13 @@ namespace {
 // address looked up by scratch_base().
 static __device__ __align__(256) unsigned char g_noalloc_scratch[SSD_NOALLOC_SCRATCH_BYTES];
 
-constexpr int kMaxDevices = 64;
-std::atomic<unsigned char*> g_scratch_base[kMaxDevices];
-
-// Device address of g_noalloc_scratch on the current device; looked up on the
-// first call on each device (with that device current) and cached.
+// Device address of g_noalloc_scratch on the current device, looked up on every call
+// (with that device current), so that a context recreated after a device reset is
+// never handed an address from the old one.  The lookup allocates nothing.
 unsigned char* scratch_base() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  unsigned char* p = g_scratch_base[dev].load();
-  if (!p) {
-    void* sym = nullptr;
-    if (cudaGetSymbolAddress(&sym, g_noalloc_scratch) != cudaSuccess || !sym) return nullptr;
-    p = (unsigned char*)sym;
-    g_scratch_base[dev].store(p);
-  }
-  return p;
+  void* sym = nullptr;
+  if (cudaGetSymbolAddress(&sym, g_noalloc_scratch) != cudaSuccess || !sym) return nullptr;
+  return (unsigned char*)sym;
 }
 
 size_t up256(size_t v) { return (v + 255) & ~(size_t)255; }
@@ -48,7 +37,7 @@ extern "C" int ssd_forward_noalloc(const ssd_shape* s, const void* x, const floa
   const int rc = ssd::check_shape(s, cu != nullptr, chunk);
   if (rc) return rc;
   const int64_t tokens = s->batch * s->seqlen;
-  if (!A || !dt || (tokens > 0 && (!x || !B || !C || !y))) return SSD_ERR_INVALID_ARG;
+  if (!A || (tokens > 0 && (!x || !dt || !B || !C || !y))) return SSD_ERR_INVALID_ARG;  // as ssd_forward
   const void* ptrs[] = {x, dt, A, B, C, D, init_state, cu, y, fin};
   for (const void* p : ptrs)
     if (p && ((uintptr_t)p & 15u)) return SSD_ERR_MISALIGNED;

@@ -72,3 +72,99 @@ extern "C" int ssd_state_prefix(int rank, int64_t nheads, int64_t headdim, int64
   ssd::count_launches(1);
   return cudaGetLastError() == cudaSuccess ? SSD_OK : SSD_ERR_CUDA;
 }
+
+// ----------------------------------------------------------- long sequences in segments
+// A dense batch whose units are long enough that one unit would span several CTAs of the
+// tensor-core kernel is cut into segments (the chunked algorithm one level up): a
+// final-state-only pass from zero gives every segment's end state s, the segments' decays
+// give each segment's true start state by the same recurrence as above, and the full pass
+// runs on the segments as independent packed sequences from those states.
+namespace ssd {
+namespace {
+
+// cu[j] = first token of segment j: sequence s = j / k has segments [s L + i seg, ...),
+// the last one of each sequence ending at the sequence's end.
+__global__ void segment_offsets_kernel(int nseq, int64_t L, int k, int64_t seg, int32_t* cu) {
+  const int j = blockIdx.x * blockDim.x + threadIdx.x;
+  if (j > nseq * k) return;
+  const int s = j / k, i = j % k;
+  cu[j] = (int32_t)(s == nseq ? (int64_t)nseq * L : (int64_t)s * L + (int64_t)i * seg);
+}
+
+// lam[j][h] = A[h] * sum of dt over segment j; grid (ceil(H / 32), nseg).
+__global__ void __launch_bounds__(kHeadsPerBlock * kTokLanes)
+    segments_logdecay_kernel(const int32_t* cu, int H, const float* dt, const float* A, float* lam) {
+  __shared__ float part[kTokLanes][kHeadsPerBlock];
+  const int hl = threadIdx.x % kHeadsPerBlock, tl = threadIdx.x / kHeadsPerBlock;
+  const int h = blockIdx.x * kHeadsPerBlock + hl, j = blockIdx.y;
+  float acc = 0.f;
+  if (h < H)
+    for (int64_t t = cu[j] + tl; t < cu[j + 1]; t += kTokLanes) acc += dt[t * H + h];
+  part[tl][hl] = acc;
+  __syncthreads();
+  if (tl == 0 && h < H) {
+    float s = 0.f;
+#pragma unroll
+    for (int q = 0; q < kTokLanes; ++q) s += part[q][hl];
+    lam[(int64_t)j * H + h] = s * A[h];
+  }
+}
+
+// Start state of every segment: for each sequence s (k segments) and state element e,
+// h[s k] = init[s], h[s k + i + 1] = exp(lam[s k + i]) h[s k + i] + states[s k + i].
+__global__ void __launch_bounds__(256) segments_prefix_kernel(int nseq, int k, int64_t H, int64_t PN,
+                                                              const float* states, const float* lam,
+                                                              const float* init, float* out) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int s = blockIdx.y;
+  if (e >= H * PN) return;
+  const int64_t h = e / PN;
+  float acc = init ? init[(int64_t)s * H * PN + e] : 0.f;
+  for (int i = 0; i < k; ++i) {
+    const int64_t j = (int64_t)s * k + i;
+    out[j * H * PN + e] = acc;
+    acc = fmaf(expf(lam[j * H + h]), acc, states[j * H * PN + e]);
+  }
+}
+
+// final[s] = the final state of sequence s's last segment.
+__global__ void __launch_bounds__(256) segments_final_kernel(int k, int64_t HPN, const float* seg_final,
+                                                             float* fin) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  const int s = blockIdx.y;
+  if (e < HPN) fin[(int64_t)s * HPN + e] = seg_final[((int64_t)s * k + k - 1) * HPN + e];
+}
+
+}  // namespace
+
+cudaError_t launch_segment_offsets(int nseq, int64_t L, int k, int64_t seg, int32_t* cu, cudaStream_t st) {
+  const int n = nseq * k + 1;
+  segment_offsets_kernel<<<(n + 255) / 256, 256, 0, st>>>(nseq, L, k, seg, cu);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_segments_logdecay(const int32_t* cu, int nseg, int H, const float* dt, const float* A,
+                                     float* lam, cudaStream_t st) {
+  segments_logdecay_kernel<<<dim3((H + kHeadsPerBlock - 1) / kHeadsPerBlock, nseg), kHeadsPerBlock * kTokLanes, 0,
+                             st>>>(cu, H, dt, A, lam);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_segments_prefix(int nseq, int k, int64_t H, int64_t PN, const float* states, const float* lam,
+                                   const float* init, float* out, cudaStream_t st) {
+  segments_prefix_kernel<<<dim3((unsigned)((H * PN + 255) / 256), nseq), 256, 0, st>>>(nseq, k, H, PN, states,
+                                                                                       lam, init, out);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_segments_final(int nseq, int k, int64_t HPN, const float* seg_final, float* fin,
+                                  cudaStream_t st) {
+  segments_final_kernel<<<dim3((unsigned)((HPN + 255) / 256), nseq), 256, 0, st>>>(k, HPN, seg_final, fin);
+  count_launches(1);
+  return cudaGetLastError();
+}
+
+}  // namespace ssd

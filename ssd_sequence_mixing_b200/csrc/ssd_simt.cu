@@ -393,7 +393,7 @@ static cudaError_t launch_simt_t(const Problem& pb, cudaStream_t st) {
   const int64_t PN = (int64_t)pb.P * pb.N;
   state_passing_kernel<<<dim3(pb.nseq, pb.H, (unsigned)((PN + 255) / 256)), 256, 0, st>>>(pb);
   ++n;
-  if (pb.Cmax > 0) {
+  if (pb.Cmax > 0 && pb.y) {  // y == null: only the final states are wanted
     if (pb.prof_start) cudaEventRecord(pb.prof_start, st);
     chunk_output_kernel<T><<<dim3(pb.Cmax * (pb.Q / 64), pb.H, (pb.P + 63) / 64), 256, 0, st>>>(pb);
     if (pb.prof_stop) cudaEventRecord(pb.prof_stop, st);

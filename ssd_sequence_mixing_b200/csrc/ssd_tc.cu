@@ -5,26 +5,39 @@
 // (the tcgen05 M) of all units (sequence, pair of heads sharing a B/C group), handing
 // the state on through global memory where its share starts or ends inside a unit.
 // The P x N state of each head never leaves the chip: it stays in fp32 in tensor
-// memory, with a bf16 copy in shared memory as an MMA operand.  Per tile:
+// memory, with a bf16 copy in shared memory as an MMA operand.
 //
-//   cumsum   cs_j = running in-chunk cumsum of dt_j A_h in log2 units (restarted at
-//            each chunk start, so a 256-token chunk spans two tiles)   [helper warps]
-//   MMA  S   = C B^T                                   (128 x 128, K = N, once per pair)
-//   MMA  Yo  = C [h0 h1]^T        left factor           (128 x 128, K = N)
-//   MMA  h^T += B^T [w0 o x0 | w1 o x1]   right factor  (N x 128, K = 128),
-//            w_j = exp(cs_end - cs_j) dt_j, onto the decay-scaled state
-//   mask     P_ij = S_ij exp(cs_i - cs_j) dt_j for j <= i, else 0 (mask before exp),
-//            written as bf16 pairs to tensor memory
-//   scale    Y_i = exp(cs_i - cs_start) Yo_i
-//   MMA  Y  += P_h x_h            diagonal block, A from tensor memory  (128 x 64, K = 128)
-//   state    h <- exp(cs_end' - cs_start') h for the next tile (centre factor), its bf16
-//            copy, or the final state / hand-on at the end of a piece
-//   epilogue y_i = Y_i + D x_i    (bf16, staged over the x tile, TMA store)
+// Decay factorisation.  Inside a tile, with c_i the inclusive cumsum of dt A (log2 units,
+// restarted at the tile start) of one head, the diagonal block needs the factor
+// 2^(c_i - c_j) for j <= i.  Around a reference m (per tile and head) it splits into a
+// row factor r_i = 2^(c_i - m) and a column factor 2^(m - c_j).  The column factor (with
+// dt_j) goes onto x:  U_j = 2^(m - c_j) dt_j x_j, and the row factor into the epilogue.
+// What is left of the masked matrix, P = causal(C B^T), no longer depends on the head:
+// it is computed once per pair, without exponentials, and both heads' diagonal blocks
+// are one N = 128 product P [U_0 | U_1].  The same U feeds the chunk state, and the
+// carried-in state enters scaled as h^ = 2^(m - c_start) h, so that one accumulator
+// holds everything a row needs before its factor r_i:
 //
-// Roles: 16 compute warps (per head, two column halves x four lane quarters), one
-// issuer warp (every TMA load of x, B, C and every tcgen05.mma) and two helper warps
-// (dt loads and the per-tile descriptors: cumsums, column factors, decays, flags).
-// Tensor memory: S 128 columns, P 2 x 64, Y 2 x 64, h^T 2 x 64.
+//   MMA  S   = C B^T                               (128 x 128, K = N, once per pair)
+//   mask     P = bf16(S) on and below the diagonal, 0 above (mask before use)
+//   MMA  Y   = C [h^_0 h^_1]^T     left factor     (128 x 128, K = N)
+//   MMA  H  += B^T [U_0 | U_1]     right factor    (N x 128, K = 128), H holds h^
+//   MMA  Y  += P [U_0 | U_1]       diagonal block  (128 x 128, K = 128, A in tensor memory)
+//   state    h_end = 2^(c_end - m) H  (centre factor: the next tile's h^ is this times
+//            2^(m' - c'_start)), or the final state / hand-on at the end of a piece
+//   epilogue y_i = r_i Y_i + D x_i  (bf16, staged over the tile's U, TMA store)
+//
+// The split needs 2^(m - c_j) and 2^(c_i - m) to stay well inside the fp32 / bf16
+// range: a tile whose decay range over its rows exceeds kRangeMax (log2 units) is
+// processed in several passes over the same loaded data, each over a run of rows
+// whose range fits (on the pages' input distributions, 1 - 3 % of tiles).
+//
+// Roles: 16 compute warps (Û, the mask, the state step, the epilogue), one MMA warp
+// (every tcgen05.mma), one load warp (every TMA load of x, B, C) and one helper warp
+// (dt loads, the per-pass descriptors: passes, references, row factors, flags).
+// Tensor memory: two S/P buffers of 128 columns (P is written in place over S),
+// Y 128, H 128.  Shared memory: x (two stages; U and then y are written in place),
+// a ring of three B/C tiles, the bf16 state, the descriptors and the dt stages.
 // Every wait is bounded; a wait that gives up records SSD_ERR_DEVICE_TIMEOUT in the
 // status word, drains what is in flight (bounded), frees tensor memory and exits.
 #include <cuda.h>
@@ -32,40 +45,10 @@
 #include <stdio.h>
 #include <stdlib.h>
 
+#include <atomic>
+
 #include "sm100_ptx.cuh"
 #include "ssd_tc.cuh"
-
-#ifndef SSD_TRACE
-#define SSD_TRACE 0  // 1: record per-phase clock64 stamps of the first CTAs (profiling builds only)
-#endif
-#if SSD_TRACE
-namespace ssd {
-constexpr int kTraceCtas = 4, kTraceTiles = 64, kTraceMarks = 24;
-__device__ unsigned long long g_trace[3 * kTraceCtas * kTraceTiles * kTraceMarks];
-}  // namespace ssd
-extern "C" int ssd_trace_dump(unsigned long long* host, int n) {
-  return (int)cudaMemcpyFromSymbol(host, ssd::g_trace, sizeof(unsigned long long) * n);
-}
-#define TRACE_MARK(m)                                                                              \
-  do {                                                                                             \
-    if ((tid == 0 || tid == 96) && blockIdx.x < kTraceCtas && trace_tile < kTraceTiles)            \
-      g_trace[(((tid != 0) * kTraceCtas + blockIdx.x) * kTraceTiles + trace_tile) * kTraceMarks +  \
-              (m)] = clock64();                                                                    \
-  } while (0)
-#define TRACE_ISSUE(m)                                                                             \
-  do {                                                                                             \
-    if (blockIdx.x < kTraceCtas && t < kTraceTiles)                                                \
-      g_trace[((2 * kTraceCtas + blockIdx.x) * kTraceTiles + t) * kTraceMarks + (m)] = clock64();  \
-  } while (0)
-#else
-#define TRACE_ISSUE(m) \
-  do {                 \
-  } while (0)
-#define TRACE_MARK(m) \
-  do {                \
-  } while (0)
-#endif
-
 
 namespace ssd {
 
@@ -75,92 +58,85 @@ using namespace sm100;
 
 constexpr int kTile = 128;          // tokens per tile (UMMA M)
 constexpr int kHeadDim = 64;        // P supported by this path
-constexpr int kWGThreads = 128;     // a warpgroup: thread i <-> TMEM lane i
 constexpr int kHeads = 2;           // heads of one B/C group processed together
-constexpr int kHalves = 2;          // each head's Y and state columns split over two warpgroups
-constexpr int kComputeThreads = kHeads * kHalves * kWGThreads;
-constexpr int kComputeWarps = kComputeThreads / 32;
-constexpr int kHelperWarps = kHeads;  // one helper warp per head of the pair
-constexpr int kThreads = kComputeThreads + 32 + 32 * kHelperWarps;  // + the issuer warp (TMA and UMMA), helpers
-constexpr int kIssuerWarp = kComputeWarps, kHelperWarp = kComputeWarps + 1;
-constexpr int kDescSlots = 2;  // tile descriptors the helper warp may run ahead
+constexpr int kComputeWarps = 16;   // (head, column half, lane quarter)
+constexpr int kMmaWarp = kComputeWarps, kLoadWarp = kComputeWarps + 1, kHelperWarp = kComputeWarps + 2;
+constexpr int kThreads = (kComputeWarps + 3) * 32;
+constexpr int kDescSlots = 3;  // pass descriptors the helper may run ahead
 constexpr int kDtStages = 4;   // dt tiles in flight
+constexpr int kRing = 3;       // B / C tiles in shared memory (C(t), B(t) and the next one)
 constexpr uint32_t kTmemCols = 512;
-// TMEM columns: S = C B^T (fp32, 128), P_h (bf16 pairs, 64 per head), Y_h (64 per head;
-// the left factor is written first, row-scaled, then P_h x_h accumulates on top) and
-// the fp32 state h^T of each head (64 per head): every tile it is scaled by the tile's
-// decay in place and the right-factor MMA accumulates B^T (w o x) onto it.
-constexpr uint32_t kColS = 0, kColP = 128, kColY = 256, kColSt = 384;
-constexpr long long kWaitLimit = 4ll << 30;  // SM cycles (about 2 s) before a wait gives up
-constexpr uint32_t kAtom = kTile * 128;      // one 128-row x 128-byte swizzled operand column
+// TMEM columns: two S/P buffers (S fp32, then P as bf16 pairs in the first 16 columns
+// of each 32-column block), Y (64 per head) and the fp32 state H = h^T (64 per head).
+constexpr uint32_t kColSP = 0, kColY = 256, kColH = 384;
+constexpr float kRangeMax = 200.f;            // log2 units of decay one pass may span
+constexpr uint32_t kAtom = kTile * 128;       // one 128-row x 128-byte swizzled operand column
 
-// mbarriers.  Issuer -> compute: tile loads (tx bytes) and UMMA commits.
-// Compute -> issuer (one arrival per compute warp): ht, xw, p, free, x-free.
-// Helper -> compute: a tile descriptor is written; compute -> helper: it was used up.
+// mbarriers (index = bit of the 64-bit phase masks)
 enum {
-  kBarLoad0 = 0,  // x, B, C of a tile in x stage 0
-  kBarLoad1,      // ... stage 1
-  kBarS,          // S = C B^T done
-  kBarYo,         // left factor C h^T written into Y
-  kBarSt,         // right factor accumulated onto the state
-  kBarY,          // P x accumulated into Y
-  kBarHt,         // bf16 state for the next tile written
-  kBarXw,         // w o x written and the state scaled by this tile's decay
-  kBarP,          // P written and Y rows scaled
-  kBarFree,       // Y read (the next left factor may overwrite it)
-  kBarXfree,      // a stage's x buffer (which held that tile's y for the TMA stores) is reusable
-  kBarDt0,        // kHelperWarps x kDtStages barriers: dt of a tile (4 heads x 128 tokens) in a helper's stage
-  kBarDescFull0 = kBarDt0 + kHelperWarps * kDtStages,  // kDescSlots barriers: descriptor written (both helpers)
-  kBarDescFree0 = kBarDescFull0 + kDescSlots,  // kDescSlots barriers: descriptor used up
-  kBarPair0 = kBarDescFree0 + kDescSlots,  // 8 barriers: the column-half-1 warp of a row quarter staged its y
+  kBarX0 = 0,                         // 2: x of a tile in stage s (tx bytes)
+  kBarXfree0 = kBarX0 + 2,            // 2: stage s free again (16 compute arrivals)
+  kBarRing0 = kBarXfree0 + 2,         // kRing: B or C tile in a ring slot (tx bytes)
+  kBarRingFree0 = kBarRing0 + kRing,  // kRing: ring slot free (one UMMA commit)
+  kBarS0 = kBarRingFree0 + kRing,     // 2: S = C B^T in S/P buffer b (commit)
+  kBarP0 = kBarS0 + 2,                // 2: P written in buffer b (16 arrivals)
+  kBarSt,                             // right factor accumulated onto H (commit)
+  kBarY,                              // P U accumulated into Y (commit)
+  kBarU,                              // U written (16)
+  kBarHt,                             // h^ written, bf16 in shared and fp32 in H (16)
+  kBarFree,                           // Y read by the epilogue (16)
+  kBarDrain,                          // the MMA warp's last commit after an abort
+  kBarDt0,                            // kDtStages: dt of a tile (4 heads x 128 tokens)
+  kBarDescFull0 = kBarDt0 + kDtStages,           // kDescSlots: descriptor written (helper)
+  kBarDescFree0 = kBarDescFull0 + kDescSlots,    // kDescSlots: used up (16 compute + MMA)
+  kBarPair0 = kBarDescFree0 + kDescSlots,        // 8: column-half-1 warp of (head, quarter) staged its y
   kNumBars = kBarPair0 + kHeads * 4
 };
+static_assert(kNumBars <= 64, "phase bits of a 64-bit mask");
 
-// One tile as the helper warp lays it out for the compute warps: where it is, what to do
-// with the state around it, and per head the in-chunk cumsum of dt A (log2 units), the
-// 32-block column factors exp(cs(block end) - cs_j) dt_j, and dt.
+// Pass descriptor flags
 enum {
-  kDescFirst = 1,    // first tile of a piece: load the state (initial or handed on) before it
-  kDescCarryIn = 2,  // ... from the carry of CTA carry_src
-  kDescToFinal = 4,  // last tile of a unit: the state after it is the final state
-  kDescToCarry = 8,  // last tile of a range that ends inside a unit: hand the state on
-  kDescEnd = 16      // no tile: the range is done
+  kPFirst = 1,       // first pass of a tile: S / P, x into registers
+  kPLast = 2,        // last pass of a tile: its B / C / x may be released
+  kPPieceStart = 4,  // the state before this pass is the piece's initial state ...
+  kPCarryIn = 8,     // ... handed on by CTA carry_src
+  kPToFinal = 16,    // the state after this pass is the unit's final state
+  kPToCarry = 32,    // ... is handed on to the next CTA
+  kPEnd = 64         // no pass: the range is done
 };
-struct TileDesc {
-  int t0;         // token index of row 0
+struct PassDesc {
+  int t0;         // token index of row 0 of the tile
   int rem;        // rows of the tile inside the sequence (1..128)
+  int lo, hi;     // rows of this pass
   int s;          // sequence
   int h0;         // first head of the pair
   int flags;
   int carry_src;
-  int pad[2];
-  float cs_start[kHeads];  // cumsum before row 0
-  float cs_end[kHeads];    // cumsum after the last row (rows past the end add 0)
-  float decay[kHeads];     // exp2(cs_end - cs_start)
-  float dskip[kHeads];     // D
-  float cs[kHeads][kTile];
-  float cc[kHeads][kTile];
-  float dtv[kHeads][kTile];  // 0 past the end of the sequence
+  float sig_in[kHeads];   // h^ = sig_in h_in: 2^(m - c_before(lo))
+  float sig_out[kHeads];  // h_out = sig_out H: 2^(c(hi - 1) - m)
+  float dskip[kHeads];    // D
+  float pad[2];
+  float u[kHeads][kTile];  // 2^(m - c_j) dt_j on the pass's rows, else 0
+  float r[kHeads][kTile];  // 2^(c_i - m) on the pass's rows, else 0
 };
-constexpr uint32_t kDescBytes = (sizeof(TileDesc) + 127) / 128 * 128;
+constexpr uint32_t kDescBytes = (sizeof(PassDesc) + 127) / 128 * 128;
 
 template <int NS>
 struct Layout {
-  static constexpr uint32_t x = 0;                          // [stage][head] [128 tok][64 p]
-  static constexpr uint32_t b = x + 2 * kHeads * kAtom;     // NS/64 atoms [128 tok][64 n]
-  static constexpr uint32_t c = b + (NS / 64) * kAtom;
-  static constexpr uint32_t xw = c + (NS / 64) * kAtom;     // [head] [128 tok][64 p]
-  static constexpr uint32_t ht = xw + kHeads * kAtom;       // [head] [NS n][64 p]
-  static constexpr uint32_t desc = ht + kHeads * NS * 128;           // TileDesc[kDescSlots]
-  static constexpr uint32_t sdt = desc + kDescSlots * kDescBytes;    // float[helper][stage][128 tok][4 heads]
-  static constexpr uint32_t bars = sdt + kHelperWarps * kDtStages * kTile * 16;  // uint64[kNumBars]
-  static constexpr uint32_t flag = bars + kNumBars * 8;     // int: a wait gave up
+  static constexpr uint32_t kSlot = (NS / 64) * kAtom;             // one B or C tile
+  static constexpr uint32_t x = 0;                                 // [stage][head] [128 tok][64 p]
+  static constexpr uint32_t ring = x + 2 * kHeads * kAtom;         // kRing slots [NS/64 atoms][128 tok][64 n]
+  static constexpr uint32_t ht = ring + kRing * kSlot;             // [head] [NS n][64 p]
+  static constexpr uint32_t desc = ht + kHeads * NS * 128;         // PassDesc[kDescSlots]
+  static constexpr uint32_t scan = desc + kDescSlots * kDescBytes; // helper: c[2][128]
+  static constexpr uint32_t sdt = scan + kHeads * kTile * 4;       // float[stage][128 tok][4 heads]
+  static constexpr uint32_t bars = sdt + kDtStages * kTile * 16;   // uint64[kNumBars]
+  static constexpr uint32_t flag = bars + kNumBars * 8;            // int: a wait gave up
   static constexpr uint32_t bytes = flag + 16;
 };
 template <int NS>
 constexpr uint32_t kDynSmem = Layout<NS>::bytes + 1024;  // + base alignment slack
 static_assert(kDynSmem<128> <= 227 * 1024, "shared memory per CTA");
-static_assert(kNumBars <= 32, "phase bits of a 32-bit mask");
 
 // Work split.  The tiles of all units (sequence, head pair), unit by unit and each
 // unit's 128-token tiles in order, form one flat list; CTA r takes the contiguous
@@ -168,7 +144,7 @@ static_assert(kNumBars <= 32, "phase bits of a 32-bit mask");
 // state the previous CTA reached there: "carry in") and end inside one (it then hands
 // its state on: "carry out").  A CTA processes its last, truncated piece first, so the
 // state it hands on is ready early; then the whole units; then the piece that needs a
-// carry.  Issuer and compute threads walk the same sequence.
+// carry.  The load, helper and compute roles walk the same sequence.
 struct TileCursor {
   int unit, k0, len;  // k0: token offset of the tile in the sequence
   int tb;             // first token of the sequence (tokens < 2^31 on this path)
@@ -183,20 +159,28 @@ struct RangePlan {
   int carry_src;                 // the CTA whose range holds the tile before this range's first
 };
 
+// First tile of sequence s in the per-sequence tile prefix (dense batches: every
+// sequence has dense_tiles tiles; packed ones: the table kernel's prefix).
+__device__ __forceinline__ int64_t seq_tile0(const Problem& pb, int s) {
+  return pb.cu ? (int64_t)pb.seq_tiles[s] : (int64_t)s * pb.dense_tiles;
+}
+
 __device__ __forceinline__ int unit_tiles(const Problem& pb, int u) {
   const int s = u / (pb.H / kHeads);
-  return pb.seq_tiles[s + 1] - pb.seq_tiles[s];
+  return (int)(seq_tile0(pb, s + 1) - seq_tile0(pb, s));
 }
 
 __device__ __forceinline__ int64_t unit_first_tile(const Problem& pb, int u) {
   const int pairs = pb.H / kHeads;
   const int s = u / pairs;
-  return (int64_t)pb.seq_tiles[s] * pairs + (int64_t)(u % pairs) * (pb.seq_tiles[s + 1] - pb.seq_tiles[s]);
+  const int64_t a = seq_tile0(pb, s), b = seq_tile0(pb, s + 1);
+  return a * pairs + (int64_t)(u % pairs) * (b - a);
 }
 
 // The unit holding flat tile w (0 <= w < W).
 __device__ __forceinline__ int unit_of_tile(const Problem& pb, int64_t w) {
   const int pairs = pb.H / kHeads;
+  if (!pb.cu) return (int)(w / pb.dense_tiles);
   int lo = 0, hi = pb.nseq;  // seq_tiles[lo] * pairs <= w < seq_tiles[hi] * pairs
   while (hi - lo > 1) {
     const int mid = (lo + hi) >> 1;
@@ -211,7 +195,7 @@ __device__ __forceinline__ int unit_of_tile(const Problem& pb, int64_t w) {
 
 __device__ __forceinline__ RangePlan plan_range(const Problem& pb) {
   RangePlan rp{};
-  const int64_t W = (int64_t)pb.seq_tiles[pb.nseq] * (pb.H / kHeads);
+  const int64_t W = seq_tile0(pb, pb.nseq) * (pb.H / kHeads);
   const int64_t w0 = W * blockIdx.x / gridDim.x, w1 = W * (blockIdx.x + 1) / gridDim.x;
   if (w0 >= w1) return rp;
   rp.u0 = unit_of_tile(pb, w0);
@@ -276,13 +260,15 @@ __device__ __forceinline__ void warp_arrive(uint64_t* bar) {
   __syncwarp();
 }
 
-// Bounded wait that also gives up when another thread has recorded a failure.
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag) {
+// Bounded wait (at most `limit` SM cycles) that also gives up when another thread has
+// recorded a failure.
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                              long long limit) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (*abort_flag) return false;
-    if (clock64() - t0 > kWaitLimit) {
+    if (clock64() - t0 > limit) {
       *abort_flag = 1;
       return false;
     }
@@ -290,201 +276,247 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
   return true;
 }
 
-// ------------------------------------------------------------------ issuer
+// Phase bookkeeping of one thread (or one warp, waiting uniformly) over all barriers.
+struct Phases {
+  uint64_t bits = 0;  // bit k: parity of the next phase of bars[k] to wait for
+  __device__ __forceinline__ uint32_t parity(int k) const { return (uint32_t)(bits >> k) & 1u; }
+  __device__ __forceinline__ void flip(int k) { bits ^= 1ull << k; }
+};
+
+// ------------------------------------------------------------------ load warp
 template <int NS>
-__device__ void issuer_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, const CUtensorMap* tm_c,
-                            const Problem& pb, uint8_t* smem, uint32_t tmem, uint64_t* bars,
-                            volatile int* abort_flag) {
+__device__ void load_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, const CUtensorMap* tm_c,
+                          const Problem& pb, uint8_t* smem, uint64_t* bars, volatile int* abort_flag) {
   using L = Layout<NS>;
-  uint8_t* sx = smem + L::x;
-  uint8_t* sb = smem + L::b;
-  uint8_t* sc = smem + L::c;
-  constexpr uint32_t kLoadBytes = kHeads * kAtom + 2u * (NS / 64) * kAtom;
-  const uint32_t id_s = idesc_bf16(128, 128, 0, 0);
-  const uint32_t id_y = idesc_bf16(128, 64, 0, 1);
-  const uint32_t id_yo = idesc_bf16(128, 128, 0, 1);
-  const uint32_t id_st = idesc_bf16(128, 128, 1, 1);
-  const uint32_t a_sb = smem_u32(sb), a_sc = smem_u32(sc);
-  const uint32_t a_sxw = smem_u32(smem + L::xw), a_sht = smem_u32(smem + L::ht);
-  // For N = 64 the B^T operand has one M atom; the second (unused) half of s^T reads
-  // the C tile that follows it, and those lanes are ignored.
-  const uint32_t lbo_bt = kAtom;
-  const int pairs = pb.H / kHeads;
-
-  auto issue_x = [&](int stage, const TileCursor& c) {
-    const int h0 = (c.unit % pairs) * kHeads;
-#pragma unroll
-    for (int hh = 0; hh < kHeads; ++hh)
-      tma_load_3d(sx + (stage * kHeads + hh) * kAtom, tm_x, 0, h0 + hh, c.tb + c.k0, &bars[stage]);
-  };
-  auto issue_bc = [&](int stage, const TileCursor& c) {
-    const int g = ((c.unit % pairs) * kHeads) / pb.hpg;
-#pragma unroll
-    for (int a = 0; a < NS / 64; ++a) {
-      tma_load_3d(sb + a * kAtom, tm_b, a * 64, g, c.tb + c.k0, &bars[stage]);
-      tma_load_3d(sc + a * kAtom, tm_c, a * 64, g, c.tb + c.k0, &bars[stage]);
-    }
-  };
-
-  uint32_t phase = 0;    // bit k: parity of the next phase of bars[k] this thread waits for
-  uint32_t pending = 0;  // bit k: async work on bars[k] issued and not waited for
+  Phases ph;
   auto wait = [&](int k) -> bool {
-    if (!wait_or_abort(&bars[k], (phase >> k) & 1u, abort_flag)) return false;
-    phase ^= 1u << k;
-    pending &= ~(1u << k);
+    if (!wait_or_abort(&bars[k], ph.parity(k), abort_flag, pb.wait_limit)) return false;
+    ph.flip(k);
     return true;
   };
-
   const RangePlan rp = plan_range(pb);
+  const int pairs = pb.H / kHeads;
   TileCursor cur;
   bool have = cursor_first(pb, rp, cur);
-  int stage = 0, t = 0;
-  if (have) {
-    mbar_expect_tx(&bars[kBarLoad0], kLoadBytes);
-    issue_x(0, cur);
-    issue_bc(0, cur);
-    pending |= 1u << kBarLoad0;
-  }
+  uint32_t nring = 0;  // ring loads issued
+  int t = 0;
   bool ok = true;
+  // last issued load per barrier (parity of its phase), for the drain after an abort
+  uint64_t issued = 0, issued_par = 0;
+  auto note = [&](int k, uint32_t par) {
+    issued |= 1ull << k;
+    issued_par = (issued_par & ~(1ull << k)) | ((uint64_t)par << k);
+  };
+  auto ring_load = [&](const CUtensorMap* tm, int g, int tok) -> bool {
+    const int slot = nring % kRing;
+    if (nring >= (uint32_t)kRing && !wait(kBarRingFree0 + slot)) return false;
+    uint8_t* dst = smem + L::ring + slot * L::kSlot;
+    mbar_expect_tx(&bars[kBarRing0 + slot], L::kSlot);
+#pragma unroll
+    for (int a = 0; a < NS / 64; ++a) tma_load_3d(dst + a * kAtom, tm, a * 64, g, tok, &bars[kBarRing0 + slot]);
+    note(kBarRing0 + slot, (nring / kRing) & 1u);
+    ++nring;
+    return true;
+  };
+  const bool state_only = pb.y == nullptr;  // no y: C is not needed
   while (have) {
-    TileCursor nxt = cur;
-    const bool have_next = cursor_next(pb, rp, nxt);
-    TRACE_ISSUE(0);
-    // S = C B^T once this tile's x, B, C are in (the previous mask finished with S).
-    if (!(ok = wait(stage))) break;
-    TRACE_ISSUE(1);
-    tc_fence_after();
+    const int h0 = (cur.unit % pairs) * kHeads, g = h0 / pb.hpg, tok = cur.tb + cur.k0;
+    // C(t) goes into the slot B(t-2) held, x(t) into stage t & 1 once tile t-2's y is
+    // out of it, B(t) into the slot C(t-1) held (free once the left factor of t-1 is done)
+    if (!state_only && !(ok = ring_load(tm_c, g, tok))) break;
+    const int st = t & 1;
+    if (t >= 2 && !(ok = wait(kBarXfree0 + st))) break;
+    mbar_expect_tx(&bars[kBarX0 + st], kHeads * kAtom);
 #pragma unroll
-    for (int kk = 0; kk < NS / 16; ++kk) {
-      const uint32_t koff = (kk >> 2) * kAtom + (kk & 3) * 32;
-      umma_f16(tmem + kColS, sdesc_sw128(a_sc + koff, 16, 1024), sdesc_sw128(a_sb + koff, 16, 1024), id_s, kk > 0);
-    }
-    umma_commit(&bars[kBarS]);
-    pending |= 1u << kBarS;
-    // Left factor C h^T into Y: needs the bf16 state and the previous epilogue done with Y.
-    if (!(ok = wait(kBarHt))) break;
-    TRACE_ISSUE(2);
-    if (t > 0 && !(ok = wait(kBarFree))) break;
-    TRACE_ISSUE(3);
-    tc_fence_after();
-#pragma unroll
-    for (int kk = 0; kk < NS / 16; ++kk) {
-      const uint32_t koff = (kk >> 2) * kAtom + (kk & 3) * 32;
-      umma_f16(tmem + kColY, sdesc_sw128(a_sc + koff, 16, 1024), sdesc_sw128(a_sht + kk * 2048, NS * 128, 1024),
-               id_yo, kk > 0);
-    }
-    umma_commit(&bars[kBarYo]);
-    pending |= 1u << kBarYo;
-    if (have_next) {  // the other x stage (tile t-1's x, then its y) is free once its y store read it
-      if (t > 0 && !(ok = wait(kBarXfree))) break;
-      TRACE_ISSUE(4);
-      fence_proxy_async();
-      mbar_expect_tx(&bars[stage ^ 1], kLoadBytes);
-      issue_x(stage ^ 1, nxt);
-      pending |= 1u << (stage ^ 1);
-    }
-    // Right factor onto the (decay-scaled) state: h^T += B^T [w0 x0 | w1 x1].
-    if (!(ok = wait(kBarXw))) break;
-    TRACE_ISSUE(5);
-    tc_fence_after();
-#pragma unroll
-    for (int kk = 0; kk < kTile / 16; ++kk)
-      umma_f16(tmem + kColSt, sdesc_sw128(a_sb + kk * 2048, lbo_bt, 1024),
-               sdesc_sw128(a_sxw + kk * 2048, kAtom, 1024), id_st, 1);
-    umma_commit(&bars[kBarSt]);
-    pending |= 1u << kBarSt;
-    // B and C are free once S and both factors are done: next tile's, issued now so that
-    // the load runs under this tile's masked product and epilogue.
-    if (have_next) {
-      if (!(ok = wait(kBarS)) || !(ok = wait(kBarYo)) || !(ok = wait(kBarSt))) break;
-      TRACE_ISSUE(6);
-      fence_proxy_async();
-      issue_bc(stage ^ 1, nxt);
-    }
-    // Y_h += P_h x_h (A from tensor memory).
-    if (!(ok = wait(kBarP))) break;
-    TRACE_ISSUE(7);
-    tc_fence_after();
-    {
-      const uint32_t a_sx = smem_u32(sx + stage * kHeads * kAtom);
-#pragma unroll
-      for (int hh = 0; hh < kHeads; ++hh) {
-#pragma unroll
-        for (int kk = 0; kk < kTile / 16; ++kk)
-          umma_f16_ta(tmem + kColY + hh * 64, tmem + kColP + hh * 64 + kk * 8,
-                      sdesc_sw128(a_sx + hh * kAtom + kk * 2048, kAtom, 1024), id_y, 1);
-      }
-    }
-    umma_commit(&bars[kBarY]);
-    pending |= 1u << kBarY;
-    cur = nxt;
-    have = have_next;
-    stage ^= 1;
+    for (int hh = 0; hh < kHeads; ++hh)
+      tma_load_3d(smem + L::x + (st * kHeads + hh) * kAtom, tm_x, 0, h0 + hh, tok, &bars[kBarX0 + st]);
+    note(kBarX0 + st, (uint32_t)(t >> 1) & 1u);
+    if (!(ok = ring_load(tm_b, g, tok))) break;
     ++t;
+    have = cursor_next(pb, rp, cur);
   }
   if (!ok) {
     *abort_flag = 1;
-    // Drain what this thread issued (again bounded) before tensor memory is freed.
+    // loads still in flight land before the CTA ends (bounded)
     for (int k = 0; k < kNumBars; ++k)
-      if (pending & (1u << k)) mbar_wait_bounded(&bars[k], (phase >> k) & 1u, kWaitLimit);
+      if (issued & (1ull << k)) mbar_wait_bounded(&bars[k], (uint32_t)(issued_par >> k) & 1u, pb.wait_limit);
   }
 }
 
-// --------------------------------------------------------- compute warpgroups
-// Four warpgroups: two per head of the pair, one per 32-column half of that head's Y and
-// state columns in tensor memory.  Warp (head hw, half ch, quarter wq) owns TMEM lanes /
-// tile rows 32 wq .. 32 wq + 31 and columns 32 ch .. 32 ch + 31 of its head's Y and state;
-// of the masked product it computes the 32-column blocks ch and ch + 2.  What is the same
-// for every row of a tile (where it is, the cumsums and column factors) comes from the
-// helper warp's tile descriptor.  The two halves of a row quarter meet once a tile, on a
-// one-arrival barrier, before the half-0 warp stores their 32 rows of y by TMA.  Every
-// wait is warp-uniform and bounded.
+// ------------------------------------------------------------------ MMA warp
+template <int NS>
+__device__ void mma_loop(const Problem& pb, uint8_t* smem, uint32_t tmem, uint64_t* bars,
+                         volatile int* abort_flag) {
+  using L = Layout<NS>;
+  const uint32_t id_s = idesc_bf16(128, 128, 0, 0);   // C (K-major) x B (K-major)
+  const uint32_t id_y = idesc_bf16(128, 128, 0, 1);   // C or P x (N-major h^ / U)
+  const uint32_t id_h = idesc_bf16(128, 128, 1, 1);   // B^T (M-major) x U (N-major)
+  const uint32_t a_ht = smem_u32(smem + L::ht);
+  const PassDesc* descs = reinterpret_cast<const PassDesc*>(smem + L::desc);
+  // For N = 64 the B^T operand has one M atom; the second (unused) half of H^T reads
+  // the next ring slot or the state copy after it, and those lanes are never read.
+  Phases ph;
+  auto wait = [&](int k) -> bool {
+    if (!wait_or_abort(&bars[k], ph.parity(k), abort_flag, pb.wait_limit)) return false;
+    ph.flip(k);
+    return true;
+  };
+  const bool state_only = pb.y == nullptr;  // only the right factor: no S, P, Y
+  bool ok = true, issued_any = false;
+  int t = -1;
+  uint32_t a_c = 0, a_b = 0, a_x = 0, c_slot = 0, b_slot = 0;
+  for (int p = 0;; ++p) {
+    const int ds = p % kDescSlots;
+    if (!(ok = wait(kBarDescFull0 + ds))) break;
+    const PassDesc& d = descs[ds];
+    const int flags = d.flags;
+    if (flags & kPEnd) break;
+    if ((flags & kPFirst) && state_only) {
+      ++t;
+      b_slot = t % kRing;
+      a_b = smem_u32(smem + L::ring + b_slot * L::kSlot);
+      a_x = smem_u32(smem + L::x + (t & 1) * kHeads * kAtom);
+      if (!(ok = wait(kBarRing0 + b_slot))) break;
+    } else if (flags & kPFirst) {
+      ++t;
+      c_slot = (2 * t) % kRing;
+      b_slot = (2 * t + 1) % kRing;
+      a_c = smem_u32(smem + L::ring + c_slot * L::kSlot);
+      a_b = smem_u32(smem + L::ring + b_slot * L::kSlot);
+      a_x = smem_u32(smem + L::x + (t & 1) * kHeads * kAtom);
+      if (!(ok = wait(kBarRing0 + c_slot)) || !(ok = wait(kBarRing0 + b_slot))) break;
+      tc_fence_after();
+      // S = C B^T into buffer t & 1 (the diagonal product that read P(t - 2) from it was
+      // issued earlier by this thread, and tcgen05.mma executes in issue order)
+      const uint32_t d_s = tmem + kColSP + (t & 1) * 128;
+#pragma unroll
+      for (int kk = 0; kk < NS / 16; ++kk) {
+        const uint32_t koff = (kk >> 2) * kAtom + (kk & 3) * 32;
+        umma_f16(d_s, sdesc_sw128(a_c + koff, 16, 1024), sdesc_sw128(a_b + koff, 16, 1024), id_s, kk > 0);
+      }
+      umma_commit(&bars[kBarS0 + (t & 1)]);
+      issued_any = true;
+    }
+    if (state_only) {  // H += B^T [U_0 | U_1] onto h^
+      if (!(ok = wait(kBarHt)) || !(ok = wait(kBarU))) break;
+      tc_fence_after();
+#pragma unroll
+      for (int kk = 0; kk < kTile / 16; ++kk)
+        umma_f16(tmem + kColH, sdesc_sw128(a_b + kk * 2048, kAtom, 1024),
+                 sdesc_sw128(a_x + kk * 2048, kAtom, 1024), id_h, 1);
+      umma_commit(&bars[kBarSt]);
+      if (flags & kPLast) umma_commit(&bars[kBarRingFree0 + b_slot]);
+      issued_any = true;
+      mbar_arrive(&bars[kBarDescFree0 + ds]);
+      continue;
+    }
+    // left factor Y = C [h^_0 h^_1]^T: needs h^ and the previous epilogue done with Y
+    if (!(ok = wait(kBarHt))) break;
+    if (p > 0 && !(ok = wait(kBarFree))) break;
+    tc_fence_after();
+#pragma unroll
+    for (int kk = 0; kk < NS / 16; ++kk) {
+      const uint32_t koff = (kk >> 2) * kAtom + (kk & 3) * 32;
+      umma_f16(tmem + kColY, sdesc_sw128(a_c + koff, 16, 1024), sdesc_sw128(a_ht + kk * 2048, NS * 128, 1024),
+               id_y, kk > 0);
+    }
+    if (flags & kPLast) umma_commit(&bars[kBarRingFree0 + c_slot]);  // C(t) read for the last time
+    // right factor H += B^T [U_0 | U_1]
+    if (!(ok = wait(kBarU))) break;
+    tc_fence_after();
+#pragma unroll
+    for (int kk = 0; kk < kTile / 16; ++kk)
+      umma_f16(tmem + kColH, sdesc_sw128(a_b + kk * 2048, kAtom, 1024), sdesc_sw128(a_x + kk * 2048, kAtom, 1024),
+               id_h, 1);
+    umma_commit(&bars[kBarSt]);
+    if (flags & kPLast) umma_commit(&bars[kBarRingFree0 + b_slot]);  // B(t) read for the last time
+    // diagonal block Y += P [U_0 | U_1], P from tensor memory: K step kk (16 tokens) is
+    // 8 columns at 32 (kk / 2) + 8 (kk % 2) of the buffer
+    if ((flags & kPFirst) && !(ok = wait(kBarP0 + (t & 1)))) break;
+    tc_fence_after();
+    {
+      const uint32_t a_p = tmem + kColSP + (t & 1) * 128;
+#pragma unroll
+      for (int kk = 0; kk < kTile / 16; ++kk)
+        umma_f16_ta(tmem + kColY, a_p + 32 * (kk >> 1) + 8 * (kk & 1), sdesc_sw128(a_x + kk * 2048, kAtom, 1024),
+                    id_y, 1);
+    }
+    umma_commit(&bars[kBarY]);
+    mbar_arrive(&bars[kBarDescFree0 + ds]);
+  }
+  if (!ok) {
+    *abort_flag = 1;
+    // every tcgen05.mma this thread issued completes before tensor memory is freed
+    if (issued_any) {
+      umma_commit(&bars[kBarDrain]);
+      mbar_wait_bounded(&bars[kBarDrain], 0, pb.wait_limit);
+    }
+  }
+}
+
+// --------------------------------------------------------- compute warps
+// Warp w: lane quarter q = w % 4 (TMEM lanes / tile rows 32 q .. 32 q + 31, or state
+// rows n), head hw = w / 8 and column half ch = (w / 4) % 2 of that head's Y, U and
+// state columns; of the mask it converts the 32 x 32 block (q, 2 hw + ch) of S.
+// What is the same for every row of a pass (where it is, the factors, the flags)
+// comes from the helper warp's descriptor.  The two halves of a row quarter meet
+// once a pass, on a one-arrival barrier, before the half-0 warp stores their 32 rows
+// of y by TMA.  Every wait is warp-uniform and bounded.
 template <int NS>
 __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8_t* smem, uint32_t tmem,
                              uint64_t* bars, volatile int* abort_flag) {
   using L = Layout<NS>;
   const int tid = threadIdx.x;
-  const int wid = tid >> 5;                 // compute warp 0..15
-  const int hw = wid >> 3;                  // head of the pair
-  const int ch = (wid >> 2) & 1;            // column half
-  const int wq = wid & 3, lane = tid & 31;  // lane quarter (a warp reaches TMEM lanes 32 (warp % 4) ..)
-  const int i = wq * 32 + lane;             // row / TMEM lane
-  const int pair_bar = kBarPair0 + hw * 4 + wq;
-  const uint32_t lane_base = (uint32_t)(wq * 32) << 16;
+  const int wid = tid >> 5;
+  const int hw = wid >> 3;                   // head of the pair
+  const int ch = (wid >> 2) & 1;             // column half
+  const int q = wid & 3, lane = tid & 31;    // lane quarter
+  const int kb = wid >> 2;                   // S block column of the mask
+  const int i = q * 32 + lane;               // row / TMEM lane
+  const int pair_bar = kBarPair0 + hw * 4 + q;
+  const uint32_t lane_base = (uint32_t)(q * 32) << 16;
   const uint32_t col_h = hw * 64 + ch * 32;  // this warp's Y and state columns
   uint8_t* sx = smem + L::x;
-  uint8_t* sxw = smem + L::xw;
   uint8_t* sht = smem + L::ht;
-  const TileDesc* descs = reinterpret_cast<const TileDesc*>(smem + L::desc);
+  const PassDesc* descs = reinterpret_cast<const PassDesc*>(smem + L::desc);
   const int pairs = pb.H / kHeads;
   const int units = pb.nseq * pairs;
 
-  uint32_t phase = 0;
-  // Warp-uniform bounded wait on a barrier.
+  Phases ph;
   auto wait = [&](int k) -> bool {
-    const bool mine = wait_or_abort(&bars[k], (phase >> k) & 1u, abort_flag);
+    const bool mine = wait_or_abort(&bars[k], ph.parity(k), abort_flag, pb.wait_limit);
     if (__any_sync(0xffffffffu, !mine)) return false;
-    phase ^= 1u << k;
+    ph.flip(k);
     return true;
   };
 
   // Units whose sequences are empty have no tiles: CTA r writes final = init for the
   // empty units u with u % R == r.
-  if (pb.final_state && i < NS) {
+  const int N = pb.N;  // state size (NS, the operand width, is N rounded up; columns past N are 0)
+  if (pb.final_state && i < N) {
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
       if (unit_tiles(pb, u) != 0) continue;
       const int s = u / pairs;
       const int h = (u % pairs) * kHeads + hw;
-      const int64_t base = ((int64_t)s * pb.H + h) * kHeadDim * NS;
+      const int64_t base = ((int64_t)s * pb.H + h) * kHeadDim * N;
       for (int p = 32 * ch; p < 32 * ch + 32; ++p)
-        pb.final_state[base + (int64_t)p * NS + i] = pb.init ? pb.init[base + (int64_t)p * NS + i] : 0.f;
+        pb.final_state[base + (int64_t)p * N + i] = pb.init ? pb.init[base + (int64_t)p * N + i] : 0.f;
     }
   }
 
-  // The head state lives in tensor memory as h^T (lane n = state column n, 64 fp32
-  // columns, 32 per half); its bf16 copy in shared memory is the B operand of the left factor.
-  const uint32_t t_state = tmem + lane_base + kColSt + col_h;
-  auto write_ht_from = [&](const uint32_t (&r)[32]) {
+  // The head state lives in tensor memory as H = h^T (lane n = state column n, 64 fp32
+  // columns per head, 32 per half); its bf16 copy in shared memory is the B operand of
+  // the left factor.  Both hold the same scaled value h^.
+  const uint32_t t_state = tmem + lane_base + kColH + col_h;
+  auto write_state = [&](uint32_t (&r)[32], float sig) {
+    const uint64_t s2 = f2(sig, sig);
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      float lo, hi;
+      unf2(mul2(s2, f2u(r[2 * k], r[2 * k + 1])), lo, hi);
+      r[2 * k] = __float_as_uint(lo);
+      r[2 * k + 1] = __float_as_uint(hi);
+    }
     if (i < NS) {
       uint8_t* hdst = sht + hw * NS * 128;
 #pragma unroll
@@ -497,310 +529,261 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
         *reinterpret_cast<uint4*>(hdst + sw128_off(i, 4 * ch + c)) = hv;
       }
     }
+    tmem_st32(t_state, r);
+    tmem_st_wait();
   };
-  // The state at the start of the piece whose first tile d describes, into r: the
-  // sequence's initial state (or zero), or the state the previous CTA handed on.
-  // False if the wait for that hand-on gave up.
-  auto load_state = [&](const TileDesc& d, uint32_t (&r)[32]) -> bool {
+  // The state at the start of the piece whose first pass d describes, into r: the
+  // sequence's initial state (or zero), or the state the previous CTA handed on (each
+  // warp waits for the matching warp of that CTA).  False if that wait gave up.
+  auto load_state = [&](const PassDesc& d, uint32_t (&r)[32]) -> bool {
     const float* src_p = nullptr;
-    if (d.flags & kDescCarryIn) {
+    if (d.flags & kPCarryIn) {
       const int src = d.carry_src;
       bool mine = true;
       if (lane == 0) {
         const long long t0 = clock64();
-        while (ld_acquire_gpu(&pb.carry_flag[src]) < kComputeWarps) {
-          if (*abort_flag || clock64() - t0 > kWaitLimit) {
+        while (ld_acquire_gpu_u64(&pb.carry_flag[src * kComputeWarps + wid]) != pb.epoch) {
+          if (*abort_flag || clock64() - t0 > pb.wait_limit) {
             *abort_flag = 1;
             mine = false;
             break;
           }
-          __nanosleep(200);
+          __nanosleep(100);
         }
       }
       if (__any_sync(0xffffffffu, !mine)) return false;
       __threadfence();
-      src_p = pb.carry + ((size_t)src * kHeads + hw) * kHeadDim * NS + i;
+      src_p = pb.carry + ((size_t)src * kHeads + hw) * kHeadDim * N + i;
     } else if (pb.init) {
-      src_p = pb.init + ((int64_t)d.s * pb.H + d.h0 + hw) * kHeadDim * NS + i;
+      src_p = pb.init + ((int64_t)d.s * pb.H + d.h0 + hw) * kHeadDim * N + i;
     }
 #pragma unroll
-    for (int q = 0; q < 32; ++q)
-      r[q] = __float_as_uint((src_p && i < NS) ? __ldcg(src_p + (size_t)(32 * ch + q) * NS) : 0.f);
+    for (int k = 0; k < 32; ++k)
+      r[k] = __float_as_uint((src_p && i < N) ? __ldcg(src_p + (size_t)(32 * ch + k) * N) : 0.f);
     return true;
-  };
-  // r holds the state at the start of the tile d describes: its bf16 copy is the left
-  // factor's operand; scaled by the tile's decay it is what the right factor accumulates onto.
-  auto start_tile_state = [&](const TileDesc& d, uint32_t (&r)[32]) {
-    write_ht_from(r);
-    const float decay = d.decay[hw];
-    const uint64_t decay2 = f2(decay, decay);
-#pragma unroll
-    for (int q = 0; q < 16; ++q) {
-      float lo, hi;
-      unf2(mul2(decay2, f2u(r[2 * q], r[2 * q + 1])), lo, hi);
-      r[2 * q] = __float_as_uint(lo);
-      r[2 * q + 1] = __float_as_uint(hi);
-    }
-    tmem_st32(t_state, r);
-    tmem_st_wait();
-  };
-  // P values of one 32-column block of S (fp32 bits in r) for row i.
-  auto mask_block = [&](int cb, const uint32_t* r, float cs_i, const float* dcs, const float* dcc,
-                        const float* ddt, uint32_t (&pk)[16]) {
-    if (cb < wq) {  // strictly below the diagonal: exp(cs_i - cs_j) = rf * exp(cs_ref - cs_j)
-      const float rf = ex2(cs_i - dcs[cb * 32 + 31]);
-      const uint64_t rf2 = f2(rf, rf);
-      const float4* cc4 = reinterpret_cast<const float4*>(dcc + cb * 32);
-#pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4) {
-        const float4 c = cc4[q4];
-        const uint64_t f0 = mul2(rf2, f2(c.x, c.y)), f1 = mul2(rf2, f2(c.z, c.w));
-        pk[2 * q4] = bf16x2_of(mul2(f0, f2u(r[4 * q4], r[4 * q4 + 1])));
-        pk[2 * q4 + 1] = bf16x2_of(mul2(f1, f2u(r[4 * q4 + 2], r[4 * q4 + 3])));
-      }
-    } else {  // diagonal block: mask first (-inf), then exp
-      const float4* c4 = reinterpret_cast<const float4*>(dcs + cb * 32);
-      const float4* d4 = reinterpret_cast<const float4*>(ddt + cb * 32);
-#pragma unroll
-      for (int q4 = 0; q4 < 8; ++q4) {
-        const float4 cj = c4[q4], dj = d4[q4];
-        const int j0 = 4 * q4;  // column within the block; this row is `lane`
-        const float e0 = ex2(j0 <= lane ? cs_i - cj.x : -INFINITY);
-        const float e1 = ex2(j0 + 1 <= lane ? cs_i - cj.y : -INFINITY);
-        const float e2 = ex2(j0 + 2 <= lane ? cs_i - cj.z : -INFINITY);
-        const float e3 = ex2(j0 + 3 <= lane ? cs_i - cj.w : -INFINITY);
-        pk[2 * q4] = bf16x2_of(mul2(mul2(f2(e0, e1), f2(dj.x, dj.y)), f2u(r[j0], r[j0 + 1])));
-        pk[2 * q4 + 1] = bf16x2_of(mul2(mul2(f2(e2, e3), f2(dj.z, dj.w)), f2u(r[j0 + 2], r[j0 + 3])));
-      }
-    }
   };
 
   if (!wait(kBarDescFull0)) return;
-  if (descs[0].flags & kDescEnd) return;
+  if (descs[0].flags & kPEnd) return;
   {
     uint32_t r[32];
     if (!load_state(descs[0], r)) return;
-    start_tile_state(descs[0], r);
+    write_state(r, descs[0].sig_in[hw]);
   }
   fence_proxy_async();
   tc_fence_before();
   warp_arrive(&bars[kBarHt]);
-  int trace_tile = 0;
-  (void)trace_tile;
 
-  for (int t = 0;; ++t) {
-    const int slot = t % kDescSlots, stage = t & 1;
-    const TileDesc& d = descs[slot];
-    TRACE_MARK(0);
-    const int h = d.h0 + hw;
-    const int t0 = d.t0, rem = d.rem, flags = d.flags;
-    const float* dcs = d.cs[hw];
-    const float* dcc = d.cc[hw];
-    const float* ddt = d.dtv[hw];
-    const float cs_start = d.cs_start[hw], cs_end = d.cs_end[hw];
-    const float cs_i = dcs[i];
-    const float w_i = ex2(cs_end - cs_i) * ddt[i];  // right-factor weight (0 past the end)
-    const float carry = ex2(cs_i - cs_start);      // decay of the carried-in state to token i
-    TRACE_MARK(1);
+  const bool state_only = pb.y == nullptr;  // only the final states: no mask, no epilogue
+  uint32_t xr[16];  // this thread's x of the current tile: row i, columns 32 ch .. 32 ch + 31 of head hw
+  int t = -1;
+  bool staged_prev = false;  // the previous tile's y went out by TMA from its x stage
+  for (int p = 0;; ++p) {
+    const int ds = p % kDescSlots;
+    const PassDesc& d = descs[ds];
+    const int flags = d.flags;
+    if (flags & kPFirst) ++t;
+    const int st = t & 1;
+    uint8_t* sxh = sx + (st * kHeads + hw) * kAtom;
 
-    // ---- this tile's x: w o x, the right-factor input
-    if (!wait(stage)) return;
-    TRACE_MARK(2);
-    const uint8_t* sxh = sx + (stage * kHeads + hw) * kAtom;
-    {
-      uint8_t* dst = sxw + hw * kAtom;
-      const uint32_t w2 = pack_bf16(w_i, w_i);
+    // ---- U = u_i x_i over the tile's x, in place (x itself stays in registers)
+    if (flags & kPFirst) {
+      if (!wait(kBarX0 + st)) return;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const uint32_t o = sw128_off(i, 4 * ch + cc);
-        uint4 xv = *reinterpret_cast<const uint4*>(sxh + o);
-        xv.x = mul_bf16x2(xv.x, w2);
-        xv.y = mul_bf16x2(xv.y, w2);
-        xv.z = mul_bf16x2(xv.z, w2);
-        xv.w = mul_bf16x2(xv.w, w2);
-        *reinterpret_cast<uint4*>(dst + o) = xv;
+      for (int c = 0; c < 4; ++c) {
+        const uint4 v = *reinterpret_cast<const uint4*>(sxh + sw128_off(i, 4 * ch + c));
+        xr[4 * c] = v.x, xr[4 * c + 1] = v.y, xr[4 * c + 2] = v.z, xr[4 * c + 3] = v.w;
+      }
+    }
+    {
+      const float u = d.u[hw][i];
+      const uint32_t u2 = pack_bf16(u, u);
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        uint4 v;
+        v.x = mul_bf16x2(xr[4 * c], u2);
+        v.y = mul_bf16x2(xr[4 * c + 1], u2);
+        v.z = mul_bf16x2(xr[4 * c + 2], u2);
+        v.w = mul_bf16x2(xr[4 * c + 3], u2);
+        *reinterpret_cast<uint4*>(sxh + sw128_off(i, 4 * ch + c)) = v;
       }
     }
     fence_proxy_async();
-    warp_arrive(&bars[kBarXw]);
-    if (t > 0) {  // this warp's y store of the previous tile has read its x stage: release it
-      if (lane == 0) bulk_wait_read();
-      warp_arrive(&bars[kBarXfree]);
-    }
-    TRACE_MARK(3);
+    warp_arrive(&bars[kBarU]);
 
-    // ---- P_h = mask_h(S), bf16 pairs in tensor memory
-    if (!wait(kBarS)) return;
-    TRACE_MARK(4);
-    tc_fence_after();
-    {
-      // blocks ch and ch + 2 (32 columns of S each) -> P columns 16 cb .. 16 cb + 15
-      const uint32_t colp = kColP + hw * 64;
-#pragma unroll 1
-      for (int cb = ch; cb < 4; cb += 2) {
-        uint32_t pk[16];
-        if (cb <= wq) {
-          uint32_t r[32];
-          tmem_ld32(tmem + lane_base + kColS + cb * 32, r);
-          tmem_ld_wait();
-          mask_block(cb, r, cs_i, dcs, dcc, ddt, pk);
-        } else {  // above the diagonal: zero
+    if (flags & kPFirst) {
+      // the previous tile's x stage: its y store has read it, so it may take tile t + 1's x
+      if (t > 0) {
+        if (staged_prev && ch == 0 && lane == 0) bulk_wait_read();
+        warp_arrive(&bars[kBarXfree0 + (st ^ 1)]);
+      }
+    }
+    // ---- P = bf16(S) on and below the diagonal, written in place over S
+    if ((flags & kPFirst) && !state_only) {
+      if (!wait(kBarS0 + st)) return;
+      tc_fence_after();
+      const uint32_t t_blk = tmem + lane_base + kColSP + st * 128 + kb * 32;
+      uint32_t pk[16];
+      if (kb < q) {
+        uint32_t s[32];
+        tmem_ld32(t_blk, s);
+        tmem_ld_wait();
 #pragma unroll
-          for (int q = 0; q < 16; ++q) pk[q] = 0u;
+        for (int k = 0; k < 16; ++k) pk[k] = bf16x2_of(f2u(s[2 * k], s[2 * k + 1]));
+      } else if (kb == q) {  // diagonal block: column 32 kb + j of row 32 q + lane kept for j <= lane
+        uint32_t s[32];
+        tmem_ld32(t_blk, s);
+        tmem_ld_wait();
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          const uint32_t lo = 2 * k <= lane ? s[2 * k] : 0u;
+          const uint32_t hi = 2 * k + 1 <= lane ? s[2 * k + 1] : 0u;
+          pk[k] = bf16x2_of(f2u(lo, hi));
         }
-        tmem_st16(tmem + lane_base + colp + cb * 16, pk);
-      }
-    }
-    TRACE_MARK(5);
-
-    // ---- scale the left factor's row by exp(cs_i - cs_start), in place in Y
-    if (!wait(kBarYo)) return;
-    tc_fence_after();
-    {
-      const uint64_t carry2 = f2(carry, carry);
-      uint32_t r[32];
-      tmem_ld32(tmem + lane_base + kColY + col_h, r);
-      tmem_ld_wait();
+      } else {
 #pragma unroll
-      for (int q = 0; q < 16; ++q) {
-        float lo, hi;
-        unf2(mul2(carry2, f2u(r[2 * q], r[2 * q + 1])), lo, hi);
-        r[2 * q] = __float_as_uint(lo);
-        r[2 * q + 1] = __float_as_uint(hi);
+        for (int k = 0; k < 16; ++k) pk[k] = 0u;
       }
-      tmem_st32(tmem + lane_base + kColY + col_h, r);
+      tmem_st16(t_blk, pk);
+      tmem_st_wait();
+      tc_fence_before();
+      warp_arrive(&bars[kBarP0 + st]);
     }
-    tmem_st_wait();
-    tc_fence_before();
-    warp_arrive(&bars[kBarP]);
-    TRACE_MARK(6);
 
-    // ---- the state after this tile: at the end of a piece the final state or the
-    // hand-on to the next CTA; then the next tile's start state (this one, or the next
-    // piece's) as its bf16 copy and, decay-scaled, in tensor memory
+    // ---- the state after this pass: at the end of a piece the final state or the
+    // hand-on to the next CTA; then the next pass's h^ (this state rescaled, or the next
+    // piece's initial state) as its bf16 copy and in tensor memory
     if (!wait(kBarSt)) return;
     tc_fence_after();
-    const int nslot = (t + 1) % kDescSlots;
+    const int nds = (p + 1) % kDescSlots;
     bool more;
     {
       uint32_t r[32];
       tmem_ld32(t_state, r);
       tmem_ld_wait();
-      if ((flags & kDescToFinal) && i < NS) {
-        float* fp = pb.final_state + ((int64_t)d.s * pb.H + h) * kHeadDim * NS + i;
+      if (flags & (kPToFinal | kPToCarry)) {
+        const float so = d.sig_out[hw];
+        float* dst = (flags & kPToFinal)
+                         ? pb.final_state + ((int64_t)d.s * pb.H + d.h0 + hw) * kHeadDim * N + i
+                         : pb.carry + ((size_t)blockIdx.x * kHeads + hw) * kHeadDim * N + i;
+        if (i < N) {
 #pragma unroll
-        for (int q = 0; q < 32; ++q) fp[(size_t)(32 * ch + q) * NS] = __uint_as_float(r[q]);
-      }
-      if (flags & kDescToCarry) {  // hand the state on: one release increment per warp once its part is out
-        if (i < NS) {
-          float* cp = pb.carry + ((size_t)blockIdx.x * kHeads + hw) * kHeadDim * NS + i;
-#pragma unroll
-          for (int q = 0; q < 32; ++q) cp[(size_t)(32 * ch + q) * NS] = __uint_as_float(r[q]);
+          for (int k = 0; k < 32; ++k) dst[(size_t)(32 * ch + k) * N] = so * __uint_as_float(r[k]);
         }
-        if (i == 0 && ch == 0)
-          pb.carry[(size_t)pb.ranges * kHeads * kHeadDim * NS + blockIdx.x * kHeads + hw] = cs_end;
-        __threadfence();
-        __syncwarp();
-        if (lane == 0) red_add_release_gpu(&pb.carry_flag[blockIdx.x], 1);
-        __syncwarp();
+        if (flags & kPToCarry) {  // this warp's part is out: one release per warp
+          __threadfence();
+          __syncwarp();
+          if (lane == 0 && !pb.withhold_carry)
+            st_release_gpu_u64(&pb.carry_flag[blockIdx.x * kComputeWarps + wid], pb.epoch);
+          __syncwarp();
+        }
       }
-      TRACE_MARK(10);
-      if (!wait(kBarDescFull0 + nslot)) return;
-      TRACE_MARK(11);
-      const TileDesc& dn = descs[nslot];
-      more = !(dn.flags & kDescEnd);
+      if (!wait(kBarDescFull0 + nds)) return;
+      const PassDesc& dn = descs[nds];
+      more = !(dn.flags & kPEnd);
       if (more) {
-        if ((dn.flags & kDescFirst) && !load_state(dn, r)) return;
-        start_tile_state(dn, r);
+        float sig;
+        if (dn.flags & kPPieceStart) {
+          if (!load_state(dn, r)) return;
+          sig = dn.sig_in[hw];
+        } else {
+          sig = d.sig_out[hw] * dn.sig_in[hw];
+        }
+        write_state(r, sig);
       }
     }
     fence_proxy_async();
     tc_fence_before();
     warp_arrive(&bars[kBarHt]);
-    TRACE_MARK(7);
 
-    // ---- epilogue: y = Y + D x, staged over this tile's x; the half-0 warp of each row
-    // quarter stores the quarter's 32 rows by TMA once the half-1 warp has staged its columns
+    if (state_only) {
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kBarDescFree0 + ds]);
+      __syncwarp();
+      if (!more) break;
+      continue;
+    }
+    // ---- epilogue: y = r_i Y + D x; a single-pass tile stages y over its U and the
+    // half-0 warp of each row quarter stores the quarter's 32 rows by TMA once the
+    // half-1 warp has staged its columns; other rows go out as row stores
     if (!wait(kBarY)) return;
-    TRACE_MARK(8);
     tc_fence_after();
+    const bool single = (flags & (kPFirst | kPLast)) == (kPFirst | kPLast);
+    const bool staged = single && d.rem >= 32 * q + 32;  // all 32 rows of this quarter are in the sequence
     {
+      const float rr = d.r[hw][i];
       const float Dh = d.dskip[hw];
-      const uint64_t d2 = f2(Dh, Dh);
-      const bool full = rem >= 32 * wq + 32;  // all 32 rows of this quarter are in the sequence
-      uint8_t* ystage = const_cast<uint8_t*>(sxh);  // each thread overwrites the x chunks it reads
-      __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(pb.y) + ((int64_t)(t0 + i) * pb.H + h) * kHeadDim;
+      const uint64_t r2 = f2(rr, rr), d2 = f2(Dh, Dh);
+      const int h = d.h0 + hw;
       uint32_t ry[32];
       tmem_ld32(tmem + lane_base + kColY + col_h, ry);
       tmem_ld_wait();
+      const bool row_ok = !staged && i >= d.lo && i < d.hi && i < d.rem;
+      __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(pb.y) + ((int64_t)(d.t0 + i) * pb.H + h) * kHeadDim;
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
-        const int c = 4 * ch + cc;
-        const uint32_t o = sw128_off(i, c);
-        const uint4 xv = *reinterpret_cast<const uint4*>(sxh + o);
-        const uint32_t xu[4] = {xv.x, xv.y, xv.z, xv.w};
+      for (int c = 0; c < 4; ++c) {
         uint32_t out[4];
 #pragma unroll
-        for (int q = 0; q < 4; ++q) {  // bf16 pair -> fp32 pair (exact), then D x + Y as one f32x2 fma
-          const uint64_t x2 = f2u(xu[q] << 16, xu[q] & 0xFFFF0000u);
-          out[q] = bf16x2_of(fma2(d2, x2, f2u(ry[8 * cc + 2 * q], ry[8 * cc + 2 * q + 1])));
+        for (int k = 0; k < 4; ++k) {  // bf16 pair -> fp32 pair (exact), then r Y + D x
+          const uint32_t xu = xr[4 * c + k];
+          const uint64_t x2 = f2u(xu << 16, xu & 0xFFFF0000u);
+          out[k] = bf16x2_of(fma2(r2, f2u(ry[8 * c + 2 * k], ry[8 * c + 2 * k + 1]), mul2(d2, x2)));
         }
         const uint4 ov = make_uint4(out[0], out[1], out[2], out[3]);
-        if (full)
-          *reinterpret_cast<uint4*>(ystage + o) = ov;
-        else if (i < rem)
-          *reinterpret_cast<uint4*>(yrow + 8 * c) = ov;
+        if (staged)
+          *reinterpret_cast<uint4*>(sxh + sw128_off(i, 4 * ch + c)) = ov;
+        else if (row_ok)
+          *reinterpret_cast<uint4*>(yrow + 32 * ch + 8 * c) = ov;
       }
       tc_fence_before();
-      if (full) fence_proxy_async();
+      if (staged) fence_proxy_async();
       __syncwarp();
       if (ch == 1) {
         if (lane == 0) mbar_arrive(&bars[pair_bar]);
       } else {
         if (!wait(pair_bar)) return;
-        if (full && lane == 0) {
-          tma_store_3d(tm_y32, ystage + wq * 32 * 128, 0, h, t0 + 32 * wq);
+        if (staged && lane == 0) {
+          tma_store_3d(tm_y32, sxh + q * 32 * 128, 0, h, d.t0 + 32 * q);
           bulk_commit();
         }
       }
       __syncwarp();
     }
-    // Y is free for the next left factor; this tile's descriptor is used up
+    if (flags & kPLast) staged_prev = staged;
+    // Y is free for the next left factor; this pass's descriptor is used up
     __syncwarp();
     if (lane == 0) {
       mbar_arrive(&bars[kBarFree]);
-      mbar_arrive(&bars[kBarDescFree0 + slot]);
+      mbar_arrive(&bars[kBarDescFree0 + ds]);
     }
     __syncwarp();
-    TRACE_MARK(9);
-    ++trace_tile;
     if (!more) break;
   }
 }
 
-// ------------------------------------------------------------------ helper warps
-// Helper warp hh walks the CTA's tile sequence a few tiles ahead of the compute warps,
-// loads each tile's dt by TMA into a ring of its own (kDtStages tiles in flight) and
-// writes head hh's part of the tile's descriptor into a ring of kDescSlots: the in-chunk
-// cumsum of dt A in log2 units (restarted at every chunk boundary, and continued from the
-// handing-on CTA's value at a hand-on), the column factors exp2(cs(end of 32-block) -
-// cs_j) dt_j, dt (0 past the sequence end), the decay and D.  Helper 0 also writes where
-// the tile is and what happens to the state around it.  The descriptor is complete when
-// both helpers have arrived.
+// ------------------------------------------------------------------ helper warp
+// The helper walks the CTA's tile sequence ahead of the compute warps, loads each
+// tile's dt by TMA into a ring of its own (kDtStages tiles in flight), and writes one
+// descriptor per pass into a ring of kDescSlots: where the pass is, its rows, the
+// factors u and r of both heads, the state scalings and the piece flags.  Per tile it
+// forms c (the inclusive cumsum of dt A in log2 units from the tile start, both heads)
+// and cuts the valid rows into passes whose decay range is at most kRangeMax: one pass
+// unless a head decays by more than 2^-kRangeMax across the tile.
 template <int NS>
 __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t* smem, uint64_t* bars,
-                            volatile int* abort_flag, int hh) {
+                            volatile int* abort_flag) {
   using L = Layout<NS>;
   const int lane = threadIdx.x & 31;
-  uint8_t* my_dt = smem + L::sdt + hh * kDtStages * kTile * 16;
-  uint64_t* my_bar = bars + kBarDt0 + hh * kDtStages;
+  uint8_t* sdt = smem + L::sdt;
+  uint64_t* dt_bar = bars + kBarDt0;
+  float* sc = reinterpret_cast<float*>(smem + L::scan);  // c[head][128]
   const int pairs = pb.H / kHeads;
-  TileDesc* descs = reinterpret_cast<TileDesc*>(smem + L::desc);
-  uint32_t phase = 0;
+  PassDesc* descs = reinterpret_cast<PassDesc*>(smem + L::desc);
+  Phases ph;
   auto wait = [&](int k) -> bool {
-    const bool mine = wait_or_abort(&bars[k], (phase >> k) & 1u, abort_flag);
+    const bool mine = wait_or_abort(&bars[k], ph.parity(k), abort_flag, pb.wait_limit);
     if (__any_sync(0xffffffffu, !mine)) return false;
-    phase ^= 1u << k;
+    ph.flip(k);
     return true;
   };
   const RangePlan rp = plan_range(pb);
@@ -813,8 +796,8 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t
     if (lane == 0) {
       const int st = dt_issued % kDtStages;
       const int h0 = (ahead.unit % pairs) * kHeads;
-      mbar_expect_tx(&my_bar[st], kTile * 16);
-      tma_load_2d(my_dt + st * kTile * 16, tm_dt, h0 & ~3, ahead.tb + ahead.k0, &my_bar[st]);
+      mbar_expect_tx(&dt_bar[st], kTile * 16);
+      tma_load_2d(sdt + st * kTile * 16, tm_dt, h0 & ~3, ahead.tb + ahead.k0, &dt_bar[st]);
     }
     ++dt_issued;
     have_ahead = cursor_next(pb, rp, ahead);
@@ -823,120 +806,156 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t
 
   TileCursor cur;
   bool have = cursor_first(pb, rp, cur);
-  float cs_base = 0.f, a2 = 0.f, dsk = 0.f;
+  float a2[kHeads] = {0.f, 0.f}, dsk[kHeads] = {0.f, 0.f};
   int a_unit = -1, prev_piece = -1;
   bool ok = true;
-  int t = 0;
+  int t = 0, p = 0;
+  auto take_slot = [&]() -> PassDesc* {
+    const int slot = p % kDescSlots;
+    if (p >= kDescSlots && !wait(kBarDescFree0 + slot)) return nullptr;
+    return &descs[slot];
+  };
+  auto publish = [&]() {
+    __syncwarp();
+    if (lane == 0) mbar_arrive(&bars[kBarDescFull0 + p % kDescSlots]);
+    ++p;
+  };
   for (;; ++t) {
-    const int slot = t % kDescSlots;
-    if (t >= kDescSlots && !(ok = wait(kBarDescFree0 + slot))) break;
-    TileDesc& d = descs[slot];
     if (!have) {
-      if (hh == 0 && lane == 0) d.flags = kDescEnd;
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[kBarDescFull0 + slot]);
+      PassDesc* d = take_slot();
+      if (!d) {
+        ok = false;
+        break;
+      }
+      if (lane == 0) d->flags = kPEnd;
+      publish();
       break;
     }
     TileCursor nxt = cur;
     const bool have_next = cursor_next(pb, rp, nxt);
-    const bool first = cur.piece != prev_piece;
-    const bool last = !have_next || nxt.piece != cur.piece;
+    const bool first_tile = cur.piece != prev_piece;
+    const bool last_tile = !have_next || nxt.piece != cur.piece;
     prev_piece = cur.piece;
     const int h0 = (cur.unit % pairs) * kHeads;
     if (cur.unit != a_unit) {
       a_unit = cur.unit;
-      a2 = pb.A[h0 + hh] * 1.4426950408889634f;  // A_h log2(e): cumsums are in log2 units
-      dsk = pb.D ? pb.D[h0 + hh] : 0.f;
-    }
-    int flags = 0;
-    if (first) {
-      flags |= kDescFirst;
-      cs_base = 0.f;
-      if (cur.flags & kCarryIn) {  // continue from the cumsum the previous CTA reached
-        flags |= kDescCarryIn;
-        bool mine = true;
-        if (lane == 0) {
-          const long long c0 = clock64();
-          while (ld_acquire_gpu(&pb.carry_flag[rp.carry_src]) < kComputeWarps) {
-            if (*abort_flag || clock64() - c0 > kWaitLimit) {
-              *abort_flag = 1;
-              mine = false;
-              break;
-            }
-            __nanosleep(200);
-          }
-        }
-        if (__any_sync(0xffffffffu, !mine)) {
-          ok = false;
-          break;
-        }
-        __threadfence();
-        cs_base = __ldcg(pb.carry + (size_t)pb.ranges * kHeads * kHeadDim * NS + rp.carry_src * kHeads + hh);
+#pragma unroll
+      for (int hh = 0; hh < kHeads; ++hh) {
+        a2[hh] = pb.A[h0 + hh] * 1.4426950408889634f;  // A_h log2(e): cumsums are in log2 units
+        dsk[hh] = pb.D ? pb.D[h0 + hh] : 0.f;
       }
     }
-    if (last && (cur.flags & kUnitEnd) && pb.final_state) flags |= kDescToFinal;
-    if (last && (cur.flags & kCarryOut)) flags |= kDescToCarry;
-    if (cur.k0 % pb.Q == 0) cs_base = 0.f;
+    const int rem = min(kTile, cur.len - cur.k0);
 
     // this tile's dt: row 4 lane + j holds the 4 heads' dt of one token; a lane reads its
     // rows in the order j = (k + rot) & 3, rot = (lane / 2) & 3, so each quarter warp's
     // 16-byte loads fall in distinct banks
-    if (!(ok = wait(kBarDt0 + hh * kDtStages + t % kDtStages))) break;
-    float dtt[4];
+    if (!(ok = wait(kBarDt0 + t % kDtStages))) break;
+    float dtt[kHeads][4];
     {
-      const float4* rows = reinterpret_cast<const float4*>(my_dt + (t % kDtStages) * kTile * 16) + 4 * lane;
-      const int rot = (lane >> 1) & 3, c = (h0 & 3) + hh;  // this head's column in the 4-head row
-      float v[4];
+      const float4* rows = reinterpret_cast<const float4*>(sdt + (t % kDtStages) * kTile * 16) + 4 * lane;
+      const int rot = (lane >> 1) & 3, c0 = h0 & 3;  // the pair's first column in the 4-head row
+      float v0[4], v1[4];
 #pragma unroll
       for (int k = 0; k < 4; ++k) {
-        const float4 q = rows[(k + rot) & 3];
-        v[k] = c == 0 ? q.x : c == 1 ? q.y : c == 2 ? q.z : q.w;
+        const float4 qv = rows[(k + rot) & 3];
+        v0[k] = c0 == 0 ? qv.x : qv.z;
+        v1[k] = c0 == 0 ? qv.y : qv.w;
       }
-      const int left = cur.len - cur.k0 - 4 * lane;
+      const int left = rem - 4 * lane;
 #pragma unroll
       for (int j = 0; j < 4; ++j) {  // token j came in as k = (j - rot) & 3
         const int k = (j - rot) & 3;
-        const float val = k == 0 ? v[0] : k == 1 ? v[1] : k == 2 ? v[2] : v[3];
-        dtt[j] = j < left ? dt_value(pb, val, h0 + hh) : 0.f;
+        const float x0 = k == 0 ? v0[0] : k == 1 ? v0[1] : k == 2 ? v0[2] : v0[3];
+        const float x1 = k == 0 ? v1[0] : k == 1 ? v1[1] : k == 2 ? v1[2] : v1[3];
+        dtt[0][j] = j < left ? dt_value(pb, x0, h0) : 0.f;
+        dtt[1][j] = j < left ? dt_value(pb, x1, h0 + 1) : 0.f;
       }
     }
-    {
-      float c0 = dtt[0] * a2, c1 = c0 + dtt[1] * a2, c2 = c1 + dtt[2] * a2, c3 = c2 + dtt[3] * a2;
+    // the dt stage is read: refill it
+    __syncwarp();
+    if (have_ahead) issue_dt();
+    // inclusive cumsum c of dt A (log2 units) from the tile start, both heads
+    float cth[kHeads][4];
+#pragma unroll
+    for (int hh = 0; hh < kHeads; ++hh) {
+      float c0 = dtt[hh][0] * a2[hh], c1 = c0 + dtt[hh][1] * a2[hh], c2 = c1 + dtt[hh][2] * a2[hh],
+            c3 = c2 + dtt[hh][3] * a2[hh];
       float v = c3;
 #pragma unroll
       for (int o = 1; o < 32; o <<= 1) {
         const float u = __shfl_up_sync(0xffffffffu, v, o);
         if (lane >= o) v += u;
       }
-      const float base = cs_base + v - c3;  // cumsum before token 4 lane
-      c0 += base, c1 += base, c2 += base, c3 += base;
-      reinterpret_cast<float4*>(d.cs[hh])[lane] = make_float4(c0, c1, c2, c3);
-      reinterpret_cast<float4*>(d.dtv[hh])[lane] = make_float4(dtt[0], dtt[1], dtt[2], dtt[3]);
-      // block ends (tokens 31, 63, 95, 127) live in lanes 7, 15, 23, 31
-      const float ref = __shfl_sync(0xffffffffu, c3, (lane & ~7) | 7);
-      reinterpret_cast<float4*>(d.cc[hh])[lane] = make_float4(ex2(ref - c0) * dtt[0], ex2(ref - c1) * dtt[1],
-                                                              ex2(ref - c2) * dtt[2], ex2(ref - c3) * dtt[3]);
-      const float cs_end = __shfl_sync(0xffffffffu, c3, 31);  // tokens past the end add 0
-      if (lane == 0) {
-        d.cs_start[hh] = cs_base;
-        d.cs_end[hh] = cs_end;
-        d.decay[hh] = ex2(cs_end - cs_base);
-        d.dskip[hh] = dsk;
-      }
-      cs_base = cs_end;
-    }
-    if (hh == 0 && lane == 0) {
-      d.t0 = cur.tb + cur.k0;
-      d.rem = min(kTile, cur.len - cur.k0);
-      d.s = cur.unit / pairs;
-      d.h0 = h0;
-      d.flags = flags;
-      d.carry_src = rp.carry_src;
+      const float base = v - c3;  // cumsum before token 4 lane
+      cth[hh][0] = c0 + base, cth[hh][1] = c1 + base, cth[hh][2] = c2 + base, cth[hh][3] = c3 + base;
+      reinterpret_cast<float4*>(sc + hh * kTile)[lane] = make_float4(cth[hh][0], cth[hh][1], cth[hh][2], cth[hh][3]);
     }
     __syncwarp();
-    if (lane == 0) mbar_arrive(&bars[kBarDescFull0 + slot]);
-    // the dt stage this tile used is read: refill it
-    if (have_ahead) issue_dt();
+
+    // passes over rows [0, rem): each as long as both heads' decay range fits
+    for (int lo = 0; lo < rem;) {
+      const float clo0 = sc[lo], clo1 = sc[kTile + lo];
+      int bad = kTile;  // first row j > lo whose range from lo is too wide
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int row = 4 * lane + j;
+        if (row > lo && row < rem && bad == kTile &&
+            (fabsf(clo0 - cth[0][j]) > kRangeMax || fabsf(clo1 - cth[1][j]) > kRangeMax))
+          bad = row;
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) bad = min(bad, __shfl_xor_sync(0xffffffffu, bad, o));
+      const int hi = min(bad, rem);
+
+      PassDesc* d = take_slot();
+      if (!d) {
+        ok = false;
+        break;
+      }
+#pragma unroll
+      for (int hh = 0; hh < kHeads; ++hh) {
+        const float* ch_ = sc + hh * kTile;
+        const float m = 0.5f * (ch_[lo] + ch_[hi - 1]);
+        float u[4], r[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int row = 4 * lane + j;
+          const bool in = row >= lo && row < hi;
+          u[j] = in ? ex2(m - cth[hh][j]) * dtt[hh][j] : 0.f;
+          r[j] = in ? ex2(cth[hh][j] - m) : 0.f;
+        }
+        reinterpret_cast<float4*>(d->u[hh])[lane] = make_float4(u[0], u[1], u[2], u[3]);
+        reinterpret_cast<float4*>(d->r[hh])[lane] = make_float4(r[0], r[1], r[2], r[3]);
+        if (lane == 0) {
+          const float cb = lo > 0 ? ch_[lo - 1] : 0.f;
+          d->sig_in[hh] = ex2(m - cb);
+          d->sig_out[hh] = ex2(ch_[hi - 1] - m);
+          d->dskip[hh] = dsk[hh];
+        }
+      }
+      if (lane == 0) {
+        int flags = 0;
+        if (lo == 0) flags |= kPFirst;
+        if (hi == rem) flags |= kPLast;
+        if (first_tile && lo == 0) flags |= kPPieceStart | ((cur.flags & kCarryIn) ? kPCarryIn : 0);
+        if (last_tile && hi == rem) {
+          if ((cur.flags & kUnitEnd) && pb.final_state) flags |= kPToFinal;
+          if (cur.flags & kCarryOut) flags |= kPToCarry;
+        }
+        d->t0 = cur.tb + cur.k0;
+        d->rem = rem;
+        d->lo = lo;
+        d->hi = hi;
+        d->s = cur.unit / pairs;
+        d->h0 = h0;
+        d->flags = flags;
+        d->carry_src = rp.carry_src;
+      }
+      publish();
+      lo = hi;
+    }
+    if (!ok) break;
     cur = nxt;
     have = have_next;
   }
@@ -944,8 +963,7 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t
     *abort_flag = 1;
     // dt loads still in flight land before the CTA ends (bounded)
     if (lane == 0)
-      for (int n = t; n < dt_issued; ++n)
-        mbar_wait_bounded(&my_bar[n % kDtStages], (n / kDtStages) & 1, kWaitLimit);
+      for (int n = t; n < dt_issued; ++n) mbar_wait_bounded(&dt_bar[n % kDtStages], (n / kDtStages) & 1, pb.wait_limit);
   }
 }
 
@@ -962,28 +980,33 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* bars = reinterpret_cast<uint64_t*>(smem + L::bars);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + L::flag);
 
-  if (*pb.nchunks < 0) return;  // cu_seqlens rejected by the table kernel
+  if (pb.cu && *pb.nchunks < 0) return;  // cu_seqlens rejected by the table kernel
 
   if (warp == 0) {
     tmem_alloc(&s_tmem_base, kTmemCols);
     tmem_relinquish();
   }
   if (tid == 0) {
-    mbar_init(&bars[kBarLoad0], 1);
-    mbar_init(&bars[kBarLoad1], 1);
-    mbar_init(&bars[kBarS], 1);
-    mbar_init(&bars[kBarYo], 1);
+    for (int k = 0; k < 2; ++k) {
+      mbar_init(&bars[kBarX0 + k], 1);
+      mbar_init(&bars[kBarXfree0 + k], kComputeWarps);
+      mbar_init(&bars[kBarS0 + k], 1);
+      mbar_init(&bars[kBarP0 + k], kComputeWarps);
+    }
+    for (int k = 0; k < kRing; ++k) {
+      mbar_init(&bars[kBarRing0 + k], 1);
+      mbar_init(&bars[kBarRingFree0 + k], 1);
+    }
     mbar_init(&bars[kBarSt], 1);
     mbar_init(&bars[kBarY], 1);
+    mbar_init(&bars[kBarU], kComputeWarps);
     mbar_init(&bars[kBarHt], kComputeWarps);
-    mbar_init(&bars[kBarXw], kComputeWarps);
-    mbar_init(&bars[kBarP], kComputeWarps);
     mbar_init(&bars[kBarFree], kComputeWarps);
-    mbar_init(&bars[kBarXfree], kComputeWarps);
-    for (int k = 0; k < kHelperWarps * kDtStages; ++k) mbar_init(&bars[kBarDt0 + k], 1);
+    mbar_init(&bars[kBarDrain], 1);
+    for (int k = 0; k < kDtStages; ++k) mbar_init(&bars[kBarDt0 + k], 1);
     for (int k = 0; k < kDescSlots; ++k) {
-      mbar_init(&bars[kBarDescFull0 + k], kHelperWarps);
-      mbar_init(&bars[kBarDescFree0 + k], kComputeWarps);
+      mbar_init(&bars[kBarDescFull0 + k], 1);
+      mbar_init(&bars[kBarDescFree0 + k], kComputeWarps + 1);
     }
     for (int k = 0; k < kHeads * 4; ++k) mbar_init(&bars[kBarPair0 + k], 1);
     *abort_flag = 0;
@@ -999,11 +1022,14 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = s_tmem_base;
 
-  if (warp == kIssuerWarp) {
-    if ((tid & 31) == 0) issuer_loop<NS>(&tm_x, &tm_b, &tm_c, pb, smem, tmem, bars, abort_flag);
-    __syncwarp();  // the issuer warp reconverges before the CTA-wide barrier
-  } else if (warp >= kHelperWarp) {
-    helper_loop<NS>(&tm_dt, pb, smem, bars, abort_flag, warp - kHelperWarp);
+  if (warp == kMmaWarp) {
+    if ((tid & 31) == 0) mma_loop<NS>(pb, smem, tmem, bars, abort_flag);
+    __syncwarp();  // the warp reconverges before the CTA-wide barrier
+  } else if (warp == kLoadWarp) {
+    if ((tid & 31) == 0) load_loop<NS>(&tm_x, &tm_b, &tm_c, pb, smem, bars, abort_flag);
+    __syncwarp();
+  } else if (warp == kHelperWarp) {
+    helper_loop<NS>(&tm_dt, pb, smem, bars, abort_flag);
     __syncwarp();
   } else {
     compute_loop<NS>(&tm_y32, pb, smem, tmem, bars, abort_flag);
@@ -1021,7 +1047,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ----------------------------------------------------------------- host side
-PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+}  // namespace
+
+PFN_cuTensorMapEncodeTiled_v12000 tensor_map_encoder() {
   static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
   if (!fn) {
     void* p = nullptr;
@@ -1032,6 +1060,10 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   }
   return fn;
 }
+
+namespace {
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() { return tensor_map_encoder(); }
 
 // 3-D bf16 map {inner, mid, tokens} with a {64, 1, rows} box and 128-byte swizzle.
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t tokens,
@@ -1060,16 +1092,33 @@ bool make_dt_map(CUtensorMap* m, const float* dt, uint64_t H, uint64_t tokens) {
             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// The kernel's shared-memory size is set once per device and kernel instance.
+template <int NS>
+cudaError_t set_smem_attribute() {
+  static std::atomic<uint64_t> done{0};  // bit d: set on device d
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
+  if (bit && (done.load() & bit)) return cudaSuccess;
+  e = cudaFuncSetAttribute(ssd_fused_tc_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDynSmem<NS>);
+  if (e == cudaSuccess && bit) done.fetch_or(bit);
+  return e;
+}
+
 template <int NS>
 cudaError_t launch_ns(const Problem& pb, cudaStream_t st) {
   CUtensorMap mx, mb, mc, my, mdt;
   const uint64_t tokens = (uint64_t)pb.tokens;
-  if (!make_map(&mx, pb.x, kHeadDim, pb.H, tokens) || !make_map(&mb, pb.B, NS, pb.G, tokens) ||
-      !make_map(&mc, pb.C, NS, pb.G, tokens) || !make_map(&my, pb.y, kHeadDim, pb.H, tokens, 32) ||
+  // B and C: boxes of 64 state columns; past N the box reads zeros (N < NS).  Without y
+  // (final states only) C and y are not read and their maps stand in as copies.
+  const bool state_only = pb.y == nullptr;
+  if (!make_map(&mx, pb.x, kHeadDim, pb.H, tokens) || !make_map(&mb, pb.B, pb.N, pb.G, tokens) ||
+      (!state_only && (!make_map(&mc, pb.C, pb.N, pb.G, tokens) || !make_map(&my, pb.y, kHeadDim, pb.H, tokens, 32))) ||
       !make_dt_map(&mdt, pb.dt, pb.H, tokens))
     return cudaErrorInvalidValue;
-  cudaError_t e = cudaFuncSetAttribute(ssd_fused_tc_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       (int)kDynSmem<NS>);
+  if (state_only) mc = mb, my = mx;
+  cudaError_t e = set_smem_attribute<NS>();
   if (e != cudaSuccess) {
     if (getenv("SSD_DEBUG")) fprintf(stderr, "ssd: smem attribute failed: %s\n", cudaGetErrorString(e));
     return e;
@@ -1079,8 +1128,6 @@ cudaError_t launch_ns(const Problem& pb, cudaStream_t st) {
   // ranges may be empty when there are fewer tiles than SMs.
   const int grid = pb.ranges;
   if (grid <= 0) return cudaSuccess;
-  e = cudaMemsetAsync(pb.carry_flag, 0, sizeof(int32_t) * (size_t)grid, st);
-  if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
@@ -1105,17 +1152,18 @@ cudaError_t launch_ns(const Problem& pb, cudaStream_t st) {
 }  // namespace
 
 bool tc_supports(const ssd_shape* s, int chunk) {
+  (void)chunk;  // the tiles are 128 tokens whatever the chunk length; results do not depend on it
   if (!s || s->io_dtype != SSD_BF16 || s->headdim != kHeadDim) return false;
-  if (s->dstate != 64 && s->dstate != 128) return false;
+  // N up to 128 in steps of 8 (16-byte rows of B and C), run as 64 or 128 with zero columns
+  if (s->dstate > 128 || s->dstate % 8) return false;
   if (s->nheads % kHeads || (s->nheads / s->ngroups) % kHeads) return false;  // head pairs share a group
   if (s->nheads % 4) return false;  // dt rows of 4 heads (16 bytes) per TMA box
-  if (chunk != 128 && chunk != 256) return false;
   const int64_t tokens = s->batch * s->seqlen;
   return tokens >= 1 && tokens < ((int64_t)1 << 31) - kTile;
 }
 
 cudaError_t launch_tc(const Problem& pb, cudaStream_t st) {
-  return pb.N == 128 ? launch_ns<128>(pb, st) : launch_ns<64>(pb, st);
+  return pb.N > 64 ? launch_ns<128>(pb, st) : launch_ns<64>(pb, st);
 }
 
 }  // namespace ssd

@@ -5,16 +5,20 @@ The state passes from segment to segment as it passes from chunk to chunk in the
 chunked algorithm ("Transformers are SSMs", the wikillm.com card, Method step 5: the
 centre factor).  Each rank
 
-1. runs its segment from a zero state: end state s_r (H, P, N) and segment log-decay
-   lambda_r[h] = A[h] * sum_t dt[t, h] (two library kernels);
+1. computes only its segment's end state from a zero state, s_r (H, P, N), with the
+   final-state-only form of the forward pass (it reads x, dt and B, not C, and writes no
+   y), and the segment log-decay lambda_r[h] = A[h] * sum_t dt[t, h];
 2. all-gathers (s, lambda) over the process group: H*P*N + H fp32 per rank, the only
    exchange;
 3. forms its start state h_r by the recurrence h_{q+1} = exp(lambda_q) h_q + s_q over the
    preceding segments, from h_0 = init (a library kernel);
-4. runs its segment again from h_r: its y rows and, on the last rank, the final state.
+4. runs its segment from h_r: its y rows and, on the last rank, the final state.
+
+Step 1 reads the segment's x a first time; nothing else of it is repeated, so a rank
+moves about 1.5 times the bytes of one pass (x is about half of them) instead of 2.
 
 The steps are passed in as callables so that the same exchange and ordering can run
-with other implementations of the three kernels; by default they are this package's.
+with other implementations of the kernels; by default they are this package's.
 """
 from __future__ import annotations
 
@@ -25,9 +29,11 @@ import torch.distributed as dist
 
 
 def _library_steps():
-    from . import segment_logdecay, ssd_forward, state_prefix
+    from . import segment_logdecay, ssd_final_state, ssd_forward, state_prefix
 
     def forward(x, dt, A, B, C, D, init, chunk):
+        if C is None:  # only the end state is wanted
+            return None, ssd_final_state(x, dt, A, B, init, None, chunk)
         return ssd_forward(x, dt, A, B, C, D, init, None, chunk)
 
     return forward, segment_logdecay, state_prefix
@@ -41,14 +47,15 @@ def forward_sequence_parallel(x, dt, A, B, C, D=None, init_state=None, chunk: in
     this segment (on the last rank, the sequence's final state).
 
     ``steps`` = (forward, logdecay, prefix) replaces the library kernels:
-    forward(x, dt, A, B, C, D, init, chunk) -> (y, final); logdecay(dt2d, A) -> (H,);
+    forward(x, dt, A, B, C, D, init, chunk) -> (y, final), where C = None asks for the final
+    state only (y may then be None); logdecay(dt2d, A) -> (H,);
     prefix(rank, states, logdecays, init) -> (H, P, N)."""
     forward, logdecay, prefix = steps or _library_steps()
     rank = dist.get_rank(group)
     world = dist.get_world_size(group)
     H = x.shape[2]
-    # 1. this segment from a zero state
-    _, s_r = forward(x, dt, A, B, C, None, None, chunk)
+    # 1. this segment's end state from a zero state (no C, no y)
+    _, s_r = forward(x, dt, A, B, None, None, None, chunk)
     lam_r = logdecay(dt.reshape(-1, H), A)
     # 2. one exchange: every rank's (end state, log-decay)
     states = [torch.empty_like(s_r) for _ in range(world)]

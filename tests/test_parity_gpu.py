@@ -1,6 +1,6 @@
 """GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the same
 seeded inputs, at sizes the oracle finishes in seconds (several chunks and a ragged
-tail) and at the five full-size workloads on sampled (sequence, head) pairs."""
+tail) and at the five full-size workloads on every (sequence, head) pair."""
 import numpy as np
 import pytest
 import torch
@@ -8,7 +8,7 @@ import torch
 import oracle
 import ssd_sequence_mixing_b200 as ssd
 import workloads
-from harness import assert_close, check, run, sample_pairs, to_device
+from harness import assert_close, check, check_every_pair, run, sample_pairs, to_device
 
 pytestmark = pytest.mark.gpu
 
@@ -74,6 +74,49 @@ def test_small_packed_with_resets(dtype):
     for name, path in paths_for(prob, 128):
         y, fin = run(prob, path=path)
         check(prob, y, fin)
+
+
+@pytest.mark.parametrize("lengths", [[8192], [300, 12000, 5]], ids=["one_long", "long_between_short"])
+def test_packed_long_sequence_hands_state_between_ctas(lengths):
+    """A packed sequence far longer than one CTA's share of the tiles: its tiles are cut
+    across many CTAs, each waiting for the state the one before it hands on."""
+    wl = workloads.custom(1, 0, H=4, P=64, N=128, G=1, chunk=256, dtype="bf16", init=True, lengths=lengths)
+    prob = workloads.generate(wl, seed=15, lengths=lengths)
+    for name, path in paths_for(prob, 256):
+        y, fin = run(prob, path=path)
+        check(prob, y, fin)
+
+
+@pytest.mark.parametrize("case", [(1, 20000, 4, 128), (3, 9000, 8, 64), (2, 4097, 2 * 4, 128)],
+                         ids=["b1_T20000_H4", "b3_T9000_H8_N64", "b2_T4097_H8"])
+def test_dense_long_sequences_in_segments(case):
+    """Dense batches whose units are much longer than one CTA's share: the library cuts the
+    sequences into segments (a final-state-only pass, the segments' start states, the full
+    pass); every y row and final state must match the single-pass oracle."""
+    b, T, H, N = case
+    wl = workloads.custom(b, T, H=H, P=64, N=N, G=1, chunk=256, dtype="bf16", init=True)
+    prob = workloads.generate(wl, seed=16)
+    y, fin = run(prob)
+    check(prob, y, fin)
+
+
+def test_final_state_only_matches_full_pass():
+    """y = NULL: only the final states, without reading C or D; equal to the full pass's."""
+    wl = workloads.custom(3, 700, H=8, P=64, N=128, G=2, chunk=256, dtype="bf16", init=True)
+    prob = workloads.generate(wl, seed=17)
+    dev = to_device(prob)
+    for name, path in paths_for(prob, 256):
+        old = ssd.set_path(path)
+        try:
+            _, fin = ssd.ssd_forward(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init_state"],
+                                     None, 256)
+            fin_only = ssd.ssd_final_state(dev["x"], dev["dt"], dev["A"], dev["B"], dev["init_state"], None, 256)
+        finally:
+            ssd.set_path(old)
+        torch.cuda.synchronize()
+        assert torch.equal(fin, fin_only), name
+        _, f_ref = oracle.ssd_forward_problem(prob)
+        assert_close("final_state", fin_only.cpu().numpy(), f_ref, "bf16")
 
 
 def test_packed_many_sequences_grouped():
@@ -206,14 +249,13 @@ FULL = [workloads.TINY, workloads.MAMBA2_2P7B] + workloads.STATE_SWEEP + workloa
 
 
 @pytest.mark.parametrize("wl", FULL, ids=lambda w: w.name)
-def test_full_size_sampled(wl):
+def test_full_size_every_pair(wl):
     """Full-size inputs in the launch configuration the bench times (auto path), checked
-    on sampled (sequence, head) pairs against the oracle."""
+    against the oracle on every (sequence, head) pair: every output element of y and of
+    the final states, including the tiles where CTAs hand the state on."""
     prob = workloads.generate(wl, seed=0)
     y, fin = run(prob)
-    pairs = sample_pairs(prob, k=6)
-    check(prob, y, fin, pairs=pairs)
-    assert torch.isfinite(y.float()).all()
+    check_every_pair(prob, y, fin)
 
 
 # ------------------------------------------------------------------ edge cases

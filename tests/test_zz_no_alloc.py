@@ -16,7 +16,7 @@ import torch
 
 import ssd_sequence_mixing_b200 as ssd
 import workloads
-from harness import TOL, errors, to_device
+from harness import TOL, check, errors, to_device
 
 
 def _call_raw(dev, wl, y, fin):
@@ -57,6 +57,28 @@ def test_noalloc_matches_forward_on_two_calls_in_a_row():
         for name, got, ref in (("y", y, y_ref), ("final_state", fin, f_ref)):
             ok, rel, mx = _within(got, ref, wl.dtype)
             assert ok, f"{wl.name} {name}: rel-L2 {rel:.3e}, max-abs {mx:.3e}"
+        check(prob, y, fin)  # and against the fp64 oracle directly
+
+
+@pytest.mark.gpu
+def test_noalloc_all_sequences_empty_takes_null_inputs():
+    """No tokens at all: x, dt, B, C and y may be NULL, as for ssd_forward, and every
+    final state is its initial state."""
+    lens = [0, 0, 0]
+    wl = workloads.custom(1, 0, H=4, P=64, N=64, G=1, chunk=128, dtype="bf16", init=True, lengths=lens)
+    prob = workloads.generate(wl, seed=13, lengths=lens)
+    dev = to_device(prob)
+    shape = ssd.make_shape(dev["x"], dev["B"], dev["cu_seqlens"])
+    fin = torch.full_like(dev["init_state"], float("nan"))
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    stream = ctypes.c_void_p(torch.cuda.current_stream().cuda_stream)
+    rc = ssd.library().ssd_forward_noalloc(ctypes.byref(shape), None, None, p(dev["A"]), None, None, p(dev["D"]),
+                                           p(dev["init_state"]), p(dev["cu_seqlens"]), wl.chunk, None, p(fin),
+                                           stream)
+    assert rc == 0
+    torch.cuda.synchronize()
+    assert ssd.query_status() == 0
+    assert torch.equal(fin, dev["init_state"])
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch():
