@@ -558,6 +558,92 @@ def block_measurements(dev, stream, flush):
             "gated_rmsnorm": line("gated_rmsnorm_tokens16384_dim5120_bf16", t_norm, norm_bytes)}
 
 
+# ------------------------------------------------------ single-kernel targets for ncu
+PROFILE_TARGETS = ("fused", "fused_n64", "fused_n256", "segments", "final_state", "simt", "packed", "decode",
+                   "conv", "norm", "seqpar")
+
+
+def profile_target(name: str, launches: int = 3):
+    """Launch one entry point ``launches`` times on the bench's shapes (seeded inputs, L2
+    flushed between launches) and nothing else, for one-kernel ncu captures:
+
+    fused       ssd_forward, the Mamba-2-2.7B layer (the fused tensor-core kernel)
+    fused_n64   ssd_forward, the state-size sweep at N = 64
+    fused_n256  ssd_forward, the state-size sweep at N = 256 (two launches on column halves)
+    segments    ssd_forward, the (2, 65536) length-sweep point (cut into segments)
+    final_state ssd_forward with y = NULL on the layer workload
+    simt        ssd_forward on the SIMT path, the layer workload
+    packed      ssd_forward, the packed G = 8 workload (chunk-table kernel + fused kernel)
+    decode      ssd_decode_step, 64 sequences at the layer shape
+    conv        ssd_causal_conv1d_silu, batch 8 x 2048 x 5376 channels
+    norm        ssd_gated_rmsnorm, 16384 tokens x 5120 features
+    seqpar      ssd_segment_logdecay and ssd_state_prefix at the layer shape
+    """
+    import ssd_sequence_mixing_b200 as ssd
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
+    wl = {"fused": WORKLOAD, "fused_n64": workloads.STATE_SWEEP[2], "fused_n256": workloads.STATE_SWEEP[4],
+          "segments": workloads.LENGTH_SWEEP[4], "final_state": WORKLOAD, "simt": WORKLOAD,
+          "packed": workloads.PACKED}.get(name)
+    if wl is not None:
+        prob = workloads.generate(wl, seed=0)
+        d = {k: (None if getattr(prob, k) is None else getattr(prob, k).to(dev))
+             for k in ("x", "dt", "A", "B", "C", "D", "init_state", "cu_seqlens")}
+        if name == "simt":
+            ssd.set_path(ssd.PATH_SIMT)
+        for _ in range(launches):
+            flush.zero_()
+            if name == "final_state":
+                ssd.ssd_final_state(d["x"], d["dt"], d["A"], d["B"], d["init_state"], d["cu_seqlens"], wl.chunk,
+                                    stream=stream)
+            else:
+                ssd.ssd_forward(d["x"], d["dt"], d["A"], d["B"], d["C"], d["D"], d["init_state"], d["cu_seqlens"],
+                                wl.chunk, stream=stream)
+    elif name == "decode":
+        prob = workloads.generate(DECODE, seed=0)
+        x, dt, B, C = (getattr(prob, k)[:, 0].contiguous().to(dev) for k in ("x", "dt", "B", "C"))
+        A, D, state = prob.A.to(dev), prob.D.to(dev), prob.init_state.to(dev)
+        for _ in range(launches):
+            flush.zero_()
+            ssd.ssd_decode_step(x, dt, A, B, C, D, state, stream=stream)
+    elif name in ("conv", "norm"):
+        g = torch.Generator(device=dev).manual_seed(0)
+        if name == "conv":
+            ch = 5120 + 2 * 128
+            xbc = torch.randn((8, 2048, ch), generator=g, device=dev).to(torch.bfloat16)
+            w, b = torch.randn((ch, 4), generator=g, device=dev) * 0.5, torch.randn((ch,), generator=g, device=dev)
+            out = torch.empty_like(xbc)
+            for _ in range(launches):
+                flush.zero_()
+                ssd.causal_conv1d_silu(xbc, w, b, out=out, stream=stream)
+        else:
+            y = torch.randn((16384, 5120), generator=g, device=dev).to(torch.bfloat16)
+            z = torch.randn((16384, 5120), generator=g, device=dev).to(torch.bfloat16)
+            wn = 1.0 + 0.1 * torch.randn((5120,), generator=g, device=dev)
+            o = torch.empty_like(y)
+            for _ in range(launches):
+                flush.zero_()
+                ssd.gated_rmsnorm(y, z, wn, out=o, stream=stream)
+    elif name == "seqpar":
+        prob = workloads.generate(WORKLOAD, seed=0)
+        dt, A = prob.dt[0].contiguous().to(dev), prob.A.to(dev)
+        H, P, N = WORKLOAD.nheads, WORKLOAD.headdim, WORKLOAD.dstate
+        states = torch.randn((8, H, P, N), device=dev) * 0.1
+        lams = -torch.rand((8, H), device=dev)
+        for _ in range(launches):
+            flush.zero_()
+            ssd.segment_logdecay(dt, A)
+            ssd.state_prefix(7, states, lams, None)
+    else:
+        raise SystemExit(f"unknown target {name}; one of {PROFILE_TARGETS}")
+    torch.cuda.synchronize()
+    assert ssd.query_status() == 0
+    print(f"profile target {name}: {launches} launches done", flush=True)
+
+
 # ------------------------------------------------------------ reference arm
 def run_reference(args):
     """The fp64 CPU oracle on this workload: each step is a bounded sample (one sequence x
@@ -599,6 +685,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-decode", action="store_true",
                     help="skip the measurements of the decode step and the block steps around the SSD")
+    ap.add_argument("--profile-target", choices=PROFILE_TARGETS, default=None,
+                    help="only launch one entry point a few times (for one-kernel ncu captures) and exit")
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the per-workload measurements (state-size and length sweeps, packed batch)")
     ap.add_argument("--cpu-budget", type=float, default=10.0)
@@ -606,6 +694,10 @@ def main():
     args = ap.parse_args()
     if args.warmup < 3:
         ap.error("--warmup must be >= 3")
+
+    if args.profile_target:
+        profile_target(args.profile_target)
+        return
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

@@ -213,6 +213,8 @@ int segments_for(const ssd_shape* s, int path, const int32_t* cu, const ssd_dt_p
   const double share = (double)(units * tiles) / device_sms();  // tiles per CTA
   if (tiles <= 1.5 * share) return 1;
   int64_t k = (int64_t)((tiles + share - 1) / share);
+  const int64_t seg_tiles = (tiles + k - 1) / k;  // segments are whole tiles
+  k = (tiles + seg_tiles - 1) / seg_tiles;
   if (k < 2) return 1;
   if (s->batch * k > (1 << 20)) return 1;
   return (int)k;

@@ -428,18 +428,20 @@ extern "C" int ssd_gated_rmsnorm(int64_t tokens, int64_t dim, ssd_dtype io_dtype
   const int row = (int)(dim * (io_dtype == SSD_BF16 ? 2 : 4));
   // up to 4 tokens in flight per CTA within about 100 KB, at least 2
   a.stages = std::max(2, std::min(ssd::kNormMaxStages, (100 << 10) / (2 * row)));
-  const int smem = a.stages * 2 * row;
+  const int smem = a.stages * 2 * row;  // at most 2 x 2 x 32 KB (dim 8192, fp32)
   const int per_sm = std::max(1, std::min(4, (220 << 10) / (smem + 2048)));
   const int64_t grid = std::min<int64_t>(tokens, (int64_t)per_sm * ssd::device_sms());
   cudaStream_t st = (cudaStream_t)stream;
   static std::atomic<uint64_t> done_bf{0}, done_f{0};
   cudaError_t e;
+  // the attribute is raised once to the largest size any call of this kernel takes
+  constexpr int kNormSmemMax = 2 * 2 * 8192 * 4;
   if (io_dtype == SSD_BF16) {
-    e = ssd::allow_smem(ssd::gated_rmsnorm_kernel<__nv_bfloat16>, smem, done_bf);
+    e = ssd::allow_smem(ssd::gated_rmsnorm_kernel<__nv_bfloat16>, kNormSmemMax, done_bf);
     if (e == cudaSuccess)
       ssd::gated_rmsnorm_kernel<__nv_bfloat16><<<(unsigned)grid, ssd::kNormThreads, smem, st>>>(a);
   } else {
-    e = ssd::allow_smem(ssd::gated_rmsnorm_kernel<float>, smem, done_f);
+    e = ssd::allow_smem(ssd::gated_rmsnorm_kernel<float>, kNormSmemMax, done_f);
     if (e == cudaSuccess) ssd::gated_rmsnorm_kernel<float><<<(unsigned)grid, ssd::kNormThreads, smem, st>>>(a);
   }
   ssd::count_launches(1);

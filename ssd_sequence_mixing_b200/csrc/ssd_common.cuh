@@ -52,6 +52,9 @@ struct Problem {
   int ranges;            // CTAs of the tensor-core launch
   long long wait_limit;  // SM cycles a device-side wait may take before it gives up
   int withhold_carry;    // test hook: CTAs never publish the state they hand on
+  // tensor-core launches on a column range of a wider state: this launch's state columns
+  // are [n_off, n_off + N) of rows n_stride long, and y_accum adds its y to the y in memory
+  int n_off, n_stride, y_accum;
   // host-side measurement hooks (events around the dominant kernel, or null)
   cudaEvent_t prof_start, prof_stop;
   // fused dt prologue (ssd_forward_dt): dt holds the raw values, see dt_value()

@@ -80,7 +80,7 @@ enum {
   kBarRingFree0 = kBarRing0 + kRing,  // kRing: ring slot free (one UMMA commit)
   kBarS0 = kBarRingFree0 + kRing,     // 2: S = C B^T in S/P buffer b (commit)
   kBarP0 = kBarS0 + 2,                // 2: P written in buffer b (16 arrivals)
-  kBarSt,                             // right factor accumulated onto H (commit)
+  kBarSt = kBarP0 + 2,                // right factor accumulated onto H (commit)
   kBarY,                              // P U accumulated into Y (commit)
   kBarU,                              // U written (16)
   kBarHt,                             // h^ written, bf16 in shared and fp32 in H (16)
@@ -93,6 +93,12 @@ enum {
   kNumBars = kBarPair0 + kHeads * 4
 };
 static_assert(kNumBars <= 64, "phase bits of a 64-bit mask");
+// every group of barriers has its own slots: the next group starts past its last one
+static_assert(kBarXfree0 == kBarX0 + 2 && kBarRing0 == kBarXfree0 + 2 && kBarRingFree0 == kBarRing0 + kRing &&
+                  kBarS0 == kBarRingFree0 + kRing && kBarP0 == kBarS0 + 2 && kBarSt == kBarP0 + 2 &&
+                  kBarDescFull0 == kBarDt0 + kDtStages && kBarDescFree0 == kBarDescFull0 + kDescSlots &&
+                  kBarPair0 == kBarDescFree0 + kDescSlots,
+              "barrier slots");
 
 // Pass descriptor flags
 enum {
@@ -492,15 +498,18 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
 
   // Units whose sequences are empty have no tiles: CTA r writes final = init for the
   // empty units u with u % R == r.
-  const int N = pb.N;  // state size (NS, the operand width, is N rounded up; columns past N are 0)
+  // State size of this launch (NS, the operand width, is N rounded up; columns past N are
+  // 0).  In memory, state row (s, h, p) is NR = n_stride long and this launch owns its
+  // columns [n_off, n_off + N).
+  const int N = pb.N, NR = pb.n_stride;
   if (pb.final_state && i < N) {
     for (int u = blockIdx.x; u < units; u += gridDim.x) {
       if (unit_tiles(pb, u) != 0) continue;
       const int s = u / pairs;
       const int h = (u % pairs) * kHeads + hw;
-      const int64_t base = ((int64_t)s * pb.H + h) * kHeadDim * N;
+      const int64_t base = ((int64_t)s * pb.H + h) * kHeadDim * NR + pb.n_off;
       for (int p = 32 * ch; p < 32 * ch + 32; ++p)
-        pb.final_state[base + (int64_t)p * N + i] = pb.init ? pb.init[base + (int64_t)p * N + i] : 0.f;
+        pb.final_state[base + (int64_t)p * NR + i] = pb.init ? pb.init[base + (int64_t)p * NR + i] : 0.f;
     }
   }
 
@@ -537,6 +546,7 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
   // warp waits for the matching warp of that CTA).  False if that wait gave up.
   auto load_state = [&](const PassDesc& d, uint32_t (&r)[32]) -> bool {
     const float* src_p = nullptr;
+    int rs = NR;  // row stride of the source
     if (d.flags & kPCarryIn) {
       const int src = d.carry_src;
       bool mine = true;
@@ -554,12 +564,13 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
       if (__any_sync(0xffffffffu, !mine)) return false;
       __threadfence();
       src_p = pb.carry + ((size_t)src * kHeads + hw) * kHeadDim * N + i;
+      rs = N;
     } else if (pb.init) {
-      src_p = pb.init + ((int64_t)d.s * pb.H + d.h0 + hw) * kHeadDim * N + i;
+      src_p = pb.init + ((int64_t)d.s * pb.H + d.h0 + hw) * kHeadDim * NR + pb.n_off + i;
     }
 #pragma unroll
     for (int k = 0; k < 32; ++k)
-      r[k] = __float_as_uint((src_p && i < N) ? __ldcg(src_p + (size_t)(32 * ch + k) * N) : 0.f);
+      r[k] = __float_as_uint((src_p && i < N) ? __ldcg(src_p + (size_t)(32 * ch + k) * rs) : 0.f);
     return true;
   };
 
@@ -663,12 +674,13 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
       tmem_ld_wait();
       if (flags & (kPToFinal | kPToCarry)) {
         const float so = d.sig_out[hw];
-        float* dst = (flags & kPToFinal)
-                         ? pb.final_state + ((int64_t)d.s * pb.H + d.h0 + hw) * kHeadDim * N + i
-                         : pb.carry + ((size_t)blockIdx.x * kHeads + hw) * kHeadDim * N + i;
+        const bool to_final = flags & kPToFinal;
+        float* dst = to_final ? pb.final_state + ((int64_t)d.s * pb.H + d.h0 + hw) * kHeadDim * NR + pb.n_off + i
+                              : pb.carry + ((size_t)blockIdx.x * kHeads + hw) * kHeadDim * N + i;
+        const int ds_ = to_final ? NR : N;
         if (i < N) {
 #pragma unroll
-          for (int k = 0; k < 32; ++k) dst[(size_t)(32 * ch + k) * N] = so * __uint_as_float(r[k]);
+          for (int k = 0; k < 32; ++k) dst[(size_t)(32 * ch + k) * ds_] = so * __uint_as_float(r[k]);
         }
         if (flags & kPToCarry) {  // this warp's part is out: one release per warp
           __threadfence();
@@ -720,14 +732,20 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
       tmem_ld_wait();
       const bool row_ok = !staged && i >= d.lo && i < d.hi && i < d.rem;
       __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(pb.y) + ((int64_t)(d.t0 + i) * pb.H + h) * kHeadDim;
+      const bool add_prev = pb.y_accum && i >= d.lo && i < d.hi && i < d.rem;  // y of the other state columns
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t out[4];
+        uint4 prev = make_uint4(0u, 0u, 0u, 0u);
+        if (add_prev) prev = *reinterpret_cast<const uint4*>(yrow + 32 * ch + 8 * c);
+        const uint32_t pv[4] = {prev.x, prev.y, prev.z, prev.w};
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {  // bf16 pair -> fp32 pair (exact), then r Y + D x
+        for (int k = 0; k < 4; ++k) {  // bf16 pair -> fp32 pair (exact), then r Y + D x (+ y so far)
           const uint32_t xu = xr[4 * c + k];
           const uint64_t x2 = f2u(xu << 16, xu & 0xFFFF0000u);
-          out[k] = bf16x2_of(fma2(r2, f2u(ry[8 * c + 2 * k], ry[8 * c + 2 * k + 1]), mul2(d2, x2)));
+          uint64_t acc = fma2(r2, f2u(ry[8 * c + 2 * k], ry[8 * c + 2 * k + 1]), mul2(d2, x2));
+          if (pb.y_accum) acc = add2(acc, f2u(pv[k] << 16, pv[k] & 0xFFFF0000u));
+          out[k] = bf16x2_of(acc);
         }
         const uint4 ov = make_uint4(out[0], out[1], out[2], out[3]);
         if (staged)
@@ -1065,13 +1083,15 @@ namespace {
 
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() { return tensor_map_encoder(); }
 
-// 3-D bf16 map {inner, mid, tokens} with a {64, 1, rows} box and 128-byte swizzle.
+// 3-D bf16 map {inner, mid, tokens} with a {64, 1, rows} box and 128-byte swizzle; rows of
+// the innermost dimension are `pitch` elements apart (default: inner).
 bool make_map(CUtensorMap* m, const void* base, uint64_t inner, uint64_t mid, uint64_t tokens,
-              uint32_t rows = kTile) {
+              uint32_t rows = kTile, uint64_t pitch = 0) {
   auto fn = encode_fn();
   if (!fn) return false;
+  if (!pitch) pitch = inner;
   cuuint64_t dims[3] = {inner, mid, tokens};
-  cuuint64_t strides[2] = {inner * 2, inner * mid * 2};
+  cuuint64_t strides[2] = {pitch * 2, pitch * mid * 2};
   cuuint32_t box[3] = {64, 1, rows};
   cuuint32_t estr[3] = {1, 1, 1};
   return fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides, box, estr,
@@ -1113,8 +1133,11 @@ cudaError_t launch_ns(const Problem& pb, cudaStream_t st) {
   // B and C: boxes of 64 state columns; past N the box reads zeros (N < NS).  Without y
   // (final states only) C and y are not read and their maps stand in as copies.
   const bool state_only = pb.y == nullptr;
-  if (!make_map(&mx, pb.x, kHeadDim, pb.H, tokens) || !make_map(&mb, pb.B, pb.N, pb.G, tokens) ||
-      (!state_only && (!make_map(&mc, pb.C, pb.N, pb.G, tokens) || !make_map(&my, pb.y, kHeadDim, pb.H, tokens, 32))) ||
+  const __nv_bfloat16* b0 = static_cast<const __nv_bfloat16*>(pb.B) + pb.n_off;
+  const __nv_bfloat16* c0 = static_cast<const __nv_bfloat16*>(pb.C) + pb.n_off;
+  if (!make_map(&mx, pb.x, kHeadDim, pb.H, tokens) || !make_map(&mb, b0, pb.N, pb.G, tokens, kTile, pb.n_stride) ||
+      (!state_only && (!make_map(&mc, c0, pb.N, pb.G, tokens, kTile, pb.n_stride) ||
+                       !make_map(&my, pb.y, kHeadDim, pb.H, tokens, 32))) ||
       !make_dt_map(&mdt, pb.dt, pb.H, tokens))
     return cudaErrorInvalidValue;
   if (state_only) mc = mb, my = mx;
@@ -1154,8 +1177,9 @@ cudaError_t launch_ns(const Problem& pb, cudaStream_t st) {
 bool tc_supports(const ssd_shape* s, int chunk) {
   (void)chunk;  // the tiles are 128 tokens whatever the chunk length; results do not depend on it
   if (!s || s->io_dtype != SSD_BF16 || s->headdim != kHeadDim) return false;
-  // N up to 128 in steps of 8 (16-byte rows of B and C), run as 64 or 128 with zero columns
-  if (s->dstate > 128 || s->dstate % 8) return false;
+  // N up to 128 in steps of 8 (16-byte rows of B and C), run as 64 or 128 with zero columns;
+  // N = 256 as two launches on its column halves
+  if ((s->dstate > 128 && s->dstate != 256) || s->dstate % 8) return false;
   if (s->nheads % kHeads || (s->nheads / s->ngroups) % kHeads) return false;  // head pairs share a group
   if (s->nheads % 4) return false;  // dt rows of 4 heads (16 bytes) per TMA box
   const int64_t tokens = s->batch * s->seqlen;
@@ -1163,7 +1187,24 @@ bool tc_supports(const ssd_shape* s, int chunk) {
 }
 
 cudaError_t launch_tc(const Problem& pb, cudaStream_t st) {
-  return pb.N > 64 ? launch_ns<128>(pb, st) : launch_ns<64>(pb, st);
+  if (pb.N <= 128) {
+    Problem q = pb;
+    q.n_off = 0, q.n_stride = pb.N, q.y_accum = 0;
+    return pb.N > 64 ? launch_ns<128>(q, st) : launch_ns<64>(q, st);
+  }
+  // N = 256: the state's columns are independent and y is linear in them, so the call is
+  // two launches on the column halves of B, C and the states; the second adds its y to the
+  // first's (and D x only once).  The measurement events span both.
+  Problem a = pb, b = pb;
+  a.N = b.N = 128;
+  a.n_stride = b.n_stride = pb.N;
+  a.n_off = 0, b.n_off = 128;
+  a.y_accum = 0, b.y_accum = pb.y != nullptr;
+  b.D = nullptr;
+  a.prof_stop = nullptr, b.prof_start = nullptr;
+  b.epoch = pb.epoch ^ 0x8000000000000000ull;  // a value no other launch's flags hold
+  cudaError_t e = launch_ns<128>(a, st);
+  return e == cudaSuccess ? launch_ns<128>(b, st) : e;
 }
 
 }  // namespace ssd

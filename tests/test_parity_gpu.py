@@ -53,6 +53,12 @@ SMALL = [
     (1, 8192, 4, 64, 128, 1, 256, "bf16", True),
     (1, 2048, 2, 64, 128, 1, 256, "bf16", True),  # 2 heads: no 4-head dt rows, SIMT path
     (3, 1000, 16, 64, 64, 2, 128, "bf16", True),
+    # state sizes the tensor-core path pads (16, 32, 96) or splits in column halves (256)
+    (2, 700, 4, 64, 16, 1, 256, "bf16", True),
+    (1, 900, 8, 64, 32, 2, 128, "bf16", True),
+    (2, 333, 4, 64, 96, 1, 256, "bf16", True),
+    (2, 700, 4, 64, 256, 1, 256, "bf16", True),
+    (1, 1100, 8, 64, 256, 2, 64, "bf16", False),
 ]
 
 
