@@ -4,6 +4,7 @@
 #include <stdint.h>
 #include <string.h>
 
+#include <algorithm>
 #include <atomic>
 #include <chrono>
 #include <mutex>
@@ -210,13 +211,13 @@ int segments_for(const ssd_shape* s, int path, const int32_t* cu, const ssd_dt_p
   if (path != SSD_PATH_TC || cu || pro || s->batch < 1 || s->seqlen <= 0) return 1;
   const int64_t tiles = (s->seqlen + ssd::kTcTile - 1) / ssd::kTcTile;
   const int64_t units = s->batch * (s->nheads / 2);
-  const double share = (double)(units * tiles) / device_sms();  // tiles per CTA
-  if (tiles <= 1.5 * share) return 1;
-  int64_t k = (int64_t)((tiles + share - 1) / share);
-  const int64_t seg_tiles = (tiles + k - 1) / k;  // segments are whole tiles
-  k = (tiles + seg_tiles - 1) / seg_tiles;
-  if (k < 2) return 1;
-  if (s->batch * k > (1 << 20)) return 1;
+  // tiles per CTA (at least one: with fewer tiles than SMs every CTA takes one)
+  const int64_t share = std::max<int64_t>(1, units * tiles / std::max(1, device_sms()));
+  if (2 * tiles <= 3 * share) return 1;
+  const int64_t k0 = (tiles + share - 1) / share;         // segments of at most one share ...
+  const int64_t seg_tiles = (tiles + k0 - 1) / k0;        // ... of whole tiles
+  const int64_t k = (tiles + seg_tiles - 1) / seg_tiles;
+  if (k < 2 || s->batch * k > (1 << 20)) return 1;
   return (int)k;
 }
 
@@ -230,13 +231,11 @@ int forward_segmented(const ssd_shape* s, int k, const void* x, const float* dt,
   const int64_t H = s->nheads, PN = s->headdim * s->dstate, HPN = H * PN;
   auto up = [](size_t v) { return (v + 255) & ~(size_t)255; };
   const size_t o_cu = 0, o_st = up(sizeof(int32_t) * (nseg + 1)), o_lam = o_st + up(sizeof(float) * nseg * HPN),
-               o_h = o_lam + up(sizeof(float) * nseg * H), o_fin = o_h + up(sizeof(float) * nseg * HPN),
-               total = o_fin + (fin ? up(sizeof(float) * nseg * HPN) : 0);
+               o_h = o_lam + up(sizeof(float) * nseg * H), total = o_h + up(sizeof(float) * nseg * HPN);
   char* ws = nullptr;
   if (pool_alloc((void**)&ws, total, st) != cudaSuccess) return SSD_ERR_CUDA;
   int32_t* cu = (int32_t*)(ws + o_cu);
   float *states = (float*)(ws + o_st), *lam = (float*)(ws + o_lam), *h_in = (float*)(ws + o_h);
-  float* seg_fin = fin ? (float*)(ws + o_fin) : nullptr;
   ssd_shape sg = *s;
   sg.batch = 1;
   sg.seqlen = s->batch * L;
@@ -246,14 +245,12 @@ int forward_segmented(const ssd_shape* s, int k, const void* x, const float* dt,
   if (ssd::launch_segment_offsets(nseq, L, k, seg, cu, st) != cudaSuccess) rc = SSD_ERR_CUDA;
   // 1. every segment's end state from a zero state (x, dt, B only)
   if (rc == SSD_OK) rc = forward_impl(&sg, x, dt, A, B, nullptr, nullptr, nullptr, cu, chunk, nullptr, states, st);
-  // 2. the segments' decays and true start states
+  // 2. the segments' decays, true start states and the sequences' final states
   if (rc == SSD_OK && (ssd::launch_segments_logdecay(cu, nseg, (int)H, dt, A, lam, st) != cudaSuccess ||
-                       ssd::launch_segments_prefix(nseq, k, H, PN, states, lam, init, h_in, st) != cudaSuccess))
+                       ssd::launch_segments_prefix(nseq, k, H, PN, states, lam, init, h_in, fin, st) != cudaSuccess))
     rc = SSD_ERR_CUDA;
-  // 3. the full pass on the segments from their start states
-  if (rc == SSD_OK) rc = forward_impl(&sg, x, dt, A, B, C, D, h_in, cu, chunk, y, seg_fin, st);
-  if (rc == SSD_OK && fin && ssd::launch_segments_final(nseq, k, HPN, seg_fin, fin, st) != cudaSuccess)
-    rc = SSD_ERR_CUDA;
+  // 3. the full pass on the segments from their start states (y only)
+  if (rc == SSD_OK && y) rc = forward_impl(&sg, x, dt, A, B, C, D, h_in, cu, chunk, y, nullptr, st);
   if (cudaFreeAsync(ws, st) != cudaSuccess && rc == SSD_OK) rc = SSD_ERR_CUDA;
   return rc;
 }
@@ -277,7 +274,7 @@ int forward_impl(const ssd_shape* s, const void* x, const float* dt, const float
   if (nseq == 0) return SSD_OK;
   unsigned int* status = status_ptr();
   if (!status) return SSD_ERR_CUDA;
-  if (!state_only) {
+  {
     const int k = segments_for(s, path, cu, pro);
     if (k > 1) return forward_segmented(s, k, x, dt, A, B, C, D, init, chunk, y, fin, st);
   }

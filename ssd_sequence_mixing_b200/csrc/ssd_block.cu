@@ -124,7 +124,9 @@ constexpr int kConvStages = 4;
 template <typename T>
 __global__ void __launch_bounds__(kConvThreads) conv1d_silu_kernel(const __grid_constant__ CUtensorMap tm_in,
                                                                    ConvArgs a) {
-  extern __shared__ __align__(128) uint8_t smem[];
+  extern __shared__ uint8_t smem_raw[];
+  // TMA tile destinations: 128-byte aligned (the launch reserves the slack)
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 127) & ~uintptr_t(127));
   __shared__ uint64_t full[kConvStages], empty[kConvStages];
   __shared__ int64_t seq_start[2][kConvTokens];
   constexpr uint32_t kStage = kConvRows * kConvChannels * sizeof(T);
@@ -393,7 +395,7 @@ extern "C" int ssd_causal_conv1d_silu(int64_t batch, int64_t seqlen, int64_t cha
           dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) != CUDA_SUCCESS)
     return SSD_ERR_CUDA;
-  const int smem = ssd::kConvStages * ssd::kConvRows * ssd::kConvChannels * (int)es;
+  const int smem = ssd::kConvStages * ssd::kConvRows * ssd::kConvChannels * (int)es + 128;
   cudaStream_t st = (cudaStream_t)stream;
   static std::atomic<uint64_t> done_bf{0}, done_f{0};
   cudaError_t e;

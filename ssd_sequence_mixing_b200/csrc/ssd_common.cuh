@@ -111,14 +111,12 @@ cudaError_t launch_chunk_table(const Problem& pb, cudaStream_t st);
 cudaError_t launch_simt(const Problem& pb, cudaStream_t st);
 // Long sequences in segments (ssd_seqpar.cu): segment offsets of a dense batch of nseq
 // sequences of L tokens cut into k segments of `seg` tokens (the last of each shorter);
-// per-segment log-decays; every segment's start state; each sequence's final state from
-// its last segment's.
+// per-segment log-decays; every segment's start state and (fin != null) each sequence's
+// final state, by the recurrence over its segments' zero-start end states.
 cudaError_t launch_segment_offsets(int nseq, int64_t L, int k, int64_t seg, int32_t* cu, cudaStream_t st);
 cudaError_t launch_segments_logdecay(const int32_t* cu, int nseg, int H, const float* dt, const float* A,
                                      float* lam, cudaStream_t st);
 cudaError_t launch_segments_prefix(int nseq, int k, int64_t H, int64_t PN, const float* states, const float* lam,
-                                   const float* init, float* out, cudaStream_t st);
-cudaError_t launch_segments_final(int nseq, int k, int64_t HPN, const float* seg_final, float* fin,
-                                  cudaStream_t st);
+                                   const float* init, float* out, float* fin, cudaStream_t st);
 
 }  // namespace ssd

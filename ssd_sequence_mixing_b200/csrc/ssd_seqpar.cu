@@ -111,10 +111,11 @@ __global__ void __launch_bounds__(kHeadsPerBlock * kTokLanes)
 }
 
 // Start state of every segment: for each sequence s (k segments) and state element e,
-// h[s k] = init[s], h[s k + i + 1] = exp(lam[s k + i]) h[s k + i] + states[s k + i].
+// h[s k] = init[s], h[s k + i + 1] = exp(lam[s k + i]) h[s k + i] + states[s k + i];
+// the last step of the recurrence is the sequence's final state (written when fin != null).
 __global__ void __launch_bounds__(256) segments_prefix_kernel(int nseq, int k, int64_t H, int64_t PN,
                                                               const float* states, const float* lam,
-                                                              const float* init, float* out) {
+                                                              const float* init, float* out, float* fin) {
   const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   const int s = blockIdx.y;
   if (e >= H * PN) return;
@@ -125,14 +126,7 @@ __global__ void __launch_bounds__(256) segments_prefix_kernel(int nseq, int k, i
     out[j * H * PN + e] = acc;
     acc = fmaf(expf(lam[j * H + h]), acc, states[j * H * PN + e]);
   }
-}
-
-// final[s] = the final state of sequence s's last segment.
-__global__ void __launch_bounds__(256) segments_final_kernel(int k, int64_t HPN, const float* seg_final,
-                                                             float* fin) {
-  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
-  const int s = blockIdx.y;
-  if (e < HPN) fin[(int64_t)s * HPN + e] = seg_final[((int64_t)s * k + k - 1) * HPN + e];
+  if (fin) fin[(int64_t)s * H * PN + e] = acc;
 }
 
 }  // namespace
@@ -153,16 +147,9 @@ cudaError_t launch_segments_logdecay(const int32_t* cu, int nseg, int H, const f
 }
 
 cudaError_t launch_segments_prefix(int nseq, int k, int64_t H, int64_t PN, const float* states, const float* lam,
-                                   const float* init, float* out, cudaStream_t st) {
+                                   const float* init, float* out, float* fin, cudaStream_t st) {
   segments_prefix_kernel<<<dim3((unsigned)((H * PN + 255) / 256), nseq), 256, 0, st>>>(nseq, k, H, PN, states,
-                                                                                       lam, init, out);
-  count_launches(1);
-  return cudaGetLastError();
-}
-
-cudaError_t launch_segments_final(int nseq, int k, int64_t HPN, const float* seg_final, float* fin,
-                                  cudaStream_t st) {
-  segments_final_kernel<<<dim3((unsigned)((HPN + 255) / 256), nseq), 256, 0, st>>>(k, HPN, seg_final, fin);
+                                                                                       lam, init, out, fin);
   count_launches(1);
   return cudaGetLastError();
 }

@@ -24,7 +24,7 @@
 //   MMA  H  += B^T [U_0 | U_1]     right factor    (N x 128, K = 128), H holds h^
 //   MMA  Y  += P [U_0 | U_1]       diagonal block  (128 x 128, K = 128, A in tensor memory)
 //   state    h_end = 2^(c_end - m) H  (centre factor: the next tile's h^ is this times
-//            2^(m' - c'_start)), or the final state / hand-on at the end of a piece
+//            2^(m' - c'_start)); at the end of a piece the final state or the hand-on
 //   epilogue y_i = r_i Y_i + D x_i  (bf16, staged over the tile's U, TMA store)
 //
 // The split needs 2^(m - c_j) and 2^(c_i - m) to stay well inside the fp32 / bf16
@@ -669,18 +669,30 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
     const int nds = (p + 1) % kDescSlots;
     bool more;
     {
+      // h_out = sig_out H: the true state after this pass (always formed first, so the
+      // state a CTA hands on and the state it keeps are rounded alike)
       uint32_t r[32];
       tmem_ld32(t_state, r);
       tmem_ld_wait();
-      if (flags & (kPToFinal | kPToCarry)) {
+      {
         const float so = d.sig_out[hw];
+        const uint64_t so2 = f2(so, so);
+#pragma unroll
+        for (int k = 0; k < 16; ++k) {
+          float lo, hi;
+          unf2(mul2(so2, f2u(r[2 * k], r[2 * k + 1])), lo, hi);
+          r[2 * k] = __float_as_uint(lo);
+          r[2 * k + 1] = __float_as_uint(hi);
+        }
+      }
+      if (flags & (kPToFinal | kPToCarry)) {
         const bool to_final = flags & kPToFinal;
         float* dst = to_final ? pb.final_state + ((int64_t)d.s * pb.H + d.h0 + hw) * kHeadDim * NR + pb.n_off + i
                               : pb.carry + ((size_t)blockIdx.x * kHeads + hw) * kHeadDim * N + i;
         const int ds_ = to_final ? NR : N;
         if (i < N) {
 #pragma unroll
-          for (int k = 0; k < 32; ++k) dst[(size_t)(32 * ch + k) * ds_] = so * __uint_as_float(r[k]);
+          for (int k = 0; k < 32; ++k) dst[(size_t)(32 * ch + k) * ds_] = __uint_as_float(r[k]);
         }
         if (flags & kPToCarry) {  // this warp's part is out: one release per warp
           __threadfence();
@@ -694,14 +706,8 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
       const PassDesc& dn = descs[nds];
       more = !(dn.flags & kPEnd);
       if (more) {
-        float sig;
-        if (dn.flags & kPPieceStart) {
-          if (!load_state(dn, r)) return;
-          sig = dn.sig_in[hw];
-        } else {
-          sig = d.sig_out[hw] * dn.sig_in[hw];
-        }
-        write_state(r, sig);
+        if ((dn.flags & kPPieceStart) && !load_state(dn, r)) return;
+        write_state(r, dn.sig_in[hw]);  // h^ of the next pass
       }
     }
     fence_proxy_async();

@@ -106,6 +106,29 @@ def test_dense_long_sequences_in_segments(case):
     check(prob, y, fin)
 
 
+@pytest.mark.parametrize("case", [(4, 1024, 64, 128, 8), (2, 1536, 128, 64, 4)], ids=["H64_G8_N128", "H128_G4_N64"])
+def test_dense_many_tiles_per_cta(case):
+    """Enough heads that no sequence is cut into segments and every CTA runs several tiles
+    in a row (its ring of B/C tiles, both x stages and both S/P buffers in turn) and hands
+    the state on inside units."""
+    b, T, H, N, G = case
+    wl = workloads.custom(b, T, H=H, P=64, N=N, G=G, chunk=256, dtype="bf16", init=True)
+    prob = workloads.generate(wl, seed=18)
+    y, fin = run(prob)
+    check(prob, y, fin)
+
+
+def test_packed_passes_and_hand_ons():
+    """Heads that decay too fast for one pass per tile (A = -1e4 and -60), in packed
+    sequences long enough to be cut across CTAs."""
+    lens = [700, 2500, 64, 1800]
+    wl = workloads.custom(1, 0, H=8, P=64, N=128, G=2, chunk=256, dtype="bf16", init=True, lengths=lens)
+    prob = workloads.generate(wl, seed=19, lengths=lens, A_override=[-1e4, -1.0, -60.0, -2.0, -0.5, -30.0, -8.0, -1e-3])
+    for name, path in paths_for(prob, 256):
+        y, fin = run(prob, path=path)
+        check(prob, y, fin)
+
+
 def test_final_state_only_matches_full_pass():
     """y = NULL: only the final states, without reading C or D; equal to the full pass's."""
     wl = workloads.custom(3, 700, H=8, P=64, N=128, G=2, chunk=256, dtype="bf16", init=True)
@@ -221,7 +244,8 @@ def test_host_entry_point_matches_device():
 @pytest.mark.parametrize("lengths", [None, [700, 0, 1, 300, 129, 2048, 64, 5, 900, 33]], ids=["dense", "packed"])
 def test_host_entry_point_groups_match_device(lengths):
     """The host entry point copies in, computes and copies out by groups of whole sequences;
-    every sequence's outputs equal the single device call's bit for bit."""
+    every sequence's outputs match the oracle and the single device call's (each group is
+    its own launch, so the CTA split, and with it the rounding, may differ)."""
     if lengths is None:
         wl = workloads.custom(6, 500, H=8, P=64, N=128, G=2, chunk=256, dtype="bf16", init=True)
         prob = workloads.generate(wl, seed=11)
@@ -232,7 +256,9 @@ def test_host_entry_point_groups_match_device(lengths):
     pin = lambda t: None if t is None else t.pin_memory()
     yh, fh = ssd.ssd_forward_host(pin(prob.x), pin(prob.dt), pin(prob.A), pin(prob.B), pin(prob.C), pin(prob.D),
                                   pin(prob.init_state), pin(prob.cu_seqlens), chunk=wl.chunk)
-    assert torch.equal(yh, y.cpu()) and torch.equal(fh, fin.cpu())
+    check(prob, yh, fh)
+    assert_close("y vs device call", yh.float().numpy(), y.float().cpu().double().numpy(), "bf16")
+    assert_close("final vs device call", fh.numpy(), fin.cpu().double().numpy(), "bf16")
 
 
 def test_bad_device_seqlens_sets_status_and_writes_nothing():
