@@ -14,23 +14,28 @@
 // dt_j) goes onto x:  U_j = 2^(m - c_j) dt_j x_j, and the row factor into the epilogue.
 // What is left of the masked matrix, P = causal(C B^T), no longer depends on the head:
 // it is computed once per pair, without exponentials, and both heads' diagonal blocks
-// are one N = 128 product P [U_0 | U_1].  The same U feeds the chunk state, and the
-// carried-in state enters scaled as h^ = 2^(m - c_start) h, so that one accumulator
-// holds everything a row needs before its factor r_i:
+// are one N = 128 product P [U_0 | U_1].  The same U feeds the chunk state, which tensor
+// memory holds scaled as H = 2^(m - c_start) h (h^, the state in the reference's scale),
+// so that one accumulator holds everything a row needs before its factor r_i:
 //
 //   MMA  S   = C B^T                               (128 x 128, K = N, once per pair)
 //   mask     P = bf16(S) on and below the diagonal, 0 above (mask before use)
 //   MMA  Y   = C [h^_0 h^_1]^T     left factor     (128 x 128, K = N)
 //   MMA  H  += B^T [U_0 | U_1]     right factor    (N x 128, K = 128), H holds h^
 //   MMA  Y  += P [U_0 | U_1]       diagonal block  (128 x 128, K = 128, A in tensor memory)
-//   state    h_end = 2^(c_end - m) H  (centre factor: the next tile's h^ is this times
-//            2^(m' - c'_start)); at the end of a piece the final state or the hand-on
+//   state    h_end = 2^(c_end - m) H; at the end of a piece the final state or the
+//            hand-on; the bf16 copy of H for the next left factor
 //   epilogue y_i = r_i Y_i + D x_i  (bf16, staged over the tile's U, TMA store)
 //
-// The split needs 2^(m - c_j) and 2^(c_i - m) to stay well inside the fp32 / bf16
-// range: a tile whose decay range over its rows exceeds kRangeMax (log2 units) is
-// processed in several passes over the same loaded data, each over a run of rows
-// whose range fits (on the pages' input distributions, 1 - 3 % of tiles).
+// The reference m carries over from tile to tile: in the next tile's cumsum (restarted
+// at 0) it is m' = m - c_end, so H accumulates the next right factor as it stands and
+// the state step only reads it.  The split needs 2^(m - c_j) and 2^(c_i - m) to stay
+// inside the fp32 / bf16 range: while every row of a tile keeps |m - c_j| <= kRangeHalf
+// (log2 units) the reference stays; otherwise the pass re-centres it (m = the midpoint
+// of its rows' cumsums, H rescaled to match) and, if the tile's rows span more than
+// 2 kRangeHalf, the tile is processed in several passes over the same loaded data,
+// each over a run of rows whose range fits (on the pages' input distributions,
+// 1 - 3 % of tiles).
 //
 // Roles: 16 compute warps (Û, the mask, the state step, the epilogue), one MMA warp
 // (every tcgen05.mma), one load warp (every TMA load of x, B, C) and one helper warp
@@ -69,7 +74,7 @@ constexpr uint32_t kTmemCols = 512;
 // TMEM columns: two S/P buffers (S fp32, then P as bf16 pairs in the first 16 columns
 // of each 32-column block), Y (64 per head) and the fp32 state H = h^T (64 per head).
 constexpr uint32_t kColSP = 0, kColY = 256, kColH = 384;
-constexpr float kRangeMax = 200.f;            // log2 units of decay one pass may span
+constexpr float kRangeHalf = 100.f;           // |m - c_j| bound (log2 units): 2^100 stays well inside bf16
 constexpr uint32_t kAtom = kTile * 128;       // one 128-row x 128-byte swizzled operand column
 
 // mbarriers (index = bit of the 64-bit phase masks)
@@ -83,7 +88,8 @@ enum {
   kBarSt = kBarP0 + 2,                // right factor accumulated onto H (commit)
   kBarY,                              // P U accumulated into Y (commit)
   kBarU,                              // U written (16)
-  kBarHt,                             // h^ written, bf16 in shared and fp32 in H (16)
+  kBarHt,                             // bf16 copy of H written for the left factor (16)
+  kBarHRead,                          // H read (and rescaled if needed): the next right factor may add (16)
   kBarFree,                           // Y read by the epilogue (16)
   kBarDrain,                          // the MMA warp's last commit after an abort
   kBarDt0,                            // kDtStages: dt of a tile (4 heads x 128 tokens)
@@ -108,7 +114,8 @@ enum {
   kPCarryIn = 8,     // ... handed on by CTA carry_src
   kPToFinal = 16,    // the state after this pass is the unit's final state
   kPToCarry = 32,    // ... is handed on to the next CTA
-  kPEnd = 64         // no pass: the range is done
+  kPEnd = 64,        // no pass: the range is done
+  kPRescale0 = 128   // (<< head) re-centred reference: H = sig_in sig_out' H before this pass
 };
 struct PassDesc {
   int t0;         // token index of row 0 of the tile
@@ -118,8 +125,8 @@ struct PassDesc {
   int h0;         // first head of the pair
   int flags;
   int carry_src;
-  float sig_in[kHeads];   // h^ = sig_in h_in: 2^(m - c_before(lo))
-  float sig_out[kHeads];  // h_out = sig_out H: 2^(c(hi - 1) - m)
+  float sig_in[kHeads];   // piece start or re-centred: H = sig_in h before the pass, 2^(m - c_before(lo))
+  float sig_out[kHeads];  // h after the pass = sig_out H: 2^(c(hi - 1) - m)
   float dskip[kHeads];    // D
   float pad[2];
   float u[kHeads][kTile];  // 2^(m - c_j) dt_j on the pass's rows, else 0
@@ -199,7 +206,7 @@ __device__ __forceinline__ int unit_of_tile(const Problem& pb, int64_t w) {
   return lo * pairs + (int)((w - (int64_t)pb.seq_tiles[lo] * pairs) / T);
 }
 
-__device__ __forceinline__ RangePlan plan_range(const Problem& pb) {
+__device__ __noinline__ RangePlan plan_range(const Problem& pb) {
   RangePlan rp{};
   const int64_t W = seq_tile0(pb, pb.nseq) * (pb.H / kHeads);
   const int64_t w0 = W * blockIdx.x / gridDim.x, w1 = W * (blockIdx.x + 1) / gridDim.x;
@@ -216,7 +223,7 @@ __device__ __forceinline__ RangePlan plan_range(const Problem& pb) {
 }
 
 // Loads piece `pi` (processing order) into c; false when it has no tiles.
-__device__ __forceinline__ bool load_piece(const Problem& pb, const RangePlan& rp, int pi, TileCursor& c) {
+__device__ __noinline__ bool load_piece(const Problem& pb, const RangePlan& rp, int pi, TileCursor& c) {
   int u, kb, ke;
   if (rp.npieces == 1) {
     u = rp.u0, kb = rp.k0, ke = rp.ke1;
@@ -241,7 +248,7 @@ __device__ __forceinline__ bool load_piece(const Problem& pb, const RangePlan& r
   return true;
 }
 
-__device__ __forceinline__ bool cursor_from(const Problem& pb, const RangePlan& rp, int pi, TileCursor& c) {
+__device__ __noinline__ bool cursor_from(const Problem& pb, const RangePlan& rp, int pi, TileCursor& c) {
   for (; pi < rp.npieces; ++pi)
     if (load_piece(pb, rp, pi, c)) return true;
   return false;
@@ -266,11 +273,14 @@ __device__ __forceinline__ void warp_arrive(uint64_t* bar) {
   __syncwarp();
 }
 
+// dt of head h from the stored value; the prologue's softplus is out of line.
+__device__ __noinline__ float dt_prologue(const Problem& pb, float v, int h) { return dt_value(pb, v, h); }
+__device__ __forceinline__ float dt_of(const Problem& pb, float v, int h) { return pb.dt_prologue ? dt_prologue(pb, v, h) : v; }
+
 // Bounded wait (at most `limit` SM cycles) that also gives up when another thread has
-// recorded a failure.
-__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
-                                              long long limit) {
-  if (mbar_try_wait(bar, parity)) return true;
+// recorded a failure.  The spin is out of line: the hot loops stay small enough for the
+// instruction cache.
+__device__ __noinline__ bool wait_spin(uint64_t* bar, uint32_t parity, volatile int* abort_flag, long long limit) {
   const long long t0 = clock64();
   while (!mbar_try_wait(bar, parity)) {
     if (*abort_flag) return false;
@@ -280,6 +290,16 @@ __device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, vo
     }
   }
   return true;
+}
+__device__ __forceinline__ bool wait_or_abort(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                              long long limit) {
+  return mbar_try_wait(bar, parity) || wait_spin(bar, parity, abort_flag, limit);
+}
+// The same for a whole warp (every lane waits; warp-uniform result).
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort_flag,
+                                          long long limit) {
+  const bool mine = wait_or_abort(bar, parity, abort_flag, limit);
+  return !__any_sync(0xffffffffu, !mine);
 }
 
 // Phase bookkeeping of one thread (or one warp, waiting uniformly) over all barriers.
@@ -350,6 +370,8 @@ __device__ void load_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, cons
 }
 
 // ------------------------------------------------------------------ MMA warp
+// The whole warp walks the passes (so every operand is warp-uniform); one elected lane
+// issues each tcgen05.mma and commit.
 template <int NS>
 __device__ void mma_loop(const Problem& pb, uint8_t* smem, uint32_t tmem, uint64_t* bars,
                          volatile int* abort_flag) {
@@ -357,104 +379,120 @@ __device__ void mma_loop(const Problem& pb, uint8_t* smem, uint32_t tmem, uint64
   const uint32_t id_s = idesc_bf16(128, 128, 0, 0);   // C (K-major) x B (K-major)
   const uint32_t id_y = idesc_bf16(128, 128, 0, 1);   // C or P x (N-major h^ / U)
   const uint32_t id_h = idesc_bf16(128, 128, 1, 1);   // B^T (M-major) x U (N-major)
+  // Descriptors differ only in the start address field (address / 16, low bits), so a
+  // K step adds its byte offset / 16 to the operand's base descriptor.
+  const uint64_t k_major = sdesc_sw128(0, 16, 1024), mn_major = sdesc_sw128(0, kAtom, 1024);
+  const uint64_t ht_major = sdesc_sw128(0, NS * 128, 1024);
+  auto at = [](uint64_t tmpl, uint32_t addr) { return tmpl | (uint64_t)(addr >> 4); };
   const uint32_t a_ht = smem_u32(smem + L::ht);
   const PassDesc* descs = reinterpret_cast<const PassDesc*>(smem + L::desc);
+  const bool leader = elect_one();
   // For N = 64 the B^T operand has one M atom; the second (unused) half of H^T reads
   // the next ring slot or the state copy after it, and those lanes are never read.
   Phases ph;
   auto wait = [&](int k) -> bool {
-    if (!wait_or_abort(&bars[k], ph.parity(k), abort_flag, pb.wait_limit)) return false;
+    if (!warp_wait(&bars[k], ph.parity(k), abort_flag, pb.wait_limit)) return false;
     ph.flip(k);
     return true;
+  };
+  auto commit = [&](int k) {
+    if (leader) umma_commit(&bars[k]);
+  };
+  // H += B^T [U_0 | U_1] (K = 128 tokens, 8 steps of 16 rows = 2048 bytes)
+  auto right_factor = [&](uint64_t db, uint64_t dx) {
+    if (leader) {
+#pragma unroll
+      for (int kk = 0; kk < kTile / 16; ++kk) umma_f16(tmem + kColH, db + kk * 128, dx + kk * 128, id_h, 1);
+    }
   };
   const bool state_only = pb.y == nullptr;  // only the right factor: no S, P, Y
   bool ok = true, issued_any = false;
   int t = -1;
-  uint32_t a_c = 0, a_b = 0, a_x = 0, c_slot = 0, b_slot = 0;
+  uint32_t c_slot = 0, b_slot = 0;
+  uint64_t dc = 0, db = 0, dbm = 0, dx = 0;
   for (int p = 0;; ++p) {
     const int ds = p % kDescSlots;
     if (!(ok = wait(kBarDescFull0 + ds))) break;
     const PassDesc& d = descs[ds];
     const int flags = d.flags;
     if (flags & kPEnd) break;
-    if ((flags & kPFirst) && state_only) {
-      ++t;
-      b_slot = t % kRing;
-      a_b = smem_u32(smem + L::ring + b_slot * L::kSlot);
-      a_x = smem_u32(smem + L::x + (t & 1) * kHeads * kAtom);
-      if (!(ok = wait(kBarRing0 + b_slot))) break;
-    } else if (flags & kPFirst) {
+    if (flags & kPFirst) {
       ++t;
       c_slot = (2 * t) % kRing;
-      b_slot = (2 * t + 1) % kRing;
-      a_c = smem_u32(smem + L::ring + c_slot * L::kSlot);
-      a_b = smem_u32(smem + L::ring + b_slot * L::kSlot);
-      a_x = smem_u32(smem + L::x + (t & 1) * kHeads * kAtom);
-      if (!(ok = wait(kBarRing0 + c_slot)) || !(ok = wait(kBarRing0 + b_slot))) break;
-      tc_fence_after();
-      // S = C B^T into buffer t & 1 (the diagonal product that read P(t - 2) from it was
-      // issued earlier by this thread, and tcgen05.mma executes in issue order)
-      const uint32_t d_s = tmem + kColSP + (t & 1) * 128;
-#pragma unroll
-      for (int kk = 0; kk < NS / 16; ++kk) {
-        const uint32_t koff = (kk >> 2) * kAtom + (kk & 3) * 32;
-        umma_f16(d_s, sdesc_sw128(a_c + koff, 16, 1024), sdesc_sw128(a_b + koff, 16, 1024), id_s, kk > 0);
-      }
-      umma_commit(&bars[kBarS0 + (t & 1)]);
-      issued_any = true;
+      b_slot = state_only ? t % kRing : (2 * t + 1) % kRing;
+      const uint32_t a_c = smem_u32(smem + L::ring + c_slot * L::kSlot);
+      const uint32_t a_b = smem_u32(smem + L::ring + b_slot * L::kSlot);
+      dc = at(k_major, a_c);
+      db = at(k_major, a_b);
+      dbm = at(mn_major, a_b);
+      dx = at(mn_major, smem_u32(smem + L::x + (t & 1) * kHeads * kAtom));
+      if (!state_only && !(ok = wait(kBarRing0 + c_slot))) break;
+      if (!(ok = wait(kBarRing0 + b_slot))) break;
     }
     if (state_only) {  // H += B^T [U_0 | U_1] onto h^
-      if (!(ok = wait(kBarHt)) || !(ok = wait(kBarU))) break;
+      if (!(ok = wait(kBarHRead)) || !(ok = wait(kBarU))) break;
       tc_fence_after();
-#pragma unroll
-      for (int kk = 0; kk < kTile / 16; ++kk)
-        umma_f16(tmem + kColH, sdesc_sw128(a_b + kk * 2048, kAtom, 1024),
-                 sdesc_sw128(a_x + kk * 2048, kAtom, 1024), id_h, 1);
-      umma_commit(&bars[kBarSt]);
-      if (flags & kPLast) umma_commit(&bars[kBarRingFree0 + b_slot]);
+      right_factor(dbm, dx);
+      commit(kBarSt);
+      if (flags & kPLast) commit(kBarRingFree0 + b_slot);
       issued_any = true;
-      mbar_arrive(&bars[kBarDescFree0 + ds]);
+      if (leader) mbar_arrive(&bars[kBarDescFree0 + ds]);
       continue;
     }
-    // left factor Y = C [h^_0 h^_1]^T: needs h^ and the previous epilogue done with Y
+    if (flags & kPFirst) {
+      tc_fence_after();
+      // S = C B^T into buffer t & 1 (the diagonal product that read P(t - 2) from it was
+      // issued earlier by this warp, and tcgen05.mma executes in issue order); K step kk
+      // (16 state columns) is 32 bytes into 64-column atom kk / 4
+      const uint32_t d_s = tmem + kColSP + (t & 1) * 128;
+      if (leader) {
+#pragma unroll
+        for (int kk = 0; kk < NS / 16; ++kk) {
+          const uint32_t koff = ((kk >> 2) * kAtom + (kk & 3) * 32) >> 4;
+          umma_f16(d_s, dc + koff, db + koff, id_s, kk > 0);
+        }
+      }
+      commit(kBarS0 + (t & 1));
+      issued_any = true;
+    }
+    // left factor Y = C [h^_0 h^_1]^T: needs the bf16 copy of H and the previous
+    // epilogue done with Y
     if (!(ok = wait(kBarHt))) break;
     if (p > 0 && !(ok = wait(kBarFree))) break;
     tc_fence_after();
+    if (leader) {
+      const uint64_t dh = at(ht_major, a_ht);
 #pragma unroll
-    for (int kk = 0; kk < NS / 16; ++kk) {
-      const uint32_t koff = (kk >> 2) * kAtom + (kk & 3) * 32;
-      umma_f16(tmem + kColY, sdesc_sw128(a_c + koff, 16, 1024), sdesc_sw128(a_ht + kk * 2048, NS * 128, 1024),
-               id_y, kk > 0);
+      for (int kk = 0; kk < NS / 16; ++kk) {
+        const uint32_t koff = ((kk >> 2) * kAtom + (kk & 3) * 32) >> 4;
+        umma_f16(tmem + kColY, dc + koff, dh + kk * 128, id_y, kk > 0);
+      }
     }
-    if (flags & kPLast) umma_commit(&bars[kBarRingFree0 + c_slot]);  // C(t) read for the last time
-    // right factor H += B^T [U_0 | U_1]
-    if (!(ok = wait(kBarU))) break;
+    if (flags & kPLast) commit(kBarRingFree0 + c_slot);  // C(t) read for the last time
+    // right factor H += B^T [U_0 | U_1]: needs U and the state step done reading H
+    if (!(ok = wait(kBarU)) || !(ok = wait(kBarHRead))) break;
     tc_fence_after();
-#pragma unroll
-    for (int kk = 0; kk < kTile / 16; ++kk)
-      umma_f16(tmem + kColH, sdesc_sw128(a_b + kk * 2048, kAtom, 1024), sdesc_sw128(a_x + kk * 2048, kAtom, 1024),
-               id_h, 1);
-    umma_commit(&bars[kBarSt]);
-    if (flags & kPLast) umma_commit(&bars[kBarRingFree0 + b_slot]);  // B(t) read for the last time
+    right_factor(dbm, dx);
+    commit(kBarSt);
+    if (flags & kPLast) commit(kBarRingFree0 + b_slot);  // B(t) read for the last time
     // diagonal block Y += P [U_0 | U_1], P from tensor memory: K step kk (16 tokens) is
     // 8 columns at 32 (kk / 2) + 8 (kk % 2) of the buffer
     if ((flags & kPFirst) && !(ok = wait(kBarP0 + (t & 1)))) break;
     tc_fence_after();
-    {
+    if (leader) {
       const uint32_t a_p = tmem + kColSP + (t & 1) * 128;
 #pragma unroll
       for (int kk = 0; kk < kTile / 16; ++kk)
-        umma_f16_ta(tmem + kColY, a_p + 32 * (kk >> 1) + 8 * (kk & 1), sdesc_sw128(a_x + kk * 2048, kAtom, 1024),
-                    id_y, 1);
+        umma_f16_ta(tmem + kColY, a_p + 32 * (kk >> 1) + 8 * (kk & 1), dx + kk * 128, id_y, 1);
     }
-    umma_commit(&bars[kBarY]);
-    mbar_arrive(&bars[kBarDescFree0 + ds]);
+    commit(kBarY);
+    if (leader) mbar_arrive(&bars[kBarDescFree0 + ds]);
   }
   if (!ok) {
     *abort_flag = 1;
-    // every tcgen05.mma this thread issued completes before tensor memory is freed
+    // every tcgen05.mma this warp issued completes before tensor memory is freed
     if (issued_any) {
-      umma_commit(&bars[kBarDrain]);
+      commit(kBarDrain);
       mbar_wait_bounded(&bars[kBarDrain], 0, pb.wait_limit);
     }
   }
@@ -467,7 +505,98 @@ __device__ void mma_loop(const Problem& pb, uint8_t* smem, uint32_t tmem, uint64
 // What is the same for every row of a pass (where it is, the factors, the flags)
 // comes from the helper warp's descriptor.  The two halves of a row quarter meet
 // once a pass, on a one-arrival barrier, before the half-0 warp stores their 32 rows
-// of y by TMA.  Every wait is warp-uniform and bounded.
+// of y by TMA.  Every wait is warp-uniform and bounded.  The rare paths (initial
+// states, hand-ons, final states, empty units) are out-of-line functions, so the
+// per-pass loop stays small enough for the instruction cache.
+
+// Where this warp's part of the state (row n = i, columns 32 ch .. 32 ch + 31 of head hw)
+// lives in memory: state row (s, h, p) is n_stride long and this launch owns its columns
+// [n_off, n_off + N); hand-ons are N long per row, one block per CTA.
+__device__ __forceinline__ int64_t state_index(const Problem& pb, int s, int h, int ch, int i) {
+  return ((int64_t)s * pb.H + h) * kHeadDim * pb.n_stride + pb.n_off + (int64_t)(32 * ch) * pb.n_stride + i;
+}
+__device__ __forceinline__ int64_t carry_index(const Problem& pb, int cta, int hw, int ch, int i) {
+  return ((int64_t)cta * kHeads + hw) * kHeadDim * pb.N + (int64_t)(32 * ch) * pb.N + i;
+}
+
+// Units whose sequences are empty have no tiles: CTA r writes final = init (or 0) for
+// the empty units u with u % R == r.
+__device__ __noinline__ void empty_unit_states(const Problem& pb, int hw, int ch, int i) {
+  if (!pb.final_state || i >= pb.N) return;
+  const int pairs = pb.H / kHeads, units = pb.nseq * pairs;
+  for (int u = blockIdx.x; u < units; u += gridDim.x) {
+    if (unit_tiles(pb, u) != 0) continue;
+    const int64_t at = state_index(pb, u / pairs, (u % pairs) * kHeads + hw, ch, i);
+    for (int k = 0; k < 32; ++k) {
+      const int64_t o = at + (int64_t)k * pb.n_stride;
+      pb.final_state[o] = pb.init ? pb.init[o] : 0.f;
+    }
+  }
+}
+
+// The state at the start of the piece whose first pass d describes, into h: the
+// sequence's initial state (or zero), or the state CTA d.carry_src handed on (each warp
+// waits for the matching warp of that CTA).  False if that wait gave up.
+__device__ __noinline__ bool fetch_state(const Problem& pb, const PassDesc& d, int hw, int ch, int i, int wid,
+                                         volatile int* abort_flag, float* h) {
+  const float* src = nullptr;
+  int stride = pb.n_stride;
+  if (d.flags & kPCarryIn) {
+    bool mine = true;
+    if ((threadIdx.x & 31) == 0) {
+      const long long t0 = clock64();
+      while (ld_acquire_gpu_u64(&pb.carry_flag[d.carry_src * kComputeWarps + wid]) != pb.epoch) {
+        if (*abort_flag || clock64() - t0 > pb.wait_limit) {
+          *abort_flag = 1;
+          mine = false;
+          break;
+        }
+        __nanosleep(100);
+      }
+    }
+    if (__any_sync(0xffffffffu, !mine)) return false;
+    __threadfence();
+    src = pb.carry + carry_index(pb, d.carry_src, hw, ch, i);
+    stride = pb.N;
+  } else if (pb.init) {
+    src = pb.init + state_index(pb, d.s, d.h0 + hw, ch, i);
+  }
+  if (!src || i >= pb.N) src = nullptr;
+  for (int k = 0; k < 32; ++k) h[k] = src ? __ldcg(src + (int64_t)k * stride) : 0.f;
+  return true;
+}
+
+// The state after the pass d describes (h = h_out) as the unit's final state or as the
+// hand-on to the next CTA (then released to it, one flag per warp).
+__device__ __noinline__ void put_state(const Problem& pb, const PassDesc& d, int hw, int ch, int i, int wid,
+                                       const float* h) {
+  const bool to_final = d.flags & kPToFinal;
+  if (i < pb.N) {
+    float* dst = to_final ? pb.final_state + state_index(pb, d.s, d.h0 + hw, ch, i)
+                          : pb.carry + carry_index(pb, blockIdx.x, hw, ch, i);
+    const int stride = to_final ? pb.n_stride : pb.N;
+    for (int k = 0; k < 32; ++k) dst[(int64_t)k * stride] = h[k];
+  }
+  if (!to_final) {
+    __threadfence();
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0 && !pb.withhold_carry)
+      st_release_gpu_u64(&pb.carry_flag[blockIdx.x * kComputeWarps + wid], pb.epoch);
+    __syncwarp();
+  }
+}
+
+__device__ __forceinline__ void scale32(uint32_t (&r)[32], float f) {
+  const uint64_t f2v = f2(f, f);
+#pragma unroll
+  for (int k = 0; k < 16; ++k) {
+    float lo, hi;
+    unf2(mul2(f2v, f2u(r[2 * k], r[2 * k + 1])), lo, hi);
+    r[2 * k] = __float_as_uint(lo);
+    r[2 * k + 1] = __float_as_uint(hi);
+  }
+}
+
 template <int NS>
 __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8_t* smem, uint32_t tmem,
                              uint64_t* bars, volatile int* abort_flag) {
@@ -483,94 +612,50 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
   const uint32_t lane_base = (uint32_t)(q * 32) << 16;
   const uint32_t col_h = hw * 64 + ch * 32;  // this warp's Y and state columns
   uint8_t* sx = smem + L::x;
-  uint8_t* sht = smem + L::ht;
+  uint8_t* sht = smem + L::ht + hw * NS * 128;  // this head's bf16 copy of H
   const PassDesc* descs = reinterpret_cast<const PassDesc*>(smem + L::desc);
-  const int pairs = pb.H / kHeads;
-  const int units = pb.nseq * pairs;
 
   Phases ph;
   auto wait = [&](int k) -> bool {
-    const bool mine = wait_or_abort(&bars[k], ph.parity(k), abort_flag, pb.wait_limit);
-    if (__any_sync(0xffffffffu, !mine)) return false;
+    if (!warp_wait(&bars[k], ph.parity(k), abort_flag, pb.wait_limit)) return false;
     ph.flip(k);
     return true;
   };
 
-  // Units whose sequences are empty have no tiles: CTA r writes final = init for the
-  // empty units u with u % R == r.
-  // State size of this launch (NS, the operand width, is N rounded up; columns past N are
-  // 0).  In memory, state row (s, h, p) is NR = n_stride long and this launch owns its
-  // columns [n_off, n_off + N).
-  const int N = pb.N, NR = pb.n_stride;
-  if (pb.final_state && i < N) {
-    for (int u = blockIdx.x; u < units; u += gridDim.x) {
-      if (unit_tiles(pb, u) != 0) continue;
-      const int s = u / pairs;
-      const int h = (u % pairs) * kHeads + hw;
-      const int64_t base = ((int64_t)s * pb.H + h) * kHeadDim * NR + pb.n_off;
-      for (int p = 32 * ch; p < 32 * ch + 32; ++p)
-        pb.final_state[base + (int64_t)p * NR + i] = pb.init ? pb.init[base + (int64_t)p * NR + i] : 0.f;
-    }
-  }
+  empty_unit_states(pb, hw, ch, i);
 
   // The head state lives in tensor memory as H = h^T (lane n = state column n, 64 fp32
-  // columns per head, 32 per half); its bf16 copy in shared memory is the B operand of
-  // the left factor.  Both hold the same scaled value h^.
+  // columns per head, 32 per half) in the scale of the pass reference; its bf16 copy in
+  // shared memory is the B operand of the left factor.
   const uint32_t t_state = tmem + lane_base + kColH + col_h;
-  auto write_state = [&](uint32_t (&r)[32], float sig) {
-    const uint64_t s2 = f2(sig, sig);
+  const bool state_only = pb.y == nullptr;  // only the final states: no mask, no epilogue
+  auto write_copy = [&](const uint32_t (&r)[32]) {
+    if (state_only || i >= NS) return;
 #pragma unroll
-    for (int k = 0; k < 16; ++k) {
-      float lo, hi;
-      unf2(mul2(s2, f2u(r[2 * k], r[2 * k + 1])), lo, hi);
-      r[2 * k] = __float_as_uint(lo);
-      r[2 * k + 1] = __float_as_uint(hi);
+    for (int c = 0; c < 4; ++c) {
+      uint4 hv;
+      hv.x = bf16x2_of(f2u(r[8 * c + 0], r[8 * c + 1]));
+      hv.y = bf16x2_of(f2u(r[8 * c + 2], r[8 * c + 3]));
+      hv.z = bf16x2_of(f2u(r[8 * c + 4], r[8 * c + 5]));
+      hv.w = bf16x2_of(f2u(r[8 * c + 6], r[8 * c + 7]));
+      *reinterpret_cast<uint4*>(sht + sw128_off(i, 4 * ch + c)) = hv;
     }
-    if (i < NS) {
-      uint8_t* hdst = sht + hw * NS * 128;
+  };
+  // Installs the state before the pass d describes: the piece's initial state (a new
+  // piece) or H rescaled to d's reference (sig_out of the pass before, then sig_in), into
+  // tensor memory and r.  False if fetching the initial state gave up.
+  auto install = [&](const PassDesc& d, float sig_prev, uint32_t (&r)[32]) -> bool {
+    if (d.flags & kPPieceStart) {
+      float h[32];
+      if (!fetch_state(pb, d, hw, ch, i, wid, abort_flag, h)) return false;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        uint4 hv;
-        hv.x = bf16x2_of(f2u(r[8 * c + 0], r[8 * c + 1]));
-        hv.y = bf16x2_of(f2u(r[8 * c + 2], r[8 * c + 3]));
-        hv.z = bf16x2_of(f2u(r[8 * c + 4], r[8 * c + 5]));
-        hv.w = bf16x2_of(f2u(r[8 * c + 6], r[8 * c + 7]));
-        *reinterpret_cast<uint4*>(hdst + sw128_off(i, 4 * ch + c)) = hv;
-      }
+      for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(h[k]);
+    } else {
+      scale32(r, sig_prev);
     }
+    scale32(r, d.sig_in[hw]);
     tmem_st32(t_state, r);
     tmem_st_wait();
-  };
-  // The state at the start of the piece whose first pass d describes, into r: the
-  // sequence's initial state (or zero), or the state the previous CTA handed on (each
-  // warp waits for the matching warp of that CTA).  False if that wait gave up.
-  auto load_state = [&](const PassDesc& d, uint32_t (&r)[32]) -> bool {
-    const float* src_p = nullptr;
-    int rs = NR;  // row stride of the source
-    if (d.flags & kPCarryIn) {
-      const int src = d.carry_src;
-      bool mine = true;
-      if (lane == 0) {
-        const long long t0 = clock64();
-        while (ld_acquire_gpu_u64(&pb.carry_flag[src * kComputeWarps + wid]) != pb.epoch) {
-          if (*abort_flag || clock64() - t0 > pb.wait_limit) {
-            *abort_flag = 1;
-            mine = false;
-            break;
-          }
-          __nanosleep(100);
-        }
-      }
-      if (__any_sync(0xffffffffu, !mine)) return false;
-      __threadfence();
-      src_p = pb.carry + ((size_t)src * kHeads + hw) * kHeadDim * N + i;
-      rs = N;
-    } else if (pb.init) {
-      src_p = pb.init + ((int64_t)d.s * pb.H + d.h0 + hw) * kHeadDim * NR + pb.n_off + i;
-    }
-#pragma unroll
-    for (int k = 0; k < 32; ++k)
-      r[k] = __float_as_uint((src_p && i < N) ? __ldcg(src_p + (size_t)(32 * ch + k) * rs) : 0.f);
     return true;
   };
 
@@ -578,14 +663,14 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
   if (descs[0].flags & kPEnd) return;
   {
     uint32_t r[32];
-    if (!load_state(descs[0], r)) return;
-    write_state(r, descs[0].sig_in[hw]);
+    if (!install(descs[0], 1.f, r)) return;
+    tc_fence_before();
+    warp_arrive(&bars[kBarHRead]);
+    write_copy(r);
   }
   fence_proxy_async();
-  tc_fence_before();
-  warp_arrive(&bars[kBarHt]);
+  if (!state_only) warp_arrive(&bars[kBarHt]);
 
-  const bool state_only = pb.y == nullptr;  // only the final states: no mask, no epilogue
   uint32_t xr[16];  // this thread's x of the current tile: row i, columns 32 ch .. 32 ch + 31 of head hw
   int t = -1;
   bool staged_prev = false;  // the previous tile's y went out by TMA from its x stage
@@ -622,39 +707,24 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
     fence_proxy_async();
     warp_arrive(&bars[kBarU]);
 
-    if (flags & kPFirst) {
+    if ((flags & kPFirst) && t > 0) {
       // the previous tile's x stage: its y store has read it, so it may take tile t + 1's x
-      if (t > 0) {
-        if (staged_prev && ch == 0 && lane == 0) bulk_wait_read();
-        warp_arrive(&bars[kBarXfree0 + (st ^ 1)]);
-      }
+      if (staged_prev && ch == 0 && lane == 0) bulk_wait_read();
+      warp_arrive(&bars[kBarXfree0 + (st ^ 1)]);
     }
-    // ---- P = bf16(S) on and below the diagonal, written in place over S
+    // ---- P = bf16(S) on and below the diagonal, written in place over S: block (q, kb)
+    // is kept whole below the diagonal (kb < q), lower-triangular on it, zero above
     if ((flags & kPFirst) && !state_only) {
       if (!wait(kBarS0 + st)) return;
       tc_fence_after();
       const uint32_t t_blk = tmem + lane_base + kColSP + st * 128 + kb * 32;
-      uint32_t pk[16];
-      if (kb < q) {
-        uint32_t s[32];
-        tmem_ld32(t_blk, s);
-        tmem_ld_wait();
+      uint32_t sv[32], pk[16];
+      tmem_ld32(t_blk, sv);
+      tmem_ld_wait();
+      const int keep = kb < q ? 32 : kb == q ? lane + 1 : 0;  // columns kept in this row
 #pragma unroll
-        for (int k = 0; k < 16; ++k) pk[k] = bf16x2_of(f2u(s[2 * k], s[2 * k + 1]));
-      } else if (kb == q) {  // diagonal block: column 32 kb + j of row 32 q + lane kept for j <= lane
-        uint32_t s[32];
-        tmem_ld32(t_blk, s);
-        tmem_ld_wait();
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          const uint32_t lo = 2 * k <= lane ? s[2 * k] : 0u;
-          const uint32_t hi = 2 * k + 1 <= lane ? s[2 * k + 1] : 0u;
-          pk[k] = bf16x2_of(f2u(lo, hi));
-        }
-      } else {
-#pragma unroll
-        for (int k = 0; k < 16; ++k) pk[k] = 0u;
-      }
+      for (int k = 0; k < 16; ++k)
+        pk[k] = bf16x2_of(f2u(2 * k < keep ? sv[2 * k] : 0u, 2 * k + 1 < keep ? sv[2 * k + 1] : 0u));
       tmem_st16(t_blk, pk);
       tmem_st_wait();
       tc_fence_before();
@@ -662,57 +732,32 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
     }
 
     // ---- the state after this pass: at the end of a piece the final state or the
-    // hand-on to the next CTA; then the next pass's h^ (this state rescaled, or the next
-    // piece's initial state) as its bf16 copy and in tensor memory
+    // hand-on; then the next pass's H (as it stands, or re-centred, or the next piece's
+    // initial state) and its bf16 copy
     if (!wait(kBarSt)) return;
     tc_fence_after();
     const int nds = (p + 1) % kDescSlots;
     bool more;
     {
-      // h_out = sig_out H: the true state after this pass (always formed first, so the
-      // state a CTA hands on and the state it keeps are rounded alike)
       uint32_t r[32];
       tmem_ld32(t_state, r);
       tmem_ld_wait();
-      {
-        const float so = d.sig_out[hw];
-        const uint64_t so2 = f2(so, so);
-#pragma unroll
-        for (int k = 0; k < 16; ++k) {
-          float lo, hi;
-          unf2(mul2(so2, f2u(r[2 * k], r[2 * k + 1])), lo, hi);
-          r[2 * k] = __float_as_uint(lo);
-          r[2 * k + 1] = __float_as_uint(hi);
-        }
-      }
       if (flags & (kPToFinal | kPToCarry)) {
-        const bool to_final = flags & kPToFinal;
-        float* dst = to_final ? pb.final_state + ((int64_t)d.s * pb.H + d.h0 + hw) * kHeadDim * NR + pb.n_off + i
-                              : pb.carry + ((size_t)blockIdx.x * kHeads + hw) * kHeadDim * N + i;
-        const int ds_ = to_final ? NR : N;
-        if (i < N) {
+        float h[32];
 #pragma unroll
-          for (int k = 0; k < 32; ++k) dst[(size_t)(32 * ch + k) * ds_] = __uint_as_float(r[k]);
-        }
-        if (flags & kPToCarry) {  // this warp's part is out: one release per warp
-          __threadfence();
-          __syncwarp();
-          if (lane == 0 && !pb.withhold_carry)
-            st_release_gpu_u64(&pb.carry_flag[blockIdx.x * kComputeWarps + wid], pb.epoch);
-          __syncwarp();
-        }
+        for (int k = 0; k < 32; ++k) h[k] = __uint_as_float(r[k]) * d.sig_out[hw];
+        put_state(pb, d, hw, ch, i, wid, h);
       }
       if (!wait(kBarDescFull0 + nds)) return;
       const PassDesc& dn = descs[nds];
       more = !(dn.flags & kPEnd);
-      if (more) {
-        if ((dn.flags & kPPieceStart) && !load_state(dn, r)) return;
-        write_state(r, dn.sig_in[hw]);  // h^ of the next pass
-      }
+      if (more && (dn.flags & (kPPieceStart | (kPRescale0 << hw))) && !install(dn, d.sig_out[hw], r)) return;
+      tc_fence_before();
+      warp_arrive(&bars[kBarHRead]);
+      if (more) write_copy(r);
     }
     fence_proxy_async();
-    tc_fence_before();
-    warp_arrive(&bars[kBarHt]);
+    if (!state_only) warp_arrive(&bars[kBarHt]);
 
     if (state_only) {
       __syncwarp();
@@ -729,35 +774,35 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
     const bool single = (flags & (kPFirst | kPLast)) == (kPFirst | kPLast);
     const bool staged = single && d.rem >= 32 * q + 32;  // all 32 rows of this quarter are in the sequence
     {
-      const float rr = d.r[hw][i];
-      const float Dh = d.dskip[hw];
-      const uint64_t r2 = f2(rr, rr), d2 = f2(Dh, Dh);
-      const int h = d.h0 + hw;
       uint32_t ry[32];
       tmem_ld32(tmem + lane_base + kColY + col_h, ry);
+      const float rr = d.r[hw][i];
+      const float Dh = d.dskip[hw];
+      const int h = d.h0 + hw;
+      const bool in_pass = i >= d.lo && i < d.hi && i < d.rem;
+      const bool row_out = !staged && in_pass;
+      const bool add_prev = pb.y_accum && in_pass;  // y of the other state columns
+      __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(pb.y) + ((int64_t)(d.t0 + i) * pb.H + h) * kHeadDim + 32 * ch;
+      const uint64_t r2 = f2(rr, rr), d2 = f2(Dh, Dh);
       tmem_ld_wait();
-      const bool row_ok = !staged && i >= d.lo && i < d.hi && i < d.rem;
-      __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(pb.y) + ((int64_t)(d.t0 + i) * pb.H + h) * kHeadDim;
-      const bool add_prev = pb.y_accum && i >= d.lo && i < d.hi && i < d.rem;  // y of the other state columns
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
         uint32_t out[4];
         uint4 prev = make_uint4(0u, 0u, 0u, 0u);
-        if (add_prev) prev = *reinterpret_cast<const uint4*>(yrow + 32 * ch + 8 * c);
+        if (add_prev) prev = *reinterpret_cast<const uint4*>(yrow + 8 * c);
         const uint32_t pv[4] = {prev.x, prev.y, prev.z, prev.w};
 #pragma unroll
         for (int k = 0; k < 4; ++k) {  // bf16 pair -> fp32 pair (exact), then r Y + D x (+ y so far)
           const uint32_t xu = xr[4 * c + k];
-          const uint64_t x2 = f2u(xu << 16, xu & 0xFFFF0000u);
-          uint64_t acc = fma2(r2, f2u(ry[8 * c + 2 * k], ry[8 * c + 2 * k + 1]), mul2(d2, x2));
+          uint64_t acc = fma2(r2, f2u(ry[8 * c + 2 * k], ry[8 * c + 2 * k + 1]), mul2(d2, f2u(xu << 16, xu & 0xFFFF0000u)));
           if (pb.y_accum) acc = add2(acc, f2u(pv[k] << 16, pv[k] & 0xFFFF0000u));
           out[k] = bf16x2_of(acc);
         }
         const uint4 ov = make_uint4(out[0], out[1], out[2], out[3]);
         if (staged)
           *reinterpret_cast<uint4*>(sxh + sw128_off(i, 4 * ch + c)) = ov;
-        else if (row_ok)
-          *reinterpret_cast<uint4*>(yrow + 32 * ch + 8 * c) = ov;
+        else if (row_out)
+          *reinterpret_cast<uint4*>(yrow + 8 * c) = ov;
       }
       tc_fence_before();
       if (staged) fence_proxy_async();
@@ -790,9 +835,9 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
 // tile's dt by TMA into a ring of its own (kDtStages tiles in flight), and writes one
 // descriptor per pass into a ring of kDescSlots: where the pass is, its rows, the
 // factors u and r of both heads, the state scalings and the piece flags.  Per tile it
-// forms c (the inclusive cumsum of dt A in log2 units from the tile start, both heads)
-// and cuts the valid rows into passes whose decay range is at most kRangeMax: one pass
-// unless a head decays by more than 2^-kRangeMax across the tile.
+// forms c (the inclusive cumsum of dt A in log2 units from the tile start, both heads),
+// keeps or re-centres each head's reference and cuts the valid rows into passes: one
+// pass unless a head decays by more than 2^-(2 kRangeHalf) across the tile.
 template <int NS>
 __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t* smem, uint64_t* bars,
                             volatile int* abort_flag) {
@@ -805,8 +850,7 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t
   PassDesc* descs = reinterpret_cast<PassDesc*>(smem + L::desc);
   Phases ph;
   auto wait = [&](int k) -> bool {
-    const bool mine = wait_or_abort(&bars[k], ph.parity(k), abort_flag, pb.wait_limit);
-    if (__any_sync(0xffffffffu, !mine)) return false;
+    if (!warp_wait(&bars[k], ph.parity(k), abort_flag, pb.wait_limit)) return false;
     ph.flip(k);
     return true;
   };
@@ -831,6 +875,7 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t
   TileCursor cur;
   bool have = cursor_first(pb, rp, cur);
   float a2[kHeads] = {0.f, 0.f}, dsk[kHeads] = {0.f, 0.f};
+  float sg[kHeads] = {0.f, 0.f};  // per head: the pass reference m relative to the state before the next row
   int a_unit = -1, prev_piece = -1;
   bool ok = true;
   int t = 0, p = 0;
@@ -892,8 +937,8 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t
         const int k = (j - rot) & 3;
         const float x0 = k == 0 ? v0[0] : k == 1 ? v0[1] : k == 2 ? v0[2] : v0[3];
         const float x1 = k == 0 ? v1[0] : k == 1 ? v1[1] : k == 2 ? v1[2] : v1[3];
-        dtt[0][j] = j < left ? dt_value(pb, x0, h0) : 0.f;
-        dtt[1][j] = j < left ? dt_value(pb, x1, h0 + 1) : 0.f;
+        dtt[0][j] = j < left ? dt_of(pb, x0, h0) : 0.f;
+        dtt[1][j] = j < left ? dt_of(pb, x1, h0 + 1) : 0.f;
       }
     }
     // the dt stage is read: refill it
@@ -917,16 +962,34 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t
     }
     __syncwarp();
 
-    // passes over rows [0, rem): each as long as both heads' decay range fits
+    // passes over rows [0, rem).  A head keeps its reference m (sg[hh] = m - c_before(lo),
+    // carried over from the pass before) while every remaining row stays within
+    // kRangeHalf of it; otherwise the pass re-centres it on its rows, which then span at
+    // most 2 kRangeHalf (the pass ends where a re-centred head's range would be wider).
     for (int lo = 0; lo < rem;) {
-      const float clo0 = sc[lo], clo1 = sc[kTile + lo];
-      int bad = kTile;  // first row j > lo whose range from lo is too wide
+      const bool piece_start = first_tile && lo == 0;
+      float c0[kHeads], clo[kHeads];
+      bool keep[kHeads];
+#pragma unroll
+      for (int hh = 0; hh < kHeads; ++hh) {
+        c0[hh] = lo > 0 ? sc[hh * kTile + lo - 1] : 0.f;
+        clo[hh] = sc[hh * kTile + lo];
+        bool out = piece_start;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          const int row = 4 * lane + j;
+          out |= row >= lo && row < rem && fabsf(sg[hh] + c0[hh] - cth[hh][j]) > kRangeHalf;
+        }
+        keep[hh] = !__any_sync(0xffffffffu, out);
+      }
+      int bad = kTile;  // first row j > lo whose range from lo is too wide for a re-centred head
 #pragma unroll
       for (int j = 0; j < 4; ++j) {
         const int row = 4 * lane + j;
-        if (row > lo && row < rem && bad == kTile &&
-            (fabsf(clo0 - cth[0][j]) > kRangeMax || fabsf(clo1 - cth[1][j]) > kRangeMax))
-          bad = row;
+        bool over = false;
+#pragma unroll
+        for (int hh = 0; hh < kHeads; ++hh) over |= !keep[hh] && fabsf(clo[hh] - cth[hh][j]) > 2.f * kRangeHalf;
+        if (row > lo && row < rem && bad == kTile && over) bad = row;
       }
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) bad = min(bad, __shfl_xor_sync(0xffffffffu, bad, o));
@@ -937,10 +1000,11 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t
         ok = false;
         break;
       }
+      int rescale = 0;
 #pragma unroll
       for (int hh = 0; hh < kHeads; ++hh) {
         const float* ch_ = sc + hh * kTile;
-        const float m = 0.5f * (ch_[lo] + ch_[hi - 1]);
+        const float m = keep[hh] ? c0[hh] + sg[hh] : 0.5f * (clo[hh] + ch_[hi - 1]);
         float u[4], r[4];
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -952,17 +1016,18 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t
         reinterpret_cast<float4*>(d->u[hh])[lane] = make_float4(u[0], u[1], u[2], u[3]);
         reinterpret_cast<float4*>(d->r[hh])[lane] = make_float4(r[0], r[1], r[2], r[3]);
         if (lane == 0) {
-          const float cb = lo > 0 ? ch_[lo - 1] : 0.f;
-          d->sig_in[hh] = ex2(m - cb);
+          d->sig_in[hh] = ex2(m - c0[hh]);
           d->sig_out[hh] = ex2(ch_[hi - 1] - m);
           d->dskip[hh] = dsk[hh];
         }
+        if (!keep[hh] && !piece_start) rescale |= kPRescale0 << hh;
+        sg[hh] = m - ch_[hi - 1];  // the reference relative to the state after this pass
       }
       if (lane == 0) {
-        int flags = 0;
+        int flags = rescale;
         if (lo == 0) flags |= kPFirst;
         if (hi == rem) flags |= kPLast;
-        if (first_tile && lo == 0) flags |= kPPieceStart | ((cur.flags & kCarryIn) ? kPCarryIn : 0);
+        if (piece_start) flags |= kPPieceStart | ((cur.flags & kCarryIn) ? kPCarryIn : 0);
         if (last_tile && hi == rem) {
           if ((cur.flags & kUnitEnd) && pb.final_state) flags |= kPToFinal;
           if (cur.flags & kCarryOut) flags |= kPToCarry;
@@ -1025,6 +1090,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars[kBarY], 1);
     mbar_init(&bars[kBarU], kComputeWarps);
     mbar_init(&bars[kBarHt], kComputeWarps);
+    mbar_init(&bars[kBarHRead], kComputeWarps);
     mbar_init(&bars[kBarFree], kComputeWarps);
     mbar_init(&bars[kBarDrain], 1);
     for (int k = 0; k < kDtStages; ++k) mbar_init(&bars[kBarDt0 + k], 1);
@@ -1047,7 +1113,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t tmem = s_tmem_base;
 
   if (warp == kMmaWarp) {
-    if ((tid & 31) == 0) mma_loop<NS>(pb, smem, tmem, bars, abort_flag);
+    mma_loop<NS>(pb, smem, tmem, bars, abort_flag);
     __syncwarp();  // the warp reconverges before the CTA-wide barrier
   } else if (warp == kLoadWarp) {
     if ((tid & 31) == 0) load_loop<NS>(&tm_x, &tm_b, &tm_c, pb, smem, bars, abort_flag);
