@@ -70,12 +70,17 @@ constexpr int kThreads = (kComputeWarps + 3) * 32;
 constexpr int kDescSlots = 3;  // pass descriptors the helper may run ahead
 constexpr int kDtStages = 4;   // dt tiles in flight
 constexpr int kRing = 3;       // B / C tiles in shared memory (C(t), B(t) and the next one)
+constexpr int kMaxRanges = 1024;  // CTAs of one launch (one per SM)
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns: two S/P buffers (S fp32, then P as bf16 pairs in the first 16 columns
 // of each 32-column block), Y (64 per head) and the fp32 state H = h^T (64 per head).
 constexpr uint32_t kColSP = 0, kColY = 256, kColH = 384;
 constexpr float kRangeHalf = 100.f;           // |m - c_j| bound (log2 units): 2^100 stays well inside bf16
 constexpr uint32_t kAtom = kTile * 128;       // one 128-row x 128-byte swizzled operand column
+// Kernel variants (a template parameter, so each instance carries only its own code):
+// y and final states; y added to what y holds (the second column half of N = 256);
+// final states only (no C, no y).
+enum { kModeFull = 0, kModeAccum = 1, kModeState = 2 };
 
 // mbarriers (index = bit of the 64-bit phase masks)
 enum {
@@ -183,7 +188,7 @@ __device__ __forceinline__ int unit_tiles(const Problem& pb, int u) {
   return (int)(seq_tile0(pb, s + 1) - seq_tile0(pb, s));
 }
 
-__device__ __forceinline__ int64_t unit_first_tile(const Problem& pb, int u) {
+__device__ __noinline__ int64_t unit_first_tile(const Problem& pb, int u) {
   const int pairs = pb.H / kHeads;
   const int s = u / pairs;
   const int64_t a = seq_tile0(pb, s), b = seq_tile0(pb, s + 1);
@@ -191,7 +196,7 @@ __device__ __forceinline__ int64_t unit_first_tile(const Problem& pb, int u) {
 }
 
 // The unit holding flat tile w (0 <= w < W).
-__device__ __forceinline__ int unit_of_tile(const Problem& pb, int64_t w) {
+__device__ __noinline__ int unit_of_tile(const Problem& pb, int64_t w) {
   const int pairs = pb.H / kHeads;
   if (!pb.cu) return (int)(w / pb.dense_tiles);
   int lo = 0, hi = pb.nseq;  // seq_tiles[lo] * pairs <= w < seq_tiles[hi] * pairs
@@ -206,19 +211,20 @@ __device__ __forceinline__ int unit_of_tile(const Problem& pb, int64_t w) {
   return lo * pairs + (int)((w - (int64_t)pb.seq_tiles[lo] * pairs) / T);
 }
 
-__device__ __noinline__ RangePlan plan_range(const Problem& pb) {
+// dt of head h from the stored value; the prologue's softplus is out of line.
+__device__ __noinline__ float dt_prologue(const Problem& pb, float v, int h) { return dt_value(pb, v, h); }
+__device__ __forceinline__ float dt_of(const Problem& pb, float v, int h) { return pb.dt_prologue ? dt_prologue(pb, v, h) : v; }
+
+// The plan of flat tiles [w0, w1) whose first tile's predecessor is in CTA carry_src's range.
+__device__ __noinline__ RangePlan plan_of(const Problem& pb, int64_t w0, int64_t w1, int carry_src) {
   RangePlan rp{};
-  const int64_t W = seq_tile0(pb, pb.nseq) * (pb.H / kHeads);
-  const int64_t w0 = W * blockIdx.x / gridDim.x, w1 = W * (blockIdx.x + 1) / gridDim.x;
   if (w0 >= w1) return rp;
   rp.u0 = unit_of_tile(pb, w0);
   rp.k0 = (int)(w0 - unit_first_tile(pb, rp.u0));
   rp.u1 = unit_of_tile(pb, w1 - 1);
   rp.ke1 = (int)(w1 - unit_first_tile(pb, rp.u1));
   rp.npieces = rp.u0 == rp.u1 ? 1 : rp.u1 - rp.u0 + 1;
-  // range r holds tiles [W r / R, W (r + 1) / R): tile w lies in range ceil((w + 1) R / W) - 1
-  // (empty ranges are skipped over when there are fewer tiles than CTAs)
-  if (w0 > 0) rp.carry_src = (int)((w0 * gridDim.x + W - 1) / W) - 1;
+  rp.carry_src = carry_src;
   return rp;
 }
 
@@ -273,10 +279,6 @@ __device__ __forceinline__ void warp_arrive(uint64_t* bar) {
   __syncwarp();
 }
 
-// dt of head h from the stored value; the prologue's softplus is out of line.
-__device__ __noinline__ float dt_prologue(const Problem& pb, float v, int h) { return dt_value(pb, v, h); }
-__device__ __forceinline__ float dt_of(const Problem& pb, float v, int h) { return pb.dt_prologue ? dt_prologue(pb, v, h) : v; }
-
 // Bounded wait (at most `limit` SM cycles) that also gives up when another thread has
 // recorded a failure.  The spin is out of line: the hot loops stay small enough for the
 // instruction cache.
@@ -309,10 +311,250 @@ struct Phases {
   __device__ __forceinline__ void flip(int k) { bits ^= 1ull << k; }
 };
 
+// ------------------------------------------------------------------ work split
+// The flat tile list is cut at equal shares of a per-tile weight that follows the tile's
+// passes, so that CTAs whose units decay strongly (tiles of several passes) or that start
+// many short units do not finish last.  A head whose decay across a tile spans more than
+// 2 kRangeHalf (log2 units) cuts the tile into passes; such passes write y row by row and
+// weigh a little more than a single-pass tile (4 per single-pass tile, 5 per pass of a
+// multi-pass tile), and the first tile of a unit adds the cost of starting a piece (6).
+// tile_weight_kernel writes one byte per tile; every CTA then forms the same prefix sums
+// from them and takes its own cut points, so the CTAs need not wait for one another.
+constexpr int kSplitVec = 16;     // weights per 16-byte load
+struct SplitScratch {             // in the x stages, which the split runs before
+  int64_t pre[kThreads + 1];      // weight of the flat tiles before thread t's run
+};
+static_assert(sizeof(SplitScratch) <= 2 * kHeads * kAtom, "the split's scratch fits in the x stages");
+
+// Sum of the (byte) weights of tiles [a, a + 16) that lie below `end`.
+__device__ __forceinline__ int weights16(const uint8_t* tw, int64_t a, int64_t end) {
+  if (a >= end) return 0;
+  const uint4 q = __ldcg(reinterpret_cast<const uint4*>(tw + a));
+  const uint32_t qs[4] = {q.x, q.y, q.z, q.w};
+  const int64_t n = end - a;  // valid weights in this group (> 0)
+  uint32_t s = 0;             // (unsigned bytes: weights reach 251)
+#pragma unroll
+  for (int k = 0; k < 4; ++k) {
+    const int64_t left = n - 4 * k;
+    const uint32_t m = left >= 4 ? 0xFFFFFFFFu : left <= 0 ? 0u : (0xFFFFFFFFu >> (8 * (4 - left)));
+    s = __dp4a(qs[k] & m, 0x01010101u, s);
+  }
+  return (int)s;
+}
+
+// The first tile w of [a, b) whose preceding weight P(w) reaches t (P(a) = before), or
+// b; *pw = P(w).  Whole warp: each lane sums 16 weights, a scan over the lanes finds the
+// lane of the cut.  a is a multiple of 16.
+__device__ __noinline__ int64_t cut_in(const uint8_t* tw, int64_t a, int64_t b, int64_t before, int64_t t,
+                                       int64_t* pw) {
+  const int lane = threadIdx.x & 31;
+  int64_t acc = before;
+  for (int64_t base = a; base < b; base += 32 * kSplitVec) {
+    const int64_t lo = base + kSplitVec * lane;
+    const int sum = weights16(tw, lo, b);
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += x;
+    }
+    const int64_t mine = acc + incl - sum;  // P(lo)
+    // the cut lies in the first lane whose run ends at or past t (P(lo) + sum >= t)
+    const uint32_t hit = __ballot_sync(0xffffffffu, lo < b && mine + sum >= t);
+    if (hit) {
+      const int L = __ffs(hit) - 1;
+      int64_t w = b, p = 0;
+      if (lane == L) {
+        p = mine;
+        w = lo;
+        while (w < b && p < t) p += __ldcg(tw + w++);
+      }
+      *pw = __shfl_sync(0xffffffffu, p, L);
+      return __shfl_sync(0xffffffffu, w, L);
+    }
+    acc += __shfl_sync(0xffffffffu, incl, 31);
+  }
+  *pw = acc;
+  return b;
+}
+
+// This CTA's range, cut at equal weight shares (all threads of the CTA).  Thread t sums
+// the weights of its run [t per, (t + 1) per) of the flat list, a block scan gives each
+// run's preceding weight and the total T, and CTA c's range starts at the first tile
+// whose preceding weight reaches ceil(T c / R).  The tile before a CTA's first lies in
+// the range of the largest c' with ceil(T c' / R) <= that tile's preceding weight.
+__device__ __noinline__ RangePlan split_work(const Problem& pb, SplitScratch* sc) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int R = gridDim.x, r = blockIdx.x;
+  const int64_t W = seq_tile0(pb, pb.nseq) * (pb.H / kHeads);
+  if (W == 0) return RangePlan{};
+  const uint8_t* tw = pb.tile_w;
+  const int64_t per = (W + (int64_t)kThreads * kSplitVec - 1) / ((int64_t)kThreads * kSplitVec) * kSplitVec;
+  {
+    const int64_t a = tid * per, b = a + per < W ? a + per : W;
+    int sum = 0;
+    for (int64_t v = a; v < b; v += 4 * kSplitVec) {  // four loads in flight
+      int s4[4];
+#pragma unroll
+      for (int k = 0; k < 4; ++k) s4[k] = weights16(tw, v + k * kSplitVec, b);
+      sum += s4[0] + s4[1] + s4[2] + s4[3];
+    }
+    // block scan of the runs' sums: within the warp, then over the warps' totals
+    int incl = sum;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int x = __shfl_up_sync(0xffffffffu, incl, o);
+      if (lane >= o) incl += x;
+    }
+    if (lane == 31) sc->pre[warp] = incl;  // warp total, scanned below
+    __syncthreads();
+    if (warp == 0) {
+      const int64_t wt = lane < kThreads / 32 ? sc->pre[lane] : 0;
+      int64_t wi = wt;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int64_t x = __shfl_up_sync(0xffffffffu, wi, o);
+        if (lane >= o) wi += x;
+      }
+      __syncwarp();
+      if (lane < kThreads / 32) sc->pre[lane] = wi - wt;  // weight before warp `lane`
+      if (lane == kThreads / 32 - 1) sc->pre[kThreads] = wi;
+    }
+    __syncthreads();
+    const int64_t before_warp = sc->pre[warp];
+    __syncthreads();
+    sc->pre[tid] = before_warp + incl - sum;
+  }
+  __syncthreads();
+  __shared__ int64_t s_cut[2], s_at[2];
+  const int64_t T = sc->pre[kThreads];
+  if (warp < 2) {  // warp 0: this CTA's first tile, warp 1: the next CTA's
+    const int c = r + warp;
+    int64_t w = W, at = T;
+    if (c < R) {
+      const int64_t fl = T * c / R;
+      const int64_t t = fl + (fl * R < T * c);  // ceil(T c / R)
+      int lo = 0, hi = kThreads - 1;  // the last run with pre < t (pre[0] = 0)
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if (sc->pre[mid] < t)
+          lo = mid;
+        else
+          hi = mid - 1;
+      }
+      if (t <= 0) {
+        w = 0, at = 0;
+      } else {
+        const int64_t a = lo * per, b = a + per < W ? a + per : W;
+        w = cut_in(tw, a, b, sc->pre[lo], t, &at);
+      }
+    }
+    if (lane == 0) s_cut[warp] = w, s_at[warp] = at;
+  }
+  __syncthreads();
+  __shared__ RangePlan s_rp;
+  if (tid == 0) {
+    const int64_t w0 = s_cut[0], w1 = s_cut[1];
+    int src = 0;
+    if (w0 > 0 && w0 < w1) src = (int)((s_at[0] - (int64_t)__ldcg(tw + (w0 - 1))) * R / T);
+    s_rp = plan_of(pb, w0, w1, src);
+  }
+  __syncthreads();
+  return s_rp;
+}
+
+// Weight of every flat tile (a byte each, where the split reads it): one block per
+// (sequence, 128-token tile) sums that tile's dt over its tokens for all heads.  Thread t
+// owns the four heads 4 (t % G4) .. + 3 (G4 = H / 4) and the token rows t / G4 + k RP
+// (RP = rows covered at once), so the tile's rows are read as contiguous 16-byte runs and
+// summed in registers; shared memory only combines the row phases.
+constexpr int kWeightThreads = 512;
+__global__ void __launch_bounds__(kWeightThreads) tile_weight_kernel(Problem pb) {
+  extern __shared__ float4 part[];  // [RP][G4] partial sums, then hsum (H floats) after them
+  if (pb.cu && *pb.nchunks < 0) return;  // cu_seqlens rejected by the table kernel
+  const int pairs = pb.H / kHeads, H = pb.H, G4 = H / 4;
+  const int RP = G4 >= kWeightThreads ? 1 : kWeightThreads / G4;
+  float* hsum = reinterpret_cast<float*>(part + RP * (G4 < kWeightThreads ? G4 : kWeightThreads));
+  const int64_t seqtiles = seq_tile0(pb, pb.nseq);
+  for (int64_t st = blockIdx.x; st < seqtiles; st += gridDim.x) {
+    int s;
+    if (!pb.cu) {
+      s = (int)(st / pb.dense_tiles);
+    } else {
+      int lo = 0, hi = pb.nseq;  // seq_tiles[lo] <= st < seq_tiles[hi]
+      while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (pb.seq_tiles[mid] <= st)
+          lo = mid;
+        else
+          hi = mid;
+      }
+      s = lo;
+    }
+    const int kt = (int)(st - seq_tile0(pb, s));
+    const int64_t tb = seq_off(pb, s), len = seq_off(pb, s + 1) - tb;
+    const int64_t tok0 = tb + (int64_t)kt * kTile;
+    const int ntok = (int)(len - (int64_t)kt * kTile < kTile ? len - (int64_t)kt * kTile : kTile);
+    const float4* rows = reinterpret_cast<const float4*>(pb.dt + tok0 * H);  // 16-byte aligned (H % 4 == 0)
+    for (int g0 = 0; g0 < G4; g0 += kWeightThreads) {  // (one round unless H > 4 x 512)
+      const int gn = G4 - g0 < kWeightThreads ? G4 - g0 : kWeightThreads;
+      const int t = threadIdx.x, g = g0 + t % gn, ph = t / gn;
+      float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (ph < RP) {
+        for (int r0 = ph; r0 < ntok; r0 += 4 * RP) {  // four rows in flight
+          float4 v[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int r = r0 + k * RP;
+            v[k] = r < ntok ? __ldg(rows + (int64_t)r * G4 + g) : make_float4(0.f, 0.f, 0.f, 0.f);
+          }
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const int r = r0 + k * RP;
+            if (r < ntok) {
+              acc.x += dt_of(pb, v[k].x, 4 * g);
+              acc.y += dt_of(pb, v[k].y, 4 * g + 1);
+              acc.z += dt_of(pb, v[k].z, 4 * g + 2);
+              acc.w += dt_of(pb, v[k].w, 4 * g + 3);
+            }
+          }
+        }
+        part[ph * gn + t % gn] = acc;
+      }
+      __syncthreads();
+      for (int k = threadIdx.x; k < gn; k += kWeightThreads) {
+        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int p = 0; p < RP && p * gn < kWeightThreads; ++p) {
+          const float4 v = part[p * gn + k];
+          sum.x += v.x, sum.y += v.y, sum.z += v.z, sum.w += v.w;
+        }
+        hsum[4 * (g0 + k)] = sum.x, hsum[4 * (g0 + k) + 1] = sum.y, hsum[4 * (g0 + k) + 2] = sum.z,
+                      hsum[4 * (g0 + k) + 3] = sum.w;
+      }
+      __syncthreads();
+    }
+    for (int p = threadIdx.x; p < pairs; p += kWeightThreads) {
+      const int h0 = p * kHeads;
+      const float q = fmaxf(fabsf(pb.A[h0] * hsum[h0]), fabsf(pb.A[h0 + 1] * hsum[h0 + 1])) *
+                      (1.4426950408889634f / (2.f * kRangeHalf));
+      const int passes = q >= 1.f ? (q < 49.f ? 1 + (int)q : 49) : 1;  // (NaN: 1)
+      pb.tile_w[unit_first_tile(pb, s * pairs + p) + kt] = (uint8_t)((passes == 1 ? 4 : 5 * passes) + (kt == 0 ? 6 : 0));
+    }
+    __syncthreads();
+  }
+}
+
+// Dynamic shared memory of tile_weight_kernel for H heads.
+size_t tile_weight_smem(int H) {
+  const int G4 = H / 4, gn = G4 < kWeightThreads ? G4 : kWeightThreads, RP = G4 >= kWeightThreads ? 1 : kWeightThreads / G4;
+  return sizeof(float4) * (size_t)RP * gn + sizeof(float) * (size_t)H;
+}
+
 // ------------------------------------------------------------------ load warp
-template <int NS>
+template <int NS, int MODE>
 __device__ void load_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, const CUtensorMap* tm_c,
-                          const Problem& pb, uint8_t* smem, uint64_t* bars, volatile int* abort_flag) {
+                          const Problem& pb, const RangePlan& rp, uint8_t* smem, uint64_t* bars,
+                          volatile int* abort_flag) {
   using L = Layout<NS>;
   Phases ph;
   auto wait = [&](int k) -> bool {
@@ -320,7 +562,6 @@ __device__ void load_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, cons
     ph.flip(k);
     return true;
   };
-  const RangePlan rp = plan_range(pb);
   const int pairs = pb.H / kHeads;
   TileCursor cur;
   bool have = cursor_first(pb, rp, cur);
@@ -344,7 +585,7 @@ __device__ void load_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, cons
     ++nring;
     return true;
   };
-  const bool state_only = pb.y == nullptr;  // no y: C is not needed
+  constexpr bool state_only = MODE == kModeState;  // no y: C is not needed
   while (have) {
     const int h0 = (cur.unit % pairs) * kHeads, g = h0 / pb.hpg, tok = cur.tb + cur.k0;
     // C(t) goes into the slot B(t-2) held, x(t) into stage t & 1 once tile t-2's y is
@@ -372,7 +613,7 @@ __device__ void load_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, cons
 // ------------------------------------------------------------------ MMA warp
 // The whole warp walks the passes (so every operand is warp-uniform); one elected lane
 // issues each tcgen05.mma and commit.
-template <int NS>
+template <int NS, int MODE>
 __device__ void mma_loop(const Problem& pb, uint8_t* smem, uint32_t tmem, uint64_t* bars,
                          volatile int* abort_flag) {
   using L = Layout<NS>;
@@ -401,11 +642,11 @@ __device__ void mma_loop(const Problem& pb, uint8_t* smem, uint32_t tmem, uint64
   // H += B^T [U_0 | U_1] (K = 128 tokens, 8 steps of 16 rows = 2048 bytes)
   auto right_factor = [&](uint64_t db, uint64_t dx) {
     if (leader) {
-#pragma unroll
+#pragma unroll 1
       for (int kk = 0; kk < kTile / 16; ++kk) umma_f16(tmem + kColH, db + kk * 128, dx + kk * 128, id_h, 1);
     }
   };
-  const bool state_only = pb.y == nullptr;  // only the right factor: no S, P, Y
+  constexpr bool state_only = MODE == kModeState;  // only the right factor: no S, P, Y
   bool ok = true, issued_any = false;
   int t = -1;
   uint32_t c_slot = 0, b_slot = 0;
@@ -446,7 +687,7 @@ __device__ void mma_loop(const Problem& pb, uint8_t* smem, uint32_t tmem, uint64
       // (16 state columns) is 32 bytes into 64-column atom kk / 4
       const uint32_t d_s = tmem + kColSP + (t & 1) * 128;
       if (leader) {
-#pragma unroll
+#pragma unroll 1
         for (int kk = 0; kk < NS / 16; ++kk) {
           const uint32_t koff = ((kk >> 2) * kAtom + (kk & 3) * 32) >> 4;
           umma_f16(d_s, dc + koff, db + koff, id_s, kk > 0);
@@ -462,7 +703,7 @@ __device__ void mma_loop(const Problem& pb, uint8_t* smem, uint32_t tmem, uint64
     tc_fence_after();
     if (leader) {
       const uint64_t dh = at(ht_major, a_ht);
-#pragma unroll
+#pragma unroll 1
       for (int kk = 0; kk < NS / 16; ++kk) {
         const uint32_t koff = ((kk >> 2) * kAtom + (kk & 3) * 32) >> 4;
         umma_f16(tmem + kColY, dc + koff, dh + kk * 128, id_y, kk > 0);
@@ -481,7 +722,7 @@ __device__ void mma_loop(const Problem& pb, uint8_t* smem, uint32_t tmem, uint64
     tc_fence_after();
     if (leader) {
       const uint32_t a_p = tmem + kColSP + (t & 1) * 128;
-#pragma unroll
+#pragma unroll 1
       for (int kk = 0; kk < kTile / 16; ++kk)
         umma_f16_ta(tmem + kColY, a_p + 32 * (kk >> 1) + 8 * (kk & 1), dx + kk * 128, id_y, 1);
     }
@@ -587,17 +828,11 @@ __device__ __noinline__ void put_state(const Problem& pb, const PassDesc& d, int
 }
 
 __device__ __forceinline__ void scale32(uint32_t (&r)[32], float f) {
-  const uint64_t f2v = f2(f, f);
 #pragma unroll
-  for (int k = 0; k < 16; ++k) {
-    float lo, hi;
-    unf2(mul2(f2v, f2u(r[2 * k], r[2 * k + 1])), lo, hi);
-    r[2 * k] = __float_as_uint(lo);
-    r[2 * k + 1] = __float_as_uint(hi);
-  }
+  for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(__uint_as_float(r[k]) * f);
 }
 
-template <int NS>
+template <int NS, int MODE>
 __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8_t* smem, uint32_t tmem,
                              uint64_t* bars, volatile int* abort_flag) {
   using L = Layout<NS>;
@@ -628,16 +863,14 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
   // columns per head, 32 per half) in the scale of the pass reference; its bf16 copy in
   // shared memory is the B operand of the left factor.
   const uint32_t t_state = tmem + lane_base + kColH + col_h;
-  const bool state_only = pb.y == nullptr;  // only the final states: no mask, no epilogue
+  constexpr bool state_only = MODE == kModeState;  // only the final states: no mask, no epilogue
   auto write_copy = [&](const uint32_t (&r)[32]) {
-    if (state_only || i >= NS) return;
+    if constexpr (state_only) return;
+    if (i >= NS) return;
 #pragma unroll
     for (int c = 0; c < 4; ++c) {
-      uint4 hv;
-      hv.x = bf16x2_of(f2u(r[8 * c + 0], r[8 * c + 1]));
-      hv.y = bf16x2_of(f2u(r[8 * c + 2], r[8 * c + 3]));
-      hv.z = bf16x2_of(f2u(r[8 * c + 4], r[8 * c + 5]));
-      hv.w = bf16x2_of(f2u(r[8 * c + 6], r[8 * c + 7]));
+      const float* v = reinterpret_cast<const float*>(r) + 8 * c;
+      const uint4 hv = make_uint4(bf16x2(v[0], v[1]), bf16x2(v[2], v[3]), bf16x2(v[4], v[5]), bf16x2(v[6], v[7]));
       *reinterpret_cast<uint4*>(sht + sw128_off(i, 4 * ch + c)) = hv;
     }
   };
@@ -718,13 +951,21 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
       if (!wait(kBarS0 + st)) return;
       tc_fence_after();
       const uint32_t t_blk = tmem + lane_base + kColSP + st * 128 + kb * 32;
-      uint32_t sv[32], pk[16];
-      tmem_ld32(t_blk, sv);
-      tmem_ld_wait();
-      const int keep = kb < q ? 32 : kb == q ? lane + 1 : 0;  // columns kept in this row
+      uint32_t pk[16];
+      if (kb > q) {
 #pragma unroll
-      for (int k = 0; k < 16; ++k)
-        pk[k] = bf16x2_of(f2u(2 * k < keep ? sv[2 * k] : 0u, 2 * k + 1 < keep ? sv[2 * k + 1] : 0u));
+        for (int k = 0; k < 16; ++k) pk[k] = 0u;
+      } else {
+        uint32_t sv[32];
+        tmem_ld32(t_blk, sv);
+        tmem_ld_wait();
+        if (kb == q) {  // on the diagonal: column j of row lane kept for j <= lane
+#pragma unroll
+          for (int k = 0; k < 32; ++k) sv[k] = k <= lane ? sv[k] : 0u;
+        }
+#pragma unroll
+        for (int k = 0; k < 16; ++k) pk[k] = bf16x2(__uint_as_float(sv[2 * k]), __uint_as_float(sv[2 * k + 1]));
+      }
       tmem_st16(t_blk, pk);
       tmem_st_wait();
       tc_fence_before();
@@ -781,9 +1022,8 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
       const int h = d.h0 + hw;
       const bool in_pass = i >= d.lo && i < d.hi && i < d.rem;
       const bool row_out = !staged && in_pass;
-      const bool add_prev = pb.y_accum && in_pass;  // y of the other state columns
+      const bool add_prev = MODE == kModeAccum && in_pass;  // y of the other state columns
       __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(pb.y) + ((int64_t)(d.t0 + i) * pb.H + h) * kHeadDim + 32 * ch;
-      const uint64_t r2 = f2(rr, rr), d2 = f2(Dh, Dh);
       tmem_ld_wait();
 #pragma unroll
       for (int c = 0; c < 4; ++c) {
@@ -792,11 +1032,12 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
         if (add_prev) prev = *reinterpret_cast<const uint4*>(yrow + 8 * c);
         const uint32_t pv[4] = {prev.x, prev.y, prev.z, prev.w};
 #pragma unroll
-        for (int k = 0; k < 4; ++k) {  // bf16 pair -> fp32 pair (exact), then r Y + D x (+ y so far)
+        for (int k = 0; k < 4; ++k) {  // r Y + D x (+ y so far), x from its bf16 pair (exact)
           const uint32_t xu = xr[4 * c + k];
-          uint64_t acc = fma2(r2, f2u(ry[8 * c + 2 * k], ry[8 * c + 2 * k + 1]), mul2(d2, f2u(xu << 16, xu & 0xFFFF0000u)));
-          if (pb.y_accum) acc = add2(acc, f2u(pv[k] << 16, pv[k] & 0xFFFF0000u));
-          out[k] = bf16x2_of(acc);
+          float lo = fmaf(rr, __uint_as_float(ry[8 * c + 2 * k]), Dh * bf16_lo(xu));
+          float hi = fmaf(rr, __uint_as_float(ry[8 * c + 2 * k + 1]), Dh * bf16_hi(xu));
+          if (MODE == kModeAccum) lo += bf16_lo(pv[k]), hi += bf16_hi(pv[k]);
+          out[k] = bf16x2(lo, hi);
         }
         const uint4 ov = make_uint4(out[0], out[1], out[2], out[3]);
         if (staged)
@@ -838,9 +1079,9 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
 // forms c (the inclusive cumsum of dt A in log2 units from the tile start, both heads),
 // keeps or re-centres each head's reference and cuts the valid rows into passes: one
 // pass unless a head decays by more than 2^-(2 kRangeHalf) across the tile.
-template <int NS>
-__device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t* smem, uint64_t* bars,
-                            volatile int* abort_flag) {
+template <int NS, int MODE>
+__device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, const RangePlan& rp, uint8_t* smem,
+                            uint64_t* bars, volatile int* abort_flag) {
   using L = Layout<NS>;
   const int lane = threadIdx.x & 31;
   uint8_t* sdt = smem + L::sdt;
@@ -854,8 +1095,6 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t
     ph.flip(k);
     return true;
   };
-  const RangePlan rp = plan_range(pb);
-
   // dt loads run up to kDtStages tiles ahead on a cursor of their own
   TileCursor ahead;
   bool have_ahead = cursor_first(pb, rp, ahead);
@@ -1056,7 +1295,7 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, uint8_t
   }
 }
 
-template <int NS>
+template <int NS, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     ssd_fused_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
                         const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y32,
@@ -1111,18 +1350,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem_base;
+  const RangePlan rp = split_work(pb, reinterpret_cast<SplitScratch*>(smem + L::x));
 
   if (warp == kMmaWarp) {
-    mma_loop<NS>(pb, smem, tmem, bars, abort_flag);
+    mma_loop<NS, MODE>(pb, smem, tmem, bars, abort_flag);
     __syncwarp();  // the warp reconverges before the CTA-wide barrier
   } else if (warp == kLoadWarp) {
-    if ((tid & 31) == 0) load_loop<NS>(&tm_x, &tm_b, &tm_c, pb, smem, bars, abort_flag);
+    if ((tid & 31) == 0) load_loop<NS, MODE>(&tm_x, &tm_b, &tm_c, pb, rp, smem, bars, abort_flag);
     __syncwarp();
   } else if (warp == kHelperWarp) {
-    helper_loop<NS>(&tm_dt, pb, smem, bars, abort_flag);
+    helper_loop<NS, MODE>(&tm_dt, pb, rp, smem, bars, abort_flag);
     __syncwarp();
   } else {
-    compute_loop<NS>(&tm_y32, pb, smem, tmem, bars, abort_flag);
+    compute_loop<NS, MODE>(&tm_y32, pb, smem, tmem, bars, abort_flag);
     if ((tid & 31) == 0) bulk_wait_all();  // this warp's y stores complete before the CTA exits
     __syncwarp();
   }
@@ -1185,7 +1425,7 @@ bool make_dt_map(CUtensorMap* m, const float* dt, uint64_t H, uint64_t tokens) {
 }
 
 // The kernel's shared-memory size is set once per device and kernel instance.
-template <int NS>
+template <int NS, int MODE>
 cudaError_t set_smem_attribute() {
   static std::atomic<uint64_t> done{0};  // bit d: set on device d
   int dev = 0;
@@ -1193,18 +1433,19 @@ cudaError_t set_smem_attribute() {
   if (e != cudaSuccess) return e;
   const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
   if (bit && (done.load() & bit)) return cudaSuccess;
-  e = cudaFuncSetAttribute(ssd_fused_tc_kernel<NS>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kDynSmem<NS>);
+  e = cudaFuncSetAttribute(ssd_fused_tc_kernel<NS, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)kDynSmem<NS>);
   if (e == cudaSuccess && bit) done.fetch_or(bit);
   return e;
 }
 
-template <int NS>
-cudaError_t launch_ns(const Problem& pb, cudaStream_t st) {
+template <int NS, int MODE>
+cudaError_t launch_mode(const Problem& pb, cudaStream_t st) {
   CUtensorMap mx, mb, mc, my, mdt;
   const uint64_t tokens = (uint64_t)pb.tokens;
   // B and C: boxes of 64 state columns; past N the box reads zeros (N < NS).  Without y
   // (final states only) C and y are not read and their maps stand in as copies.
-  const bool state_only = pb.y == nullptr;
+  constexpr bool state_only = MODE == kModeState;
   const __nv_bfloat16* b0 = static_cast<const __nv_bfloat16*>(pb.B) + pb.n_off;
   const __nv_bfloat16* c0 = static_cast<const __nv_bfloat16*>(pb.C) + pb.n_off;
   if (!make_map(&mx, pb.x, kHeadDim, pb.H, tokens) || !make_map(&mb, b0, pb.N, pb.G, tokens, kTile, pb.n_stride) ||
@@ -1213,7 +1454,7 @@ cudaError_t launch_ns(const Problem& pb, cudaStream_t st) {
       !make_dt_map(&mdt, pb.dt, pb.H, tokens))
     return cudaErrorInvalidValue;
   if (state_only) mc = mb, my = mx;
-  cudaError_t e = set_smem_attribute<NS>();
+  cudaError_t e = set_smem_attribute<NS, MODE>();
   if (e != cudaSuccess) {
     if (getenv("SSD_DEBUG")) fprintf(stderr, "ssd: smem attribute failed: %s\n", cudaGetErrorString(e));
     return e;
@@ -1223,6 +1464,7 @@ cudaError_t launch_ns(const Problem& pb, cudaStream_t st) {
   // ranges may be empty when there are fewer tiles than SMs.
   const int grid = pb.ranges;
   if (grid <= 0) return cudaSuccess;
+  if (grid > kMaxRanges) return cudaErrorInvalidConfiguration;
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
@@ -1234,7 +1476,7 @@ cudaError_t launch_ns(const Problem& pb, cudaStream_t st) {
   cfg.attrs = attr;
   cfg.numAttrs = 1;
   if (pb.prof_start) cudaEventRecord(pb.prof_start, st);
-  e = cudaLaunchKernelEx(&cfg, ssd_fused_tc_kernel<NS>, mx, mb, mc, my, mdt, pb);
+  e = cudaLaunchKernelEx(&cfg, ssd_fused_tc_kernel<NS, MODE>, mx, mb, mc, my, mdt, pb);
   if (pb.prof_stop) cudaEventRecord(pb.prof_stop, st);
   count_launches(1);
   if (e == cudaSuccess) e = cudaGetLastError();
@@ -1242,6 +1484,12 @@ cudaError_t launch_ns(const Problem& pb, cudaStream_t st) {
     fprintf(stderr, "ssd: fused kernel launch failed: %s (smem %u, threads %d)\n", cudaGetErrorString(e),
             (unsigned)kDynSmem<NS>, kThreads);
   return e;
+}
+
+template <int NS>
+cudaError_t launch_ns(const Problem& pb, cudaStream_t st) {
+  if (!pb.y) return launch_mode<NS, kModeState>(pb, st);
+  return launch_mode<NS, kModeFull>(pb, st);
 }
 
 }  // namespace
@@ -1259,6 +1507,24 @@ bool tc_supports(const ssd_shape* s, int chunk) {
 }
 
 cudaError_t launch_tc(const Problem& pb, cudaStream_t st) {
+  // the tiles' weights for the work split (once: both column halves of N = 256 share them)
+  {
+    const int64_t seqtiles = pb.cu ? (pb.tokens + kTile - 1) / kTile + pb.nseq : (int64_t)pb.nseq * pb.dense_tiles;
+    const int grid = (int)(seqtiles < 8 * kMaxRanges ? seqtiles : 8 * kMaxRanges);
+    if (grid > 0) {
+      // the fused kernel's shared-memory carve-out, so the SMs need not switch between the launches
+      static std::atomic<uint64_t> carve{0};
+      int dev = 0;
+      if (cudaGetDevice(&dev) == cudaSuccess && dev < 64 && !(carve.load() & (1ull << dev))) {
+        cudaFuncSetAttribute(tile_weight_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+        carve.fetch_or(1ull << dev);
+      }
+      tile_weight_kernel<<<grid, kWeightThreads, tile_weight_smem(pb.H), st>>>(pb);
+      count_launches(1);
+      const cudaError_t e = cudaGetLastError();
+      if (e != cudaSuccess) return e;
+    }
+  }
   if (pb.N <= 128) {
     Problem q = pb;
     q.n_off = 0, q.n_stride = pb.N, q.y_accum = 0;
@@ -1276,7 +1542,8 @@ cudaError_t launch_tc(const Problem& pb, cudaStream_t st) {
   a.prof_stop = nullptr, b.prof_start = nullptr;
   b.epoch = pb.epoch ^ 0x8000000000000000ull;  // a value no other launch's flags hold
   cudaError_t e = launch_ns<128>(a, st);
-  return e == cudaSuccess ? launch_ns<128>(b, st) : e;
+  if (e != cudaSuccess) return e;
+  return b.y_accum ? launch_mode<128, kModeAccum>(b, st) : launch_ns<128>(b, st);
 }
 
 }  // namespace ssd
