@@ -235,12 +235,15 @@ int forward_segmented(const ssd_shape* s, int k, const void* x, const float* dt,
   const int nseq = (int)s->batch, nseg = nseq * k;
   const int64_t H = s->nheads, PN = s->headdim * s->dstate, HPN = H * PN;
   auto up = [](size_t v) { return (v + 255) & ~(size_t)255; };
+  const int Z = ssd::segments_slices(seg);
   const size_t o_cu = 0, o_st = up(sizeof(int32_t) * (nseg + 1)), o_lam = o_st + up(sizeof(float) * nseg * HPN),
-               o_h = o_lam + up(sizeof(float) * nseg * H), total = o_h + up(sizeof(float) * nseg * HPN);
+               o_part = o_lam + up(sizeof(float) * nseg * H), o_h = o_part + up(sizeof(float) * nseg * Z * H),
+               total = o_h + up(sizeof(float) * nseg * HPN);
   char* ws = nullptr;
   if (pool_alloc((void**)&ws, total, st) != cudaSuccess) return SSD_ERR_CUDA;
   int32_t* cu = (int32_t*)(ws + o_cu);
   float *states = (float*)(ws + o_st), *lam = (float*)(ws + o_lam), *h_in = (float*)(ws + o_h);
+  float* part = (float*)(ws + o_part);
   ssd_shape sg = *s;
   sg.batch = 1;
   sg.seqlen = s->batch * L;
@@ -251,7 +254,7 @@ int forward_segmented(const ssd_shape* s, int k, const void* x, const float* dt,
   // 1. every segment's end state from a zero state (x, dt, B only)
   if (rc == SSD_OK) rc = forward_impl(&sg, x, dt, A, B, nullptr, nullptr, nullptr, cu, chunk, nullptr, states, st);
   // 2. the segments' decays, true start states and the sequences' final states
-  if (rc == SSD_OK && (ssd::launch_segments_logdecay(cu, nseg, (int)H, dt, A, lam, st) != cudaSuccess ||
+  if (rc == SSD_OK && (ssd::launch_segments_logdecay(cu, nseg, seg, (int)H, dt, A, part, lam, st) != cudaSuccess ||
                        ssd::launch_segments_prefix(nseq, k, H, PN, states, lam, init, h_in, fin, st) != cudaSuccess))
     rc = SSD_ERR_CUDA;
   // 3. the full pass on the segments from their start states (y only)

@@ -115,8 +115,11 @@ cudaError_t launch_simt(const Problem& pb, cudaStream_t st);
 // per-segment log-decays; every segment's start state and (fin != null) each sequence's
 // final state, by the recurrence over its segments' zero-start end states.
 cudaError_t launch_segment_offsets(int nseq, int64_t L, int k, int64_t seg, int32_t* cu, cudaStream_t st);
-cudaError_t launch_segments_logdecay(const int32_t* cu, int nseg, int H, const float* dt, const float* A,
-                                     float* lam, cudaStream_t st);
+// Slices of 512 tokens in a segment of max_len tokens (the partial sums launch_segments_logdecay
+// keeps: nseg x slices x H floats in `part`).
+int segments_slices(int64_t max_len);
+cudaError_t launch_segments_logdecay(const int32_t* cu, int nseg, int64_t max_len, int H, const float* dt,
+                                     const float* A, float* part, float* lam, cudaStream_t st);
 cudaError_t launch_segments_prefix(int nseq, int k, int64_t H, int64_t PN, const float* states, const float* lam,
                                    const float* init, float* out, float* fin, cudaStream_t st);
 

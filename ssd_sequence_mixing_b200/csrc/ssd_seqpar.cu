@@ -15,25 +15,41 @@
 namespace ssd {
 namespace {
 
-constexpr int kHeadsPerBlock = 32, kTokLanes = 8;
+constexpr int kHeadsPerBlock = 32, kTokLanes = 32, kSliceTokens = 512;
 
-// Grid ceil(H / 32); block (32 heads x 8 token lanes): coalesced reads of dt rows.
-__global__ void __launch_bounds__(kHeadsPerBlock * kTokLanes)
-    segment_logdecay_kernel(int64_t tokens, int H, const float* dt, const float* A, float* out) {
+// The sum of dt over tokens [t0, t1) of heads blockIdx.x * 32 + (0 .. 31), into out[h]: a
+// block of 32 heads x 32 token lanes reads dt rows coalesced, each lane four tokens at a
+// time, and the lanes' sums are added in a fixed order (the result does not depend on
+// scheduling).
+__device__ void logdecay_slice(int64_t t0, int64_t t1, int H, const float* dt, float* out) {
   __shared__ float part[kTokLanes][kHeadsPerBlock];
   const int hl = threadIdx.x % kHeadsPerBlock, tl = threadIdx.x / kHeadsPerBlock;
   const int h = blockIdx.x * kHeadsPerBlock + hl;
-  float acc = 0.f;
+  float a0 = 0.f, a1 = 0.f, a2 = 0.f, a3 = 0.f;
   if (h < H)
-    for (int64_t t = tl; t < tokens; t += kTokLanes) acc += dt[t * H + h];
-  part[tl][hl] = acc;
+    for (int64_t t = t0 + tl; t < t1; t += 4 * kTokLanes) {
+      a0 += __ldg(dt + t * H + h);
+      if (t + kTokLanes < t1) a1 += __ldg(dt + (t + kTokLanes) * H + h);
+      if (t + 2 * kTokLanes < t1) a2 += __ldg(dt + (t + 2 * kTokLanes) * H + h);
+      if (t + 3 * kTokLanes < t1) a3 += __ldg(dt + (t + 3 * kTokLanes) * H + h);
+    }
+  part[tl][hl] = (a0 + a1) + (a2 + a3);
   __syncthreads();
   if (tl == 0 && h < H) {
     float s = 0.f;
 #pragma unroll
     for (int k = 0; k < kTokLanes; ++k) s += part[k][hl];
-    out[h] = s * A[h];
+    out[h] = s;
   }
+}
+
+// out[h] = A[h] * sum of dt over all tokens; grid ceil(H / 32).
+__global__ void __launch_bounds__(kHeadsPerBlock * kTokLanes)
+    segment_logdecay_kernel(int64_t tokens, int H, const float* dt, const float* A, float* out) {
+  logdecay_slice(0, tokens, H, dt, out);
+  __syncthreads();
+  const int h = blockIdx.x * kHeadsPerBlock + threadIdx.x;
+  if (threadIdx.x < kHeadsPerBlock && h < H) out[h] *= A[h];
 }
 
 // One thread per state element (h, p, n): the recurrence over the preceding segments.
@@ -91,23 +107,24 @@ __global__ void segment_offsets_kernel(int nseq, int64_t L, int k, int64_t seg, 
   cu[j] = (int32_t)(s == nseq ? (int64_t)nseq * L : (int64_t)s * L + (int64_t)i * seg);
 }
 
-// lam[j][h] = A[h] * sum of dt over segment j; grid (ceil(H / 32), nseg).
+// part[j][z][h] = sum of dt over slice z (512 tokens) of segment j (0 past its end); grid
+// (ceil(H / 32), nseg, Z).
 __global__ void __launch_bounds__(kHeadsPerBlock * kTokLanes)
-    segments_logdecay_kernel(const int32_t* cu, int H, const float* dt, const float* A, float* lam) {
-  __shared__ float part[kTokLanes][kHeadsPerBlock];
-  const int hl = threadIdx.x % kHeadsPerBlock, tl = threadIdx.x / kHeadsPerBlock;
-  const int h = blockIdx.x * kHeadsPerBlock + hl, j = blockIdx.y;
-  float acc = 0.f;
-  if (h < H)
-    for (int64_t t = cu[j] + tl; t < cu[j + 1]; t += kTokLanes) acc += dt[t * H + h];
-  part[tl][hl] = acc;
-  __syncthreads();
-  if (tl == 0 && h < H) {
-    float s = 0.f;
-#pragma unroll
-    for (int q = 0; q < kTokLanes; ++q) s += part[q][hl];
-    lam[(int64_t)j * H + h] = s * A[h];
-  }
+    segments_logdecay_kernel(const int32_t* cu, int H, int Z, const float* dt, float* part) {
+  const int j = blockIdx.y;
+  const int64_t t0 = (int64_t)cu[j] + (int64_t)blockIdx.z * kSliceTokens, end = cu[j + 1];
+  logdecay_slice(t0, t0 + kSliceTokens < end ? t0 + kSliceTokens : end, H, dt,
+                 part + ((int64_t)j * Z + blockIdx.z) * H);
+}
+
+// lam[j][h] = A[h] * sum over z of part[j][z][h], in slice order.
+__global__ void segments_lam_kernel(int nseg, int H, int Z, const float* part, const float* A, float* lam) {
+  const int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (e >= (int64_t)nseg * H) return;
+  const int64_t j = e / H, h = e % H;
+  float s = 0.f;
+  for (int z = 0; z < Z; ++z) s += part[(j * Z + z) * H + h];
+  lam[e] = s * A[h];
 }
 
 // Start state of every segment: for each sequence s (k segments) and state element e,
@@ -121,10 +138,20 @@ __global__ void __launch_bounds__(256) segments_prefix_kernel(int nseq, int k, i
   if (e >= H * PN) return;
   const int64_t h = e / PN;
   float acc = init ? init[(int64_t)s * H * PN + e] : 0.f;
-  for (int i = 0; i < k; ++i) {
-    const int64_t j = (int64_t)s * k + i;
-    out[j * H * PN + e] = acc;
-    acc = fmaf(expf(lam[j * H + h]), acc, states[j * H * PN + e]);
+  for (int i0 = 0; i0 < k; i0 += 4) {  // the states of four segments in flight at once
+    float sv[4], lv[4];
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int64_t j = (int64_t)s * k + i0 + q;
+      sv[q] = i0 + q < k ? __ldg(states + j * H * PN + e) : 0.f;
+      lv[q] = i0 + q < k ? __ldg(lam + j * H + h) : 0.f;
+    }
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      if (i0 + q >= k) break;
+      out[((int64_t)s * k + i0 + q) * H * PN + e] = acc;
+      acc = fmaf(expf(lv[q]), acc, sv[q]);
+    }
   }
   if (fin) fin[(int64_t)s * H * PN + e] = acc;
 }
@@ -138,11 +165,17 @@ cudaError_t launch_segment_offsets(int nseq, int64_t L, int k, int64_t seg, int3
   return cudaGetLastError();
 }
 
-cudaError_t launch_segments_logdecay(const int32_t* cu, int nseg, int H, const float* dt, const float* A,
-                                     float* lam, cudaStream_t st) {
-  segments_logdecay_kernel<<<dim3((H + kHeadsPerBlock - 1) / kHeadsPerBlock, nseg), kHeadsPerBlock * kTokLanes, 0,
-                             st>>>(cu, H, dt, A, lam);
-  count_launches(1);
+int segments_slices(int64_t max_len) { return (int)((max_len + kSliceTokens - 1) / kSliceTokens); }
+
+cudaError_t launch_segments_logdecay(const int32_t* cu, int nseg, int64_t max_len, int H, const float* dt,
+                                     const float* A, float* part, float* lam, cudaStream_t st) {
+  const int Z = segments_slices(max_len);
+  if (Z < 1 || Z > 65535 || nseg > 65535) return cudaErrorInvalidValue;
+  segments_logdecay_kernel<<<dim3((H + kHeadsPerBlock - 1) / kHeadsPerBlock, nseg, (unsigned)Z),
+                             kHeadsPerBlock * kTokLanes, 0, st>>>(cu, H, Z, dt, part);
+  const int64_t n = (int64_t)nseg * H;
+  segments_lam_kernel<<<(unsigned)((n + 255) / 256), 256, 0, st>>>(nseg, H, Z, part, A, lam);
+  count_launches(2);
   return cudaGetLastError();
 }
 

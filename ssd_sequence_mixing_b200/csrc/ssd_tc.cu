@@ -856,6 +856,11 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
     ph.flip(k);
     return true;
   };
+  // Final states only: the right factor of pass n completes phase n of kBarSt, and only the
+  // passes that end a piece or precede a re-centred / new state read H, so St is waited for
+  // by pass index.  A wait for phase n always comes before U(n + 1) is handed to the MMA
+  // warp, so the barrier is never two phases past it.
+  auto wait_st = [&](int n) -> bool { return warp_wait(&bars[kBarSt], (uint32_t)n & 1u, abort_flag, pb.wait_limit); };
 
   empty_unit_states(pb, hw, ch, i);
 
@@ -916,6 +921,9 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
     uint8_t* sxh = sx + (st * kHeads + hw) * kAtom;
 
     // ---- U = u_i x_i over the tile's x, in place (x itself stays in registers)
+    if constexpr (state_only) {  // a later pass of a tile rewrites U in place: the last product is done with it
+      if (!(flags & kPFirst) && !wait_st(p - 1)) return;
+    }
     if (flags & kPFirst) {
       if (!wait(kBarX0 + st)) return;
 #pragma unroll
@@ -936,6 +944,9 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
         v.w = mul_bf16x2(xr[4 * c + 3], u2);
         *reinterpret_cast<uint4*>(sxh + sw128_off(i, 4 * ch + c)) = v;
       }
+    }
+    if constexpr (state_only) {  // the previous tile's right factor is done with its x stage
+      if ((flags & kPFirst) && p > 0 && !wait_st(p - 1)) return;
     }
     fence_proxy_async();
     warp_arrive(&bars[kBarU]);
@@ -975,9 +986,37 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
     // ---- the state after this pass: at the end of a piece the final state or the
     // hand-on; then the next pass's H (as it stands, or re-centred, or the next piece's
     // initial state) and its bf16 copy
+    const int nds = (p + 1) % kDescSlots;
+    if constexpr (state_only) {  // H is read only where a piece ends or the next pass resets it
+      if (!wait(kBarDescFull0 + nds)) return;
+      const PassDesc& dn = descs[nds];
+      const bool more = !(dn.flags & kPEnd);
+      const bool out = flags & (kPToFinal | kPToCarry);
+      const bool reset = more && (dn.flags & (kPPieceStart | (kPRescale0 << hw)));
+      if (out || reset) {
+        if (!wait_st(p)) return;
+        tc_fence_after();
+        uint32_t r[32];
+        tmem_ld32(t_state, r);
+        tmem_ld_wait();
+        if (out) {
+          float h[32];
+#pragma unroll
+          for (int k = 0; k < 32; ++k) h[k] = __uint_as_float(r[k]) * d.sig_out[hw];
+          put_state(pb, d, hw, ch, i, wid, h);
+        }
+        if (reset && !install(dn, d.sig_out[hw], r)) return;
+      }
+      tc_fence_before();
+      warp_arrive(&bars[kBarHRead]);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kBarDescFree0 + ds]);
+      __syncwarp();
+      if (!more) break;
+      continue;
+    }
     if (!wait(kBarSt)) return;
     tc_fence_after();
-    const int nds = (p + 1) % kDescSlots;
     bool more;
     {
       uint32_t r[32];
@@ -998,15 +1037,8 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
       if (more) write_copy(r);
     }
     fence_proxy_async();
-    if (!state_only) warp_arrive(&bars[kBarHt]);
+    warp_arrive(&bars[kBarHt]);
 
-    if (state_only) {
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars[kBarDescFree0 + ds]);
-      __syncwarp();
-      if (!more) break;
-      continue;
-    }
     // ---- epilogue: y = r_i Y + D x; a single-pass tile stages y over its U and the
     // half-0 warp of each row quarter stores the quarter's 32 rows by TMA once the
     // half-1 warp has staged its columns; other rows go out as row stores
