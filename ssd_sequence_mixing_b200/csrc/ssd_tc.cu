@@ -70,6 +70,7 @@ constexpr int kThreads = (kComputeWarps + 3) * 32;
 constexpr int kDescSlots = 3;  // pass descriptors the helper may run ahead
 constexpr int kDtStages = 4;   // dt tiles in flight
 constexpr int kRing = 3;       // B / C tiles in shared memory (C(t), B(t) and the next one)
+constexpr int kMaxXStages = 4; // x stages of the final-state-only variant (2 otherwise)
 constexpr int kMaxRanges = 1024;  // CTAs of one launch (one per SM)
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns: two S/P buffers (S fp32, then P as bf16 pairs in the first 16 columns
@@ -84,9 +85,9 @@ enum { kModeFull = 0, kModeAccum = 1, kModeState = 2 };
 
 // mbarriers (index = bit of the 64-bit phase masks)
 enum {
-  kBarX0 = 0,                         // 2: x of a tile in stage s (tx bytes)
-  kBarXfree0 = kBarX0 + 2,            // 2: stage s free again (16 compute arrivals)
-  kBarRing0 = kBarXfree0 + 2,         // kRing: B or C tile in a ring slot (tx bytes)
+  kBarX0 = 0,                         // kMaxXStages: x of a tile in stage s (tx bytes)
+  kBarXfree0 = kBarX0 + kMaxXStages,  // kMaxXStages: stage s free again (16 compute arrivals)
+  kBarRing0 = kBarXfree0 + kMaxXStages,  // kRing: B or C tile in a ring slot (tx bytes)
   kBarRingFree0 = kBarRing0 + kRing,  // kRing: ring slot free (one UMMA commit)
   kBarS0 = kBarRingFree0 + kRing,     // 2: S = C B^T in S/P buffer b (commit)
   kBarP0 = kBarS0 + 2,                // 2: P written in buffer b (16 arrivals)
@@ -105,7 +106,8 @@ enum {
 };
 static_assert(kNumBars <= 64, "phase bits of a 64-bit mask");
 // every group of barriers has its own slots: the next group starts past its last one
-static_assert(kBarXfree0 == kBarX0 + 2 && kBarRing0 == kBarXfree0 + 2 && kBarRingFree0 == kBarRing0 + kRing &&
+static_assert(kBarXfree0 == kBarX0 + kMaxXStages && kBarRing0 == kBarXfree0 + kMaxXStages &&
+                  kBarRingFree0 == kBarRing0 + kRing &&
                   kBarS0 == kBarRingFree0 + kRing && kBarP0 == kBarS0 + 2 && kBarSt == kBarP0 + 2 &&
                   kBarDescFull0 == kBarDt0 + kDtStages && kBarDescFree0 == kBarDescFull0 + kDescSlots &&
                   kBarPair0 == kBarDescFree0 + kDescSlots,
@@ -120,7 +122,8 @@ enum {
   kPToFinal = 16,    // the state after this pass is the unit's final state
   kPToCarry = 32,    // ... is handed on to the next CTA
   kPEnd = 64,        // no pass: the range is done
-  kPRescale0 = 128   // (<< head) re-centred reference: H = sig_in sig_out' H before this pass
+  kPRescale0 = 128,  // (<< head) re-centred reference: H = sig_in sig_out' H before this pass
+  kPRescaleAny = kPRescale0 | (kPRescale0 << 1)
 };
 struct PassDesc {
   int t0;         // token index of row 0 of the tile
@@ -139,22 +142,39 @@ struct PassDesc {
 };
 constexpr uint32_t kDescBytes = (sizeof(PassDesc) + 127) / 128 * 128;
 
-template <int NS>
+// Shared memory.  The final-state-only variant (no C, no y, no state copy) spends what
+// those take on x stages instead: its tiles are short, and x loads four tiles ahead hide
+// the DRAM latency that two stages would expose.
+template <int NS, int MODE>
 struct Layout {
+  static constexpr bool kStateOnly = MODE == kModeState;
+  static constexpr int kXStages = kStateOnly ? kMaxXStages : 2;     // x stages
+  static constexpr int kRingSlots = kStateOnly ? 2 : kRing;         // B (and C) tiles
   static constexpr uint32_t kSlot = (NS / 64) * kAtom;             // one B or C tile
   static constexpr uint32_t x = 0;                                 // [stage][head] [128 tok][64 p]
-  static constexpr uint32_t ring = x + 2 * kHeads * kAtom;         // kRing slots [NS/64 atoms][128 tok][64 n]
-  static constexpr uint32_t ht = ring + kRing * kSlot;             // [head] [NS n][64 p]
-  static constexpr uint32_t desc = ht + kHeads * NS * 128;         // PassDesc[kDescSlots]
+  static constexpr uint32_t ring = x + kXStages * kHeads * kAtom;  // ring slots [NS/64 atoms][128 tok][64 n]
+  static constexpr uint32_t ht = ring + kRingSlots * kSlot;        // [head] [NS n][64 p]
+  // For N = 64 the right factor's B^T operand (M = 128) also reads the atom after its ring
+  // slot (rows never used); after the last slot that is the state copy, or in the
+  // final-state-only variant a pad of one atom, so the read stays inside the CTA's memory.
+  static constexpr uint32_t kHtBytes = kStateOnly ? (NS == 64 ? kAtom : 0) : kHeads * NS * 128;
+  static constexpr uint32_t desc = ht + kHtBytes;                   // PassDesc[kDescSlots]
   static constexpr uint32_t scan = desc + kDescSlots * kDescBytes; // helper: c[2][128]
   static constexpr uint32_t sdt = scan + kHeads * kTile * 4;       // float[stage][128 tok][4 heads]
   static constexpr uint32_t bars = sdt + kDtStages * kTile * 16;   // uint64[kNumBars]
   static constexpr uint32_t flag = bars + kNumBars * 8;            // int: a wait gave up
   static constexpr uint32_t bytes = flag + 16;
 };
-template <int NS>
-constexpr uint32_t kDynSmem = Layout<NS>::bytes + 1024;  // + base alignment slack
-static_assert(kDynSmem<128> <= 227 * 1024, "shared memory per CTA");
+template <int NS, int MODE>
+constexpr uint32_t kDynSmem = Layout<NS, MODE>::bytes + 1024;  // + base alignment slack
+template <int NS, int MODE>
+constexpr bool kBtInside = NS != 64 || Layout<NS, MODE>::ring + Layout<NS, MODE>::kRingSlots * Layout<NS, MODE>::kSlot +
+                                               kAtom <= Layout<NS, MODE>::desc;
+static_assert(kBtInside<64, kModeFull> && kBtInside<64, kModeState> && kBtInside<128, kModeFull> &&
+                  kBtInside<128, kModeAccum> && kBtInside<128, kModeState>,
+              "the N = 64 B^T operand's second atom lies inside the CTA's shared memory");
+static_assert(kDynSmem<128, kModeFull> <= 227 * 1024 && kDynSmem<128, kModeState> <= 227 * 1024,
+              "shared memory per CTA");
 
 // Work split.  The tiles of all units (sequence, head pair), unit by unit and each
 // unit's 128-token tiles in order, form one flat list; CTA r takes the contiguous
@@ -555,7 +575,7 @@ template <int NS, int MODE>
 __device__ void load_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, const CUtensorMap* tm_c,
                           const Problem& pb, const RangePlan& rp, uint8_t* smem, uint64_t* bars,
                           volatile int* abort_flag) {
-  using L = Layout<NS>;
+  using L = Layout<NS, MODE>;
   Phases ph;
   auto wait = [&](int k) -> bool {
     if (!wait_or_abort(&bars[k], ph.parity(k), abort_flag, pb.wait_limit)) return false;
@@ -575,13 +595,13 @@ __device__ void load_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, cons
     issued_par = (issued_par & ~(1ull << k)) | ((uint64_t)par << k);
   };
   auto ring_load = [&](const CUtensorMap* tm, int g, int tok) -> bool {
-    const int slot = nring % kRing;
-    if (nring >= (uint32_t)kRing && !wait(kBarRingFree0 + slot)) return false;
+    const int slot = nring % L::kRingSlots;
+    if (nring >= (uint32_t)L::kRingSlots && !wait(kBarRingFree0 + slot)) return false;
     uint8_t* dst = smem + L::ring + slot * L::kSlot;
     mbar_expect_tx(&bars[kBarRing0 + slot], L::kSlot);
 #pragma unroll
     for (int a = 0; a < NS / 64; ++a) tma_load_3d(dst + a * kAtom, tm, a * 64, g, tok, &bars[kBarRing0 + slot]);
-    note(kBarRing0 + slot, (nring / kRing) & 1u);
+    note(kBarRing0 + slot, (nring / L::kRingSlots) & 1u);
     ++nring;
     return true;
   };
@@ -591,13 +611,13 @@ __device__ void load_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, cons
     // C(t) goes into the slot B(t-2) held, x(t) into stage t & 1 once tile t-2's y is
     // out of it, B(t) into the slot C(t-1) held (free once the left factor of t-1 is done)
     if (!state_only && !(ok = ring_load(tm_c, g, tok))) break;
-    const int st = t & 1;
-    if (t >= 2 && !(ok = wait(kBarXfree0 + st))) break;
+    const int st = t % L::kXStages;
+    if (t >= L::kXStages && !(ok = wait(kBarXfree0 + st))) break;
     mbar_expect_tx(&bars[kBarX0 + st], kHeads * kAtom);
 #pragma unroll
     for (int hh = 0; hh < kHeads; ++hh)
       tma_load_3d(smem + L::x + (st * kHeads + hh) * kAtom, tm_x, 0, h0 + hh, tok, &bars[kBarX0 + st]);
-    note(kBarX0 + st, (uint32_t)(t >> 1) & 1u);
+    note(kBarX0 + st, (uint32_t)(t / L::kXStages) & 1u);
     if (!(ok = ring_load(tm_b, g, tok))) break;
     ++t;
     have = cursor_next(pb, rp, cur);
@@ -616,7 +636,7 @@ __device__ void load_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, cons
 template <int NS, int MODE>
 __device__ void mma_loop(const Problem& pb, uint8_t* smem, uint32_t tmem, uint64_t* bars,
                          volatile int* abort_flag) {
-  using L = Layout<NS>;
+  using L = Layout<NS, MODE>;
   const uint32_t id_s = idesc_bf16(128, 128, 0, 0);   // C (K-major) x B (K-major)
   const uint32_t id_y = idesc_bf16(128, 128, 0, 1);   // C or P x (N-major h^ / U)
   const uint32_t id_h = idesc_bf16(128, 128, 1, 1);   // B^T (M-major) x U (N-major)
@@ -648,6 +668,7 @@ __device__ void mma_loop(const Problem& pb, uint8_t* smem, uint32_t tmem, uint64
   };
   constexpr bool state_only = MODE == kModeState;  // only the right factor: no S, P, Y
   bool ok = true, issued_any = false;
+  int prev_flags = 0;  // (final states only) the previous pass's flags
   int t = -1;
   uint32_t c_slot = 0, b_slot = 0;
   uint64_t dc = 0, db = 0, dbm = 0, dx = 0;
@@ -660,18 +681,23 @@ __device__ void mma_loop(const Problem& pb, uint8_t* smem, uint32_t tmem, uint64
     if (flags & kPFirst) {
       ++t;
       c_slot = (2 * t) % kRing;
-      b_slot = state_only ? t % kRing : (2 * t + 1) % kRing;
+      b_slot = state_only ? t % L::kRingSlots : (2 * t + 1) % kRing;
       const uint32_t a_c = smem_u32(smem + L::ring + c_slot * L::kSlot);
       const uint32_t a_b = smem_u32(smem + L::ring + b_slot * L::kSlot);
       dc = at(k_major, a_c);
       db = at(k_major, a_b);
       dbm = at(mn_major, a_b);
-      dx = at(mn_major, smem_u32(smem + L::x + (t & 1) * kHeads * kAtom));
+      dx = at(mn_major, smem_u32(smem + L::x + (t % L::kXStages) * kHeads * kAtom));
       if (!state_only && !(ok = wait(kBarRing0 + c_slot))) break;
       if (!(ok = wait(kBarRing0 + b_slot))) break;
     }
     if (state_only) {  // H += B^T [U_0 | U_1] onto h^
-      if (!(ok = wait(kBarHRead)) || !(ok = wait(kBarU))) break;
+      // the compute warps touch H only after a pass that ends a piece or before one that
+      // starts or re-centres a state; only then does the product wait for them
+      const bool touched = (prev_flags & (kPToFinal | kPToCarry)) || (flags & (kPPieceStart | kPRescaleAny));
+      prev_flags = flags;
+      if (touched && !(ok = wait(kBarHRead))) break;
+      if (!(ok = wait(kBarU))) break;
       tc_fence_after();
       right_factor(dbm, dx);
       commit(kBarSt);
@@ -835,7 +861,7 @@ __device__ __forceinline__ void scale32(uint32_t (&r)[32], float f) {
 template <int NS, int MODE>
 __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8_t* smem, uint32_t tmem,
                              uint64_t* bars, volatile int* abort_flag) {
-  using L = Layout<NS>;
+  using L = Layout<NS, MODE>;
   const int tid = threadIdx.x;
   const int wid = tid >> 5;
   const int hw = wid >> 3;                   // head of the pair
@@ -917,7 +943,7 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
     const PassDesc& d = descs[ds];
     const int flags = d.flags;
     if (flags & kPFirst) ++t;
-    const int st = t & 1;
+    const int st = t % L::kXStages;
     uint8_t* sxh = sx + (st * kHeads + hw) * kAtom;
 
     // ---- U = u_i x_i over the tile's x, in place (x itself stays in registers)
@@ -954,14 +980,14 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
     if ((flags & kPFirst) && t > 0) {
       // the previous tile's x stage: its y store has read it, so it may take tile t + 1's x
       if (staged_prev && ch == 0 && lane == 0) bulk_wait_read();
-      warp_arrive(&bars[kBarXfree0 + (st ^ 1)]);
+      warp_arrive(&bars[kBarXfree0 + (st + L::kXStages - 1) % L::kXStages]);
     }
     // ---- P = bf16(S) on and below the diagonal, written in place over S: block (q, kb)
     // is kept whole below the diagonal (kb < q), lower-triangular on it, zero above
     if ((flags & kPFirst) && !state_only) {
-      if (!wait(kBarS0 + st)) return;
+      if (!wait(kBarS0 + (t & 1))) return;
       tc_fence_after();
-      const uint32_t t_blk = tmem + lane_base + kColSP + st * 128 + kb * 32;
+      const uint32_t t_blk = tmem + lane_base + kColSP + (t & 1) * 128 + kb * 32;
       uint32_t pk[16];
       if (kb > q) {
 #pragma unroll
@@ -980,7 +1006,7 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
       tmem_st16(t_blk, pk);
       tmem_st_wait();
       tc_fence_before();
-      warp_arrive(&bars[kBarP0 + st]);
+      warp_arrive(&bars[kBarP0 + (t & 1)]);
     }
 
     // ---- the state after this pass: at the end of a piece the final state or the
@@ -993,22 +1019,28 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
       const bool more = !(dn.flags & kPEnd);
       const bool out = flags & (kPToFinal | kPToCarry);
       const bool reset = more && (dn.flags & (kPPieceStart | (kPRescale0 << hw)));
-      if (out || reset) {
+      const bool touched = out || (more && (dn.flags & (kPPieceStart | kPRescaleAny)));  // same for all warps
+      // On such a pass every warp waits for the pass's right factor before it arrives on
+      // "H read": then no warp can arrive for the next such pass while another has not yet
+      // arrived for this one, and the MMA warp waits for it on exactly these passes.
+      if (touched) {
         if (!wait_st(p)) return;
         tc_fence_after();
-        uint32_t r[32];
-        tmem_ld32(t_state, r);
-        tmem_ld_wait();
-        if (out) {
-          float h[32];
+        if (out || reset) {
+          uint32_t r[32];
+          tmem_ld32(t_state, r);
+          tmem_ld_wait();
+          if (out) {
+            float h[32];
 #pragma unroll
-          for (int k = 0; k < 32; ++k) h[k] = __uint_as_float(r[k]) * d.sig_out[hw];
-          put_state(pb, d, hw, ch, i, wid, h);
+            for (int k = 0; k < 32; ++k) h[k] = __uint_as_float(r[k]) * d.sig_out[hw];
+            put_state(pb, d, hw, ch, i, wid, h);
+          }
+          if (reset && !install(dn, d.sig_out[hw], r)) return;
         }
-        if (reset && !install(dn, d.sig_out[hw], r)) return;
+        tc_fence_before();
+        warp_arrive(&bars[kBarHRead]);
       }
-      tc_fence_before();
-      warp_arrive(&bars[kBarHRead]);
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars[kBarDescFree0 + ds]);
       __syncwarp();
@@ -1114,7 +1146,7 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
 template <int NS, int MODE>
 __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, const RangePlan& rp, uint8_t* smem,
                             uint64_t* bars, volatile int* abort_flag) {
-  using L = Layout<NS>;
+  using L = Layout<NS, MODE>;
   const int lane = threadIdx.x & 31;
   uint8_t* sdt = smem + L::sdt;
   uint64_t* dt_bar = bars + kBarDt0;
@@ -1332,7 +1364,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     ssd_fused_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
                         const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y32,
                         const __grid_constant__ CUtensorMap tm_dt, Problem pb) {
-  using L = Layout<NS>;
+  using L = Layout<NS, MODE>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem_base;
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -1347,13 +1379,15 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int k = 0; k < 2; ++k) {
+    for (int k = 0; k < L::kXStages; ++k) {
       mbar_init(&bars[kBarX0 + k], 1);
       mbar_init(&bars[kBarXfree0 + k], kComputeWarps);
+    }
+    for (int k = 0; k < 2; ++k) {
       mbar_init(&bars[kBarS0 + k], 1);
       mbar_init(&bars[kBarP0 + k], kComputeWarps);
     }
-    for (int k = 0; k < kRing; ++k) {
+    for (int k = 0; k < L::kRingSlots; ++k) {
       mbar_init(&bars[kBarRing0 + k], 1);
       mbar_init(&bars[kBarRingFree0 + k], 1);
     }
@@ -1466,7 +1500,7 @@ cudaError_t set_smem_attribute() {
   const uint64_t bit = dev < 64 ? (1ull << dev) : 0;
   if (bit && (done.load() & bit)) return cudaSuccess;
   e = cudaFuncSetAttribute(ssd_fused_tc_kernel<NS, MODE>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                           (int)kDynSmem<NS>);
+                           (int)kDynSmem<NS, MODE>);
   if (e == cudaSuccess && bit) done.fetch_or(bit);
   return e;
 }
@@ -1500,7 +1534,7 @@ cudaError_t launch_mode(const Problem& pb, cudaStream_t st) {
   cudaLaunchConfig_t cfg{};
   cfg.gridDim = dim3(grid);
   cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = kDynSmem<NS>;
+  cfg.dynamicSmemBytes = kDynSmem<NS, MODE>;
   cfg.stream = st;
   cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeCooperative;  // all CTAs resident: carry waits always end
@@ -1514,7 +1548,7 @@ cudaError_t launch_mode(const Problem& pb, cudaStream_t st) {
   if (e == cudaSuccess) e = cudaGetLastError();
   if (e != cudaSuccess && getenv("SSD_DEBUG"))
     fprintf(stderr, "ssd: fused kernel launch failed: %s (smem %u, threads %d)\n", cudaGetErrorString(e),
-            (unsigned)kDynSmem<NS>, kThreads);
+            (unsigned)kDynSmem<NS, MODE>, kThreads);
   return e;
 }
 

@@ -346,3 +346,21 @@ def test_seeded_shape_sweep(case):
     for name, path in paths_for(prob, Q):
         y, fin = run(prob, path=path)
         check(prob, y, fin)
+
+
+def test_final_state_only_repeated_with_resets():
+    """The final-state-only variant at a size where its warps run ahead of the MMA warp:
+    heads that re-centre every tile (A = -60, -1e4) and long dense units (segments), run
+    repeatedly; every call must end without a wait giving up and match the full pass."""
+    wl = workloads.custom(4, 3000, H=16, P=64, N=128, G=2, chunk=256, dtype="bf16", init=True)
+    A = [-1e4, -1.0, -60.0, -2.0, -0.5, -30.0, -8.0, -1e-3] * 2
+    prob = workloads.generate(wl, seed=23, A_override=A)
+    dev = to_device(prob)
+    _, fin = ssd.ssd_forward(dev["x"], dev["dt"], dev["A"], dev["B"], dev["C"], dev["D"], dev["init_state"], None, 256)
+    for _ in range(5):
+        fin_only = ssd.ssd_final_state(dev["x"], dev["dt"], dev["A"], dev["B"], dev["init_state"], None, 256)
+        torch.cuda.synchronize()
+        assert ssd.query_status() == 0
+        assert torch.equal(fin, fin_only)
+    _, f_ref = oracle.ssd_forward_problem(prob)
+    assert_close("final_state", fin_only.cpu().numpy(), f_ref, "bf16")
