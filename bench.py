@@ -547,15 +547,16 @@ def block_measurements(dev, stream, flush):
     t_norm = _median_us(lambda: ssd.gated_rmsnorm(y, z, wn, out=o, stream=stream), stream, flush)
     norm_bytes = tokens * dim * 2 * 3 + dim * 4
 
-    def line(name, t_us, nbytes):
+    def line(name, t_us, nbytes, kernel):
         gbs = nbytes / (t_us * 1e-6) / 1e9
         return {"workload": name, "us": t_us, "algorithmic_bytes": nbytes,
                 "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                             "frac": gbs / peaks["hbm_gbs"], "peak_source": f"{kind} (GB/s)"},
+                             "frac": gbs / peaks["hbm_gbs"], "peak_source": f"{kind} (GB/s)",
+                             "traffic": load_traffic(kernel), "kernel": kernel},
                 "l2": "flushed between launches"}
 
-    return {"causal_conv1d_silu": line("conv1d_k4_silu_b8_L2048_ch5376_bf16", t_conv, conv_bytes),
-            "gated_rmsnorm": line("gated_rmsnorm_tokens16384_dim5120_bf16", t_norm, norm_bytes)}
+    return {"causal_conv1d_silu": line("conv1d_k4_silu_b8_L2048_ch5376_bf16", t_conv, conv_bytes, "conv1d_silu"),
+            "gated_rmsnorm": line("gated_rmsnorm_tokens16384_dim5120_bf16", t_norm, norm_bytes, "gated_rmsnorm")}
 
 
 # ------------------------------------------------------ single-kernel targets for ncu
