@@ -119,7 +119,7 @@ int validate(const ssd_shape* s, const void* x, const float* dt, const float* A,
 }
 
 struct Scratch {
-  size_t table, seq_first, nchunks, cs, states, seq_tiles, carry, carry_flag, tile_w, total;
+  size_t table, seq_first, nchunks, cs, states, seq_tiles, carry, carry_flag, split_flag, tile_w, total;
   int ranges;
 };
 
@@ -148,7 +148,7 @@ Scratch scratch_layout(const ssd_shape* s, const int32_t* cu, int chunk, int pat
   }
   w.states = w.cs + cs_bytes;
   w.seq_tiles = w.states + st_bytes;
-  w.carry = w.carry_flag = w.tile_w = w.seq_tiles;
+  w.carry = w.carry_flag = w.split_flag = w.tile_w = w.seq_tiles;
   w.total = w.seq_tiles;
   w.ranges = 0;
   if (path == SSD_PATH_TC) {
@@ -162,7 +162,9 @@ Scratch scratch_layout(const ssd_shape* s, const int32_t* cu, int chunk, int pat
     const int64_t flat = (cu ? (tokens + ssd::kTcTile - 1) / ssd::kTcTile + nseq
                              : s->batch * ((s->seqlen + ssd::kTcTile - 1) / ssd::kTcTile)) *
                          (s->nheads / 2);
-    w.tile_w = w.carry_flag + up(sizeof(uint64_t) * 16 * (size_t)w.ranges);
+    // one flag per CTA for the barrier after the split's weights
+    w.split_flag = w.carry_flag + up(sizeof(uint64_t) * 16 * (size_t)w.ranges);
+    w.tile_w = w.split_flag + up(sizeof(uint64_t) * (size_t)w.ranges);
     w.total = w.tile_w + up((size_t)flat + 16);
   }
   return w;
@@ -334,6 +336,7 @@ int forward_impl(const ssd_shape* s, const void* x, const float* dt, const float
   pb.carry = (float*)(ws + w.carry);
   pb.carry_flag = (uint64_t*)(ws + w.carry_flag);
   pb.tile_w = (uint8_t*)(ws + w.tile_w);
+  pb.split_flag = (uint64_t*)(ws + w.split_flag);
   pb.epoch = next_epoch();
   pb.ranges = w.ranges;
   pb.wait_limit = g_wait_limit.load();

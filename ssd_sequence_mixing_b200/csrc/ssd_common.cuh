@@ -49,7 +49,9 @@ struct Problem {
   float* carry;          // (ranges, 2, P, N) states handed between CTAs
   uint64_t* carry_flag;  // (ranges, 16): `epoch` once a compute warp has published its part
   uint64_t epoch;        // unique per launch, so flags left in reused scratch never match
-  uint8_t* tile_w;        // weighted work split: a weight per flat tile (then 16 bytes of slack)
+  uint8_t* tile_w;       // weighted work split: a weight per flat tile (then 16 bytes of slack)
+  uint64_t* split_flag;  // (ranges): `epoch` once a CTA has written its share of tile_w
+  int weights_ready;     // tile_w already holds this problem's weights (no barrier)
   int ranges;            // CTAs of the tensor-core launch
   long long wait_limit;  // SM cycles a device-side wait may take before it gives up
   int withhold_carry;    // test hook: CTAs never publish the state they hand on

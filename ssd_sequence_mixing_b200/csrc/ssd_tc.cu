@@ -70,7 +70,7 @@ constexpr int kThreads = (kComputeWarps + 3) * 32;
 constexpr int kDescSlots = 3;  // pass descriptors the helper may run ahead
 constexpr int kDtStages = 4;   // dt tiles in flight
 constexpr int kRing = 3;       // B / C tiles in shared memory (C(t), B(t) and the next one)
-constexpr int kMaxXStages = 4; // x stages of the final-state-only variant (2 otherwise)
+constexpr int kXStages = 2;    // x tiles in shared memory
 constexpr int kMaxRanges = 1024;  // CTAs of one launch (one per SM)
 constexpr uint32_t kTmemCols = 512;
 // TMEM columns: two S/P buffers (S fp32, then P as bf16 pairs in the first 16 columns
@@ -85,20 +85,22 @@ enum { kModeFull = 0, kModeAccum = 1, kModeState = 2 };
 
 // mbarriers (index = bit of the 64-bit phase masks)
 enum {
-  kBarX0 = 0,                         // kMaxXStages: x of a tile in stage s (tx bytes)
-  kBarXfree0 = kBarX0 + kMaxXStages,  // kMaxXStages: stage s free again (16 compute arrivals)
-  kBarRing0 = kBarXfree0 + kMaxXStages,  // kRing: B or C tile in a ring slot (tx bytes)
+  kBarX0 = 0,                         // kXStages: x of a tile in stage s (tx bytes)
+  kBarXfree0 = kBarX0 + kXStages,     // kXStages: stage s free again (16 compute arrivals)
+  kBarRing0 = kBarXfree0 + kXStages,  // kRing: B or C tile in a ring slot (tx bytes)
   kBarRingFree0 = kBarRing0 + kRing,  // kRing: ring slot free (one UMMA commit)
   kBarS0 = kBarRingFree0 + kRing,     // 2: S = C B^T in S/P buffer b (commit)
   kBarP0 = kBarS0 + 2,                // 2: P written in buffer b (16 arrivals)
   kBarSt = kBarP0 + 2,                // right factor accumulated onto H (commit)
   kBarY,                              // P U accumulated into Y (commit)
-  kBarU,                              // U written (16)
+  kBarU,                              // U written (16); with final states only, U of even passes
+  kBarU1,                             // (final states only) U of odd passes written (16)
   kBarHt,                             // bf16 copy of H written for the left factor (16)
   kBarHRead,                          // H read (and rescaled if needed): the next right factor may add (16)
   kBarFree,                           // Y read by the epilogue (16)
-  kBarDrain,                          // the MMA warp's last commit after an abort
-  kBarDt0,                            // kDtStages: dt of a tile (4 heads x 128 tokens)
+  kBarDrain,                          // the MMA warp's last commit (after its last pass or an abort)
+  kBarUFree0,                         // 2: (final states only) U buffer b read by the right factor (commit)
+  kBarDt0 = kBarUFree0 + 2,           // kDtStages: dt of a tile (4 heads x 128 tokens)
   kBarDescFull0 = kBarDt0 + kDtStages,           // kDescSlots: descriptor written (helper)
   kBarDescFree0 = kBarDescFull0 + kDescSlots,    // kDescSlots: used up (16 compute + MMA)
   kBarPair0 = kBarDescFree0 + kDescSlots,        // 8: column-half-1 warp of (head, quarter) staged its y
@@ -106,7 +108,7 @@ enum {
 };
 static_assert(kNumBars <= 64, "phase bits of a 64-bit mask");
 // every group of barriers has its own slots: the next group starts past its last one
-static_assert(kBarXfree0 == kBarX0 + kMaxXStages && kBarRing0 == kBarXfree0 + kMaxXStages &&
+static_assert(kBarXfree0 == kBarX0 + kXStages && kBarRing0 == kBarXfree0 + kXStages &&
                   kBarRingFree0 == kBarRing0 + kRing &&
                   kBarS0 == kBarRingFree0 + kRing && kBarP0 == kBarS0 + 2 && kBarSt == kBarP0 + 2 &&
                   kBarDescFull0 == kBarDt0 + kDtStages && kBarDescFree0 == kBarDescFull0 + kDescSlots &&
@@ -143,16 +145,17 @@ struct PassDesc {
 constexpr uint32_t kDescBytes = (sizeof(PassDesc) + 127) / 128 * 128;
 
 // Shared memory.  The final-state-only variant (no C, no y, no state copy) spends what
-// those take on x stages instead: its tiles are short, and x loads four tiles ahead hide
-// the DRAM latency that two stages would expose.
+// those take on two U buffers of its own: x is read into registers and its stage released
+// at once, and U of the next pass is written while the right factor still reads this one.
 template <int NS, int MODE>
 struct Layout {
   static constexpr bool kStateOnly = MODE == kModeState;
-  static constexpr int kXStages = kStateOnly ? kMaxXStages : 2;     // x stages
+  static constexpr int kUBufs = kStateOnly ? 2 : 0;                 // U buffers (else U is written over x)
   static constexpr int kRingSlots = kStateOnly ? 2 : kRing;         // B (and C) tiles
   static constexpr uint32_t kSlot = (NS / 64) * kAtom;             // one B or C tile
   static constexpr uint32_t x = 0;                                 // [stage][head] [128 tok][64 p]
-  static constexpr uint32_t ring = x + kXStages * kHeads * kAtom;  // ring slots [NS/64 atoms][128 tok][64 n]
+  static constexpr uint32_t ub = x + kXStages * kHeads * kAtom;    // [buffer][head] [128 tok][64 p]
+  static constexpr uint32_t ring = ub + kUBufs * kHeads * kAtom;   // ring slots [NS/64 atoms][128 tok][64 n]
   static constexpr uint32_t ht = ring + kRingSlots * kSlot;        // [head] [NS n][64 p]
   // For N = 64 the right factor's B^T operand (M = 128) also reads the atom after its ring
   // slot (rows never used); after the last slot that is the state copy, or in the
@@ -338,40 +341,51 @@ struct Phases {
 // 2 kRangeHalf (log2 units) cuts the tile into passes; such passes write y row by row and
 // weigh a little more than a single-pass tile (4 per single-pass tile, 5 per pass of a
 // multi-pass tile), and the first tile of a unit adds the cost of starting a piece (6).
-// tile_weight_kernel writes one byte per tile; every CTA then forms the same prefix sums
-// from them and takes its own cut points, so the CTAs need not wait for one another.
+// Each CTA first writes the weight bytes of its share of the sequence tiles; the CTAs meet
+// once at a flag barrier (all of them are resident: the launch is cooperative); then every
+// CTA forms the same prefix sums and takes its own cut points.
 constexpr int kSplitVec = 16;     // weights per 16-byte load
 struct SplitScratch {             // in the x stages, which the split runs before
   int64_t pre[kThreads + 1];      // weight of the flat tiles before thread t's run
 };
 static_assert(sizeof(SplitScratch) <= 2 * kHeads * kAtom, "the split's scratch fits in the x stages");
+static_assert(sizeof(float4) * kThreads <= 2 * kHeads * kAtom, "the weights' scratch fits in the x stages");
 
-// Sum of the (byte) weights of tiles [a, a + 16) that lie below `end`.
-__device__ __forceinline__ int weights16(const uint8_t* tw, int64_t a, int64_t end) {
+// The (byte) weights of tiles [a, a + 16) into qs, those at or past `end` zeroed; returns
+// their sum.
+__device__ __forceinline__ int load16(const uint8_t* tw, int64_t a, int64_t end, uint32_t (&qs)[4]) {
+  qs[0] = qs[1] = qs[2] = qs[3] = 0u;
   if (a >= end) return 0;
   const uint4 q = __ldcg(reinterpret_cast<const uint4*>(tw + a));
-  const uint32_t qs[4] = {q.x, q.y, q.z, q.w};
+  const uint32_t raw[4] = {q.x, q.y, q.z, q.w};
   const int64_t n = end - a;  // valid weights in this group (> 0)
   uint32_t s = 0;             // (unsigned bytes: weights reach 251)
 #pragma unroll
   for (int k = 0; k < 4; ++k) {
     const int64_t left = n - 4 * k;
     const uint32_t m = left >= 4 ? 0xFFFFFFFFu : left <= 0 ? 0u : (0xFFFFFFFFu >> (8 * (4 - left)));
-    s = __dp4a(qs[k] & m, 0x01010101u, s);
+    qs[k] = raw[k] & m;
+    s = __dp4a(qs[k], 0x01010101u, s);
   }
   return (int)s;
 }
+__device__ __forceinline__ int weights16(const uint8_t* tw, int64_t a, int64_t end) {
+  uint32_t qs[4];
+  return load16(tw, a, end, qs);
+}
 
-// The first tile w of [a, b) whose preceding weight P(w) reaches t (P(a) = before), or
-// b; *pw = P(w).  Whole warp: each lane sums 16 weights, a scan over the lanes finds the
-// lane of the cut.  a is a multiple of 16.
+// The first tile w of [a, b) whose preceding weight P(w) reaches t (P(a) = before < t), or
+// b; *pw = P(w) and *pprev = P(w - 1) (-1 if no tile reaches t).  Whole warp: each lane
+// loads 16 weights, a scan over the lanes finds the lane of the cut, and that lane walks
+// its weights in registers.  a is a multiple of 16.
 __device__ __noinline__ int64_t cut_in(const uint8_t* tw, int64_t a, int64_t b, int64_t before, int64_t t,
-                                       int64_t* pw) {
+                                       int64_t* pw, int64_t* pprev) {
   const int lane = threadIdx.x & 31;
   int64_t acc = before;
   for (int64_t base = a; base < b; base += 32 * kSplitVec) {
     const int64_t lo = base + kSplitVec * lane;
-    const int sum = weights16(tw, lo, b);
+    uint32_t qs[4];
+    const int sum = load16(tw, lo, b, qs);
     int incl = sum;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
@@ -383,18 +397,22 @@ __device__ __noinline__ int64_t cut_in(const uint8_t* tw, int64_t a, int64_t b, 
     const uint32_t hit = __ballot_sync(0xffffffffu, lo < b && mine + sum >= t);
     if (hit) {
       const int L = __ffs(hit) - 1;
-      int64_t w = b, p = 0;
-      if (lane == L) {
-        p = mine;
-        w = lo;
-        while (w < b && p < t) p += __ldcg(tw + w++);
+      // that lane's P(lo) is below t and every weight is positive, so the walk takes at
+      // least one tile and stops inside the valid ones
+      int64_t w = lo, p = mine, prev = mine;
+#pragma unroll
+      for (int k = 0; k < kSplitVec; ++k) {
+        const int64_t wt = (qs[k >> 2] >> (8 * (k & 3))) & 0xffu;
+        if (p < t) prev = p, p += wt, ++w;
       }
       *pw = __shfl_sync(0xffffffffu, p, L);
+      *pprev = __shfl_sync(0xffffffffu, prev, L);
       return __shfl_sync(0xffffffffu, w, L);
     }
     acc += __shfl_sync(0xffffffffu, incl, 31);
   }
   *pw = acc;
+  *pprev = -1;
   return b;
 }
 
@@ -446,11 +464,11 @@ __device__ __noinline__ RangePlan split_work(const Problem& pb, SplitScratch* sc
     sc->pre[tid] = before_warp + incl - sum;
   }
   __syncthreads();
-  __shared__ int64_t s_cut[2], s_at[2];
+  __shared__ int64_t s_cut[2], s_at, s_prev;
   const int64_t T = sc->pre[kThreads];
   if (warp < 2) {  // warp 0: this CTA's first tile, warp 1: the next CTA's
     const int c = r + warp;
-    int64_t w = W, at = T;
+    int64_t w = W, at = T, prev = -1;
     if (c < R) {
       const int64_t fl = T * c / R;
       const int64_t t = fl + (fl * R < T * c);  // ceil(T c / R)
@@ -466,108 +484,136 @@ __device__ __noinline__ RangePlan split_work(const Problem& pb, SplitScratch* sc
         w = 0, at = 0;
       } else {
         const int64_t a = lo * per, b = a + per < W ? a + per : W;
-        w = cut_in(tw, a, b, sc->pre[lo], t, &at);
+        w = cut_in(tw, a, b, sc->pre[lo], t, &at, &prev);
       }
     }
-    if (lane == 0) s_cut[warp] = w, s_at[warp] = at;
+    if (lane == 0) {
+      s_cut[warp] = w;
+      if (warp == 0) s_at = at, s_prev = prev;
+    }
   }
   __syncthreads();
   __shared__ RangePlan s_rp;
   if (tid == 0) {
     const int64_t w0 = s_cut[0], w1 = s_cut[1];
     int src = 0;
-    if (w0 > 0 && w0 < w1) src = (int)((s_at[0] - (int64_t)__ldcg(tw + (w0 - 1))) * R / T);
+    if (w0 > 0 && w0 < w1) {  // P(w0 - 1) R / T, rounded down
+      const int64_t pp = s_prev >= 0 ? s_prev : s_at - (int64_t)__ldcg(tw + (w0 - 1));
+      src = (int)(pp * R / T);
+    }
     s_rp = plan_of(pb, w0, w1, src);
   }
   __syncthreads();
   return s_rp;
 }
 
-// Weight of every flat tile (a byte each, where the split reads it): one block per
-// (sequence, 128-token tile) sums that tile's dt over its tokens for all heads.  Thread t
-// owns the four heads 4 (t % G4) .. + 3 (G4 = H / 4) and the token rows t / G4 + k RP
-// (RP = rows covered at once), so the tile's rows are read as contiguous 16-byte runs and
-// summed in registers; shared memory only combines the row phases.
-constexpr int kWeightThreads = 512;
-__global__ void __launch_bounds__(kWeightThreads) tile_weight_kernel(Problem pb) {
-  extern __shared__ float4 part[];  // [RP][G4] partial sums, then hsum (H floats) after them
-  if (pb.cu && *pb.nchunks < 0) return;  // cu_seqlens rejected by the table kernel
-  const int pairs = pb.H / kHeads, H = pb.H, G4 = H / 4;
-  const int RP = G4 >= kWeightThreads ? 1 : kWeightThreads / G4;
-  float* hsum = reinterpret_cast<float*>(part + RP * (G4 < kWeightThreads ? G4 : kWeightThreads));
-  const int64_t seqtiles = seq_tile0(pb, pb.nseq);
-  for (int64_t st = blockIdx.x; st < seqtiles; st += gridDim.x) {
-    int s;
-    if (!pb.cu) {
-      s = (int)(st / pb.dense_tiles);
-    } else {
-      int lo = 0, hi = pb.nseq;  // seq_tiles[lo] <= st < seq_tiles[hi]
-      while (hi - lo > 1) {
-        const int mid = (lo + hi) >> 1;
-        if (pb.seq_tiles[mid] <= st)
-          lo = mid;
-        else
-          hi = mid;
-      }
-      s = lo;
+// The weight bytes of sequence tile st: one per head pair, from the tile's dt summed per
+// head over its tokens (all NTHR threads of the block).  Thread t owns the four heads
+// 4 g .. 4 g + 3 (g = t % gn) and the token rows t / gn + k RP (RP = rows covered at
+// once), so the tile's rows are read as contiguous 16-byte runs, four in flight, and
+// summed in registers; `part` (NTHR float4 of shared memory) combines the row phases.
+template <int NTHR>
+__device__ __noinline__ void weigh_tile(const Problem& pb, int64_t st, float4* part) {
+  const int tid = threadIdx.x;
+  const int pairs = pb.H / kHeads, G4 = pb.H / 4;
+  int s;
+  if (!pb.cu) {
+    s = (int)(st / pb.dense_tiles);
+  } else {
+    int lo = 0, hi = pb.nseq;  // seq_tiles[lo] <= st < seq_tiles[hi]
+    while (hi - lo > 1) {
+      const int mid = (lo + hi) >> 1;
+      if (pb.seq_tiles[mid] <= st)
+        lo = mid;
+      else
+        hi = mid;
     }
-    const int kt = (int)(st - seq_tile0(pb, s));
-    const int64_t tb = seq_off(pb, s), len = seq_off(pb, s + 1) - tb;
-    const int64_t tok0 = tb + (int64_t)kt * kTile;
-    const int ntok = (int)(len - (int64_t)kt * kTile < kTile ? len - (int64_t)kt * kTile : kTile);
-    const float4* rows = reinterpret_cast<const float4*>(pb.dt + tok0 * H);  // 16-byte aligned (H % 4 == 0)
-    for (int g0 = 0; g0 < G4; g0 += kWeightThreads) {  // (one round unless H > 4 x 512)
-      const int gn = G4 - g0 < kWeightThreads ? G4 - g0 : kWeightThreads;
-      const int t = threadIdx.x, g = g0 + t % gn, ph = t / gn;
+    s = lo;
+  }
+  const int kt = (int)(st - seq_tile0(pb, s));
+  const int64_t tb = seq_off(pb, s), len = seq_off(pb, s + 1) - tb;
+  const int64_t tok0 = tb + (int64_t)kt * kTile;
+  const int ntok = (int)(len - (int64_t)kt * kTile < kTile ? len - (int64_t)kt * kTile : kTile);
+  const float4* rows = reinterpret_cast<const float4*>(pb.dt + tok0 * pb.H);  // 16-byte aligned (H % 4 == 0)
+  for (int g0 = 0; g0 < G4; g0 += NTHR) {  // (one round unless H > 4 NTHR)
+    const int gn = G4 - g0 < NTHR ? G4 - g0 : NTHR, RP = NTHR / gn;
+    const int g = g0 + tid % gn, ph = tid / gn;
+    if (ph < RP) {
       float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-      if (ph < RP) {
-        for (int r0 = ph; r0 < ntok; r0 += 4 * RP) {  // four rows in flight
-          float4 v[4];
+      for (int r0 = ph; r0 < ntok; r0 += 4 * RP) {  // four rows in flight
+        float4 v[4];
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int r = r0 + k * RP;
-            v[k] = r < ntok ? __ldg(rows + (int64_t)r * G4 + g) : make_float4(0.f, 0.f, 0.f, 0.f);
-          }
+        for (int k = 0; k < 4; ++k) {
+          const int rr = r0 + k * RP;
+          v[k] = rr < ntok ? __ldg(rows + (int64_t)rr * G4 + g) : make_float4(0.f, 0.f, 0.f, 0.f);
+        }
 #pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int r = r0 + k * RP;
-            if (r < ntok) {
-              acc.x += dt_of(pb, v[k].x, 4 * g);
-              acc.y += dt_of(pb, v[k].y, 4 * g + 1);
-              acc.z += dt_of(pb, v[k].z, 4 * g + 2);
-              acc.w += dt_of(pb, v[k].w, 4 * g + 3);
-            }
+        for (int k = 0; k < 4; ++k) {
+          if (r0 + k * RP < ntok) {
+            acc.x += dt_of(pb, v[k].x, 4 * g);
+            acc.y += dt_of(pb, v[k].y, 4 * g + 1);
+            acc.z += dt_of(pb, v[k].z, 4 * g + 2);
+            acc.w += dt_of(pb, v[k].w, 4 * g + 3);
           }
         }
-        part[ph * gn + t % gn] = acc;
       }
-      __syncthreads();
-      for (int k = threadIdx.x; k < gn; k += kWeightThreads) {
-        float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int p = 0; p < RP && p * gn < kWeightThreads; ++p) {
-          const float4 v = part[p * gn + k];
-          sum.x += v.x, sum.y += v.y, sum.z += v.z, sum.w += v.w;
-        }
-        hsum[4 * (g0 + k)] = sum.x, hsum[4 * (g0 + k) + 1] = sum.y, hsum[4 * (g0 + k) + 2] = sum.z,
-                      hsum[4 * (g0 + k) + 3] = sum.w;
-      }
-      __syncthreads();
+      part[ph * gn + tid % gn] = acc;
     }
-    for (int p = threadIdx.x; p < pairs; p += kWeightThreads) {
-      const int h0 = p * kHeads;
-      const float q = fmaxf(fabsf(pb.A[h0] * hsum[h0]), fabsf(pb.A[h0 + 1] * hsum[h0 + 1])) *
-                      (1.4426950408889634f / (2.f * kRangeHalf));
-      const int passes = q >= 1.f ? (q < 49.f ? 1 + (int)q : 49) : 1;  // (NaN: 1)
-      pb.tile_w[unit_first_tile(pb, s * pairs + p) + kt] = (uint8_t)((passes == 1 ? 4 : 5 * passes) + (kt == 0 ? 6 : 0));
+    __syncthreads();
+    if (tid < gn) {  // heads 4 g .. 4 g + 3 (g = g0 + tid): pairs 2 g and 2 g + 1
+      float hs[4] = {0.f, 0.f, 0.f, 0.f};
+      for (int q = 0; q < RP; ++q) {
+        const float4 v = part[q * gn + tid];
+        hs[0] += v.x, hs[1] += v.y, hs[2] += v.z, hs[3] += v.w;
+      }
+#pragma unroll
+      for (int k = 0; k < 2; ++k) {
+        const int pr = 2 * g + k, h0 = 2 * pr;
+        const float q = fmaxf(fabsf(pb.A[h0] * hs[2 * k]), fabsf(pb.A[h0 + 1] * hs[2 * k + 1])) *
+                        (1.4426950408889634f / (2.f * kRangeHalf));
+        const int passes = q >= 1.f ? (q < 49.f ? 1 + (int)q : 49) : 1;  // (NaN: 1)
+        pb.tile_w[unit_first_tile(pb, s * pairs + pr) + kt] =
+            (uint8_t)((passes == 1 ? 4 : 5 * passes) + (kt == 0 ? 6 : 0));
+      }
     }
     __syncthreads();
   }
 }
 
-// Dynamic shared memory of tile_weight_kernel for H heads.
-size_t tile_weight_smem(int H) {
-  const int G4 = H / 4, gn = G4 < kWeightThreads ? G4 : kWeightThreads, RP = G4 >= kWeightThreads ? 1 : kWeightThreads / G4;
-  return sizeof(float4) * (size_t)RP * gn + sizeof(float) * (size_t)H;
+// The weights of problems with many sequence tiles per SM, ahead of the fused kernel: one
+// block per sequence tile, several resident per SM, so the dt loads of many tiles overlap.
+constexpr int kWeightThreads = 512;
+__global__ void __launch_bounds__(kWeightThreads) tile_weight_kernel(Problem pb) {
+  __shared__ float4 part[kWeightThreads];
+  if (pb.cu && *pb.nchunks < 0) return;  // cu_seqlens rejected by the table kernel
+  const int64_t seqtiles = seq_tile0(pb, pb.nseq);
+  for (int64_t st = blockIdx.x; st < seqtiles; st += gridDim.x) weigh_tile<kWeightThreads>(pb, st, part);
+}
+
+// Every CTA's weights are written before any CTA reads them: CTA r sets split_flag[r] to
+// this launch's epoch (release) and waits, bounded, until every flag holds it.  The result
+// is the same for all threads of the CTA; false if a wait gave up.
+__device__ __noinline__ bool weights_barrier(const Problem& pb, volatile int* abort_flag) {
+  __syncthreads();  // this CTA's weight bytes are written
+  if (threadIdx.x == 0) {
+    __threadfence();
+    st_release_gpu_u64(&pb.split_flag[blockIdx.x], pb.epoch);
+  }
+  bool ok = true;
+  for (int k = threadIdx.x; k < (int)gridDim.x && ok; k += kThreads) {
+    const long long t0 = clock64();
+    while (ld_acquire_gpu_u64(&pb.split_flag[k]) != pb.epoch) {
+      if (clock64() - t0 > pb.wait_limit) {
+        ok = false;
+        break;
+      }
+      __nanosleep(32);
+    }
+  }
+  if (!ok) *abort_flag = 1;
+  __threadfence();
+  __syncthreads();
+  return !*abort_flag;
 }
 
 // ------------------------------------------------------------------ load warp
@@ -611,13 +657,13 @@ __device__ void load_loop(const CUtensorMap* tm_x, const CUtensorMap* tm_b, cons
     // C(t) goes into the slot B(t-2) held, x(t) into stage t & 1 once tile t-2's y is
     // out of it, B(t) into the slot C(t-1) held (free once the left factor of t-1 is done)
     if (!state_only && !(ok = ring_load(tm_c, g, tok))) break;
-    const int st = t % L::kXStages;
-    if (t >= L::kXStages && !(ok = wait(kBarXfree0 + st))) break;
+    const int st = t % kXStages;
+    if (t >= kXStages && !(ok = wait(kBarXfree0 + st))) break;
     mbar_expect_tx(&bars[kBarX0 + st], kHeads * kAtom);
 #pragma unroll
     for (int hh = 0; hh < kHeads; ++hh)
       tma_load_3d(smem + L::x + (st * kHeads + hh) * kAtom, tm_x, 0, h0 + hh, tok, &bars[kBarX0 + st]);
-    note(kBarX0 + st, (uint32_t)(t / L::kXStages) & 1u);
+    note(kBarX0 + st, (uint32_t)(t / kXStages) & 1u);
     if (!(ok = ring_load(tm_b, g, tok))) break;
     ++t;
     have = cursor_next(pb, rp, cur);
@@ -687,20 +733,20 @@ __device__ void mma_loop(const Problem& pb, uint8_t* smem, uint32_t tmem, uint64
       dc = at(k_major, a_c);
       db = at(k_major, a_b);
       dbm = at(mn_major, a_b);
-      dx = at(mn_major, smem_u32(smem + L::x + (t % L::kXStages) * kHeads * kAtom));
+      dx = at(mn_major, smem_u32(smem + L::x + (t % kXStages) * kHeads * kAtom));
       if (!state_only && !(ok = wait(kBarRing0 + c_slot))) break;
       if (!(ok = wait(kBarRing0 + b_slot))) break;
     }
-    if (state_only) {  // H += B^T [U_0 | U_1] onto h^
+    if (state_only) {  // H += B^T [U_0 | U_1] onto h^, U from buffer p & 1
       // the compute warps touch H only after a pass that ends a piece or before one that
       // starts or re-centres a state; only then does the product wait for them
       const bool touched = (prev_flags & (kPToFinal | kPToCarry)) || (flags & (kPPieceStart | kPRescaleAny));
       prev_flags = flags;
       if (touched && !(ok = wait(kBarHRead))) break;
-      if (!(ok = wait(kBarU))) break;
+      if (!(ok = wait(kBarU + (p & 1)))) break;
       tc_fence_after();
-      right_factor(dbm, dx);
-      commit(kBarSt);
+      right_factor(dbm, at(mn_major, smem_u32(smem + L::ub + (p & 1) * kHeads * kAtom)));
+      commit(kBarUFree0 + (p & 1));  // U buffer free, and H holds this pass
       if (flags & kPLast) commit(kBarRingFree0 + b_slot);
       issued_any = true;
       if (leader) mbar_arrive(&bars[kBarDescFree0 + ds]);
@@ -755,13 +801,11 @@ __device__ void mma_loop(const Problem& pb, uint8_t* smem, uint32_t tmem, uint64
     commit(kBarY);
     if (leader) mbar_arrive(&bars[kBarDescFree0 + ds]);
   }
-  if (!ok) {
-    *abort_flag = 1;
-    // every tcgen05.mma this warp issued completes before tensor memory is freed
-    if (issued_any) {
-      commit(kBarDrain);
-      mbar_wait_bounded(&bars[kBarDrain], 0, pb.wait_limit);
-    }
+  if (!ok) *abort_flag = 1;
+  // every tcgen05.mma this warp issued completes before tensor memory is freed
+  if (issued_any) {
+    commit(kBarDrain);
+    if (!mbar_wait_bounded(&bars[kBarDrain], 0, pb.wait_limit)) *abort_flag = 1;
   }
 }
 
@@ -794,18 +838,20 @@ __device__ __noinline__ void empty_unit_states(const Problem& pb, int hw, int ch
   for (int u = blockIdx.x; u < units; u += gridDim.x) {
     if (unit_tiles(pb, u) != 0) continue;
     const int64_t at = state_index(pb, u / pairs, (u % pairs) * kHeads + hw, ch, i);
-    for (int k = 0; k < 32; ++k) {
-      const int64_t o = at + (int64_t)k * pb.n_stride;
-      pb.final_state[o] = pb.init ? pb.init[o] : 0.f;
-    }
+    float v[32];  // every load in flight before the first store
+#pragma unroll
+    for (int k = 0; k < 32; ++k) v[k] = pb.init ? __ldg(pb.init + at + (int64_t)k * pb.n_stride) : 0.f;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) pb.final_state[at + (int64_t)k * pb.n_stride] = v[k];
   }
 }
 
-// The state at the start of the piece whose first pass d describes, into h: the
-// sequence's initial state (or zero), or the state CTA d.carry_src handed on (each warp
-// waits for the matching warp of that CTA).  False if that wait gave up.
+// The state at the start of the piece whose first pass d describes, times `scale`, into
+// tensor memory at t_state: the sequence's initial state (or zero), or the state CTA
+// d.carry_src handed on (each warp waits for the matching warp of that CTA).  Whole warp;
+// the values stay in registers, all 32 loads in flight at once.  False if the wait gave up.
 __device__ __noinline__ bool fetch_state(const Problem& pb, const PassDesc& d, int hw, int ch, int i, int wid,
-                                         volatile int* abort_flag, float* h) {
+                                         volatile int* abort_flag, uint32_t t_state, float scale) {
   const float* src = nullptr;
   int stride = pb.n_stride;
   if (d.flags & kPCarryIn) {
@@ -829,20 +875,32 @@ __device__ __noinline__ bool fetch_state(const Problem& pb, const PassDesc& d, i
     src = pb.init + state_index(pb, d.s, d.h0 + hw, ch, i);
   }
   if (!src || i >= pb.N) src = nullptr;
-  for (int k = 0; k < 32; ++k) h[k] = src ? __ldcg(src + (int64_t)k * stride) : 0.f;
+  float v[32];
+#pragma unroll
+  for (int k = 0; k < 32; ++k) v[k] = src ? __ldcg(src + (int64_t)k * stride) : 0.f;
+  uint32_t r[32];
+#pragma unroll
+  for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(v[k] * scale);
+  tmem_st32(t_state, r);
+  tmem_st_wait();
   return true;
 }
 
-// The state after the pass d describes (h = h_out) as the unit's final state or as the
-// hand-on to the next CTA (then released to it, one flag per warp).
+// The state after the pass d describes, h = scale H (H from tensor memory at t_state), as
+// the unit's final state or as the hand-on to the next CTA (then released to it, one flag
+// per warp).  Whole warp; the values stay in registers.
 __device__ __noinline__ void put_state(const Problem& pb, const PassDesc& d, int hw, int ch, int i, int wid,
-                                       const float* h) {
+                                       uint32_t t_state, float scale) {
+  uint32_t r[32];
+  tmem_ld32(t_state, r);
+  tmem_ld_wait();
   const bool to_final = d.flags & kPToFinal;
   if (i < pb.N) {
     float* dst = to_final ? pb.final_state + state_index(pb, d.s, d.h0 + hw, ch, i)
                           : pb.carry + carry_index(pb, blockIdx.x, hw, ch, i);
-    const int stride = to_final ? pb.n_stride : pb.N;
-    for (int k = 0; k < 32; ++k) dst[(int64_t)k * stride] = h[k];
+    const int64_t stride = to_final ? pb.n_stride : pb.N;
+#pragma unroll
+    for (int k = 0; k < 32; ++k) dst[k * stride] = __uint_as_float(r[k]) * scale;
   }
   if (!to_final) {
     __threadfence();
@@ -882,11 +940,19 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
     ph.flip(k);
     return true;
   };
-  // Final states only: the right factor of pass n completes phase n of kBarSt, and only the
-  // passes that end a piece or precede a re-centred / new state read H, so St is waited for
-  // by pass index.  A wait for phase n always comes before U(n + 1) is handed to the MMA
-  // warp, so the barrier is never two phases past it.
-  auto wait_st = [&](int n) -> bool { return warp_wait(&bars[kBarSt], (uint32_t)n & 1u, abort_flag, pb.wait_limit); };
+  // Final states only: the right factor of pass q completes phase q / 2 of U-free barrier
+  // q & 1.  Each phase is waited for once, in order: before U(q + 2) is written into the
+  // buffer, or earlier, where pass q ends a piece or precedes a re-centred / new state and
+  // H is read.  Either wait comes after this warp's wait for phase q / 2 - 1 and before it
+  // hands U(q + 2) to the MMA warp, so the barrier is never a phase behind or two past it.
+  int uf_waited[2] = {0, 0};  // phases of U-free barrier b this warp has waited for
+  auto wait_uf = [&](int q) -> bool {
+    const int b = q & 1, k = q >> 1;
+    if (uf_waited[b] > k) return true;
+    if (!warp_wait(&bars[kBarUFree0 + b], (uint32_t)k & 1u, abort_flag, pb.wait_limit)) return false;
+    uf_waited[b] = k + 1;
+    return true;
+  };
 
   empty_unit_states(pb, hw, ch, i);
 
@@ -910,13 +976,14 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
   // tensor memory and r.  False if fetching the initial state gave up.
   auto install = [&](const PassDesc& d, float sig_prev, uint32_t (&r)[32]) -> bool {
     if (d.flags & kPPieceStart) {
-      float h[32];
-      if (!fetch_state(pb, d, hw, ch, i, wid, abort_flag, h)) return false;
-#pragma unroll
-      for (int k = 0; k < 32; ++k) r[k] = __float_as_uint(h[k]);
-    } else {
-      scale32(r, sig_prev);
+      if (!fetch_state(pb, d, hw, ch, i, wid, abort_flag, t_state, d.sig_in[hw])) return false;
+      if (!state_only) {  // r: the installed H, for its bf16 copy
+        tmem_ld32(t_state, r);
+        tmem_ld_wait();
+      }
+      return true;
     }
+    scale32(r, sig_prev);
     scale32(r, d.sig_in[hw]);
     tmem_st32(t_state, r);
     tmem_st_wait();
@@ -943,13 +1010,11 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
     const PassDesc& d = descs[ds];
     const int flags = d.flags;
     if (flags & kPFirst) ++t;
-    const int st = t % L::kXStages;
+    const int st = t % kXStages;
     uint8_t* sxh = sx + (st * kHeads + hw) * kAtom;
 
-    // ---- U = u_i x_i over the tile's x, in place (x itself stays in registers)
-    if constexpr (state_only) {  // a later pass of a tile rewrites U in place: the last product is done with it
-      if (!(flags & kPFirst) && !wait_st(p - 1)) return;
-    }
+    // ---- U = u_i x_i over the tile's x, in place (x itself stays in registers); with
+    // final states only, into U buffer p & 1 once the right factor of pass p - 2 has read it
     if (flags & kPFirst) {
       if (!wait(kBarX0 + st)) return;
 #pragma unroll
@@ -957,6 +1022,12 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
         const uint4 v = *reinterpret_cast<const uint4*>(sxh + sw128_off(i, 4 * ch + c));
         xr[4 * c] = v.x, xr[4 * c + 1] = v.y, xr[4 * c + 2] = v.z, xr[4 * c + 3] = v.w;
       }
+      if (state_only) warp_arrive(&bars[kBarXfree0 + st]);  // x is in registers: the stage may refill
+    }
+    uint8_t* suh = sxh;
+    if constexpr (state_only) {
+      suh = smem + L::ub + ((p & 1) * kHeads + hw) * kAtom;
+      if (p >= 2 && !wait_uf(p - 2)) return;
     }
     {
       const float u = d.u[hw][i];
@@ -968,19 +1039,18 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
         v.y = mul_bf16x2(xr[4 * c + 1], u2);
         v.z = mul_bf16x2(xr[4 * c + 2], u2);
         v.w = mul_bf16x2(xr[4 * c + 3], u2);
-        *reinterpret_cast<uint4*>(sxh + sw128_off(i, 4 * ch + c)) = v;
+        *reinterpret_cast<uint4*>(suh + sw128_off(i, 4 * ch + c)) = v;
       }
     }
-    if constexpr (state_only) {  // the previous tile's right factor is done with its x stage
-      if ((flags & kPFirst) && p > 0 && !wait_st(p - 1)) return;
-    }
+    // (final states only: one barrier per buffer, so an arrival for pass p + 1 never counts
+    // toward pass p; one for pass p + 2 comes after the right factor of pass p)
     fence_proxy_async();
-    warp_arrive(&bars[kBarU]);
+    warp_arrive(&bars[kBarU + (state_only ? (p & 1) : 0)]);
 
-    if ((flags & kPFirst) && t > 0) {
+    if ((flags & kPFirst) && t > 0 && !state_only) {
       // the previous tile's x stage: its y store has read it, so it may take tile t + 1's x
       if (staged_prev && ch == 0 && lane == 0) bulk_wait_read();
-      warp_arrive(&bars[kBarXfree0 + (st + L::kXStages - 1) % L::kXStages]);
+      warp_arrive(&bars[kBarXfree0 + (st + kXStages - 1) % kXStages]);
     }
     // ---- P = bf16(S) on and below the diagonal, written in place over S: block (q, kb)
     // is kept whole below the diagonal (kb < q), lower-triangular on it, zero above
@@ -1024,19 +1094,14 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
       // "H read": then no warp can arrive for the next such pass while another has not yet
       // arrived for this one, and the MMA warp waits for it on exactly these passes.
       if (touched) {
-        if (!wait_st(p)) return;
+        if (!wait_uf(p)) return;
         tc_fence_after();
-        if (out || reset) {
+        if (out) put_state(pb, d, hw, ch, i, wid, t_state, d.sig_out[hw]);
+        if (reset) {
           uint32_t r[32];
           tmem_ld32(t_state, r);
           tmem_ld_wait();
-          if (out) {
-            float h[32];
-#pragma unroll
-            for (int k = 0; k < 32; ++k) h[k] = __uint_as_float(r[k]) * d.sig_out[hw];
-            put_state(pb, d, hw, ch, i, wid, h);
-          }
-          if (reset && !install(dn, d.sig_out[hw], r)) return;
+          if (!install(dn, d.sig_out[hw], r)) return;
         }
         tc_fence_before();
         warp_arrive(&bars[kBarHRead]);
@@ -1051,15 +1116,10 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
     tc_fence_after();
     bool more;
     {
+      if (flags & (kPToFinal | kPToCarry)) put_state(pb, d, hw, ch, i, wid, t_state, d.sig_out[hw]);
       uint32_t r[32];
       tmem_ld32(t_state, r);
       tmem_ld_wait();
-      if (flags & (kPToFinal | kPToCarry)) {
-        float h[32];
-#pragma unroll
-        for (int k = 0; k < 32; ++k) h[k] = __uint_as_float(r[k]) * d.sig_out[hw];
-        put_state(pb, d, hw, ch, i, wid, h);
-      }
       if (!wait(kBarDescFull0 + nds)) return;
       const PassDesc& dn = descs[nds];
       more = !(dn.flags & kPEnd);
@@ -1379,10 +1439,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     tmem_relinquish();
   }
   if (tid == 0) {
-    for (int k = 0; k < L::kXStages; ++k) {
+    for (int k = 0; k < kXStages; ++k) {
       mbar_init(&bars[kBarX0 + k], 1);
       mbar_init(&bars[kBarXfree0 + k], kComputeWarps);
     }
+    for (int k = 0; k < 2; ++k) mbar_init(&bars[kBarUFree0 + k], 1);
     for (int k = 0; k < 2; ++k) {
       mbar_init(&bars[kBarS0 + k], 1);
       mbar_init(&bars[kBarP0 + k], kComputeWarps);
@@ -1394,6 +1455,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&bars[kBarSt], 1);
     mbar_init(&bars[kBarY], 1);
     mbar_init(&bars[kBarU], kComputeWarps);
+    mbar_init(&bars[kBarU1], kComputeWarps);
     mbar_init(&bars[kBarHt], kComputeWarps);
     mbar_init(&bars[kBarHRead], kComputeWarps);
     mbar_init(&bars[kBarFree], kComputeWarps);
@@ -1416,7 +1478,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = s_tmem_base;
-  const RangePlan rp = split_work(pb, reinterpret_cast<SplitScratch*>(smem + L::x));
+  // the split's weights (the second column half of N = 256 reuses the first launch's)
+  // the split's weights: from tile_weight_kernel or the first column half of N = 256, or
+  // here (CTA r weighs sequence tiles r, r + R, ...; few per CTA) and a barrier
+  bool weights_ok = true;
+  if (!pb.weights_ready) {
+    const int64_t seqtiles = seq_tile0(pb, pb.nseq);
+    for (int64_t st = blockIdx.x; st < seqtiles; st += gridDim.x)
+      weigh_tile<kThreads>(pb, st, reinterpret_cast<float4*>(smem + L::x));
+    weights_ok = weights_barrier(pb, abort_flag);
+  }
+  const RangePlan rp = weights_ok ? split_work(pb, reinterpret_cast<SplitScratch*>(smem + L::x)) : RangePlan{};
 
   if (warp == kMmaWarp) {
     mma_loop<NS, MODE>(pb, smem, tmem, bars, abort_flag);
@@ -1572,24 +1644,26 @@ bool tc_supports(const ssd_shape* s, int chunk) {
   return tokens >= 1 && tokens < ((int64_t)1 << 31) - kTile;
 }
 
-cudaError_t launch_tc(const Problem& pb, cudaStream_t st) {
-  // the tiles' weights for the work split (once: both column halves of N = 256 share them)
-  {
-    const int64_t seqtiles = pb.cu ? (pb.tokens + kTile - 1) / kTile + pb.nseq : (int64_t)pb.nseq * pb.dense_tiles;
-    const int grid = (int)(seqtiles < 8 * kMaxRanges ? seqtiles : 8 * kMaxRanges);
-    if (grid > 0) {
-      // the fused kernel's shared-memory carve-out, so the SMs need not switch between the launches
-      static std::atomic<uint64_t> carve{0};
-      int dev = 0;
-      if (cudaGetDevice(&dev) == cudaSuccess && dev < 64 && !(carve.load() & (1ull << dev))) {
-        cudaFuncSetAttribute(tile_weight_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
-        carve.fetch_or(1ull << dev);
-      }
-      tile_weight_kernel<<<grid, kWeightThreads, tile_weight_smem(pb.H), st>>>(pb);
-      count_launches(1);
-      const cudaError_t e = cudaGetLastError();
-      if (e != cudaSuccess) return e;
+cudaError_t launch_tc(const Problem& pb_in, cudaStream_t st) {
+  // The split's weights: each CTA weighs its share of the sequence tiles before the split,
+  // unless there are more than two per CTA; then a kernel of their own, with many tiles in
+  // flight per SM, weighs them first.
+  Problem pb = pb_in;
+  const int64_t seqtiles = pb.cu ? (pb.tokens + kTile - 1) / kTile + pb.nseq : (int64_t)pb.nseq * pb.dense_tiles;
+  if (seqtiles > 2 * (int64_t)pb.ranges) {
+    const int grid = (int)(seqtiles < 32 * kMaxRanges ? seqtiles : 32 * kMaxRanges);
+    // the fused kernel's shared-memory carve-out, so the SMs need not switch between the launches
+    static std::atomic<uint64_t> carve{0};
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && dev < 64 && !(carve.load() & (1ull << dev))) {
+      cudaFuncSetAttribute(tile_weight_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+      carve.fetch_or(1ull << dev);
     }
+    tile_weight_kernel<<<grid, kWeightThreads, 0, st>>>(pb);
+    count_launches(1);
+    const cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
+    pb.weights_ready = 1;
   }
   if (pb.N <= 128) {
     Problem q = pb;
@@ -1604,6 +1678,7 @@ cudaError_t launch_tc(const Problem& pb, cudaStream_t st) {
   a.n_stride = b.n_stride = pb.N;
   a.n_off = 0, b.n_off = 128;
   a.y_accum = 0, b.y_accum = pb.y != nullptr;
+  b.weights_ready = 1;  // the first launch wrote the split's weights
   b.D = nullptr;
   a.prof_stop = nullptr, b.prof_start = nullptr;
   b.epoch = pb.epoch ^ 0x8000000000000000ull;  // a value no other launch's flags hold
