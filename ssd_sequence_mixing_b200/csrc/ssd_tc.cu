@@ -65,10 +65,12 @@ constexpr int kTile = 128;          // tokens per tile (UMMA M)
 constexpr int kHeadDim = 64;        // P supported by this path
 constexpr int kHeads = 2;           // heads of one B/C group processed together
 constexpr int kComputeWarps = 16;   // (head, column half, lane quarter)
-constexpr int kMmaWarp = kComputeWarps, kLoadWarp = kComputeWarps + 1, kHelperWarp = kComputeWarps + 2;
-constexpr int kThreads = (kComputeWarps + 3) * 32;
+constexpr int kMmaWarp = kComputeWarps, kLoadWarp = kComputeWarps + 1, kHelperWarp = kComputeWarps + 2,
+              kScanWarp = kComputeWarps + 3;
+constexpr int kThreads = (kComputeWarps + 4) * 32;
 constexpr int kDescSlots = 3;  // pass descriptors the helper may run ahead
 constexpr int kDtStages = 4;   // dt tiles in flight
+constexpr int kScanSlots = 2;  // (final states only) tiles the scan warp has handed to the helper
 constexpr int kRing = 3;       // B / C tiles in shared memory (C(t), B(t) and the next one)
 constexpr int kXStages = 2;    // x tiles in shared memory
 constexpr int kMaxRanges = 1024;  // CTAs of one launch (one per SM)
@@ -104,7 +106,9 @@ enum {
   kBarDescFull0 = kBarDt0 + kDtStages,           // kDescSlots: descriptor written (helper)
   kBarDescFree0 = kBarDescFull0 + kDescSlots,    // kDescSlots: used up (16 compute + MMA)
   kBarPair0 = kBarDescFree0 + kDescSlots,        // 8: column-half-1 warp of (head, quarter) staged its y
-  kNumBars = kBarPair0 + kHeads * 4
+  kBarScanFull0 = kBarPair0 + kHeads * 4,        // kScanSlots: a tile's dt and cumsum written (scan warp)
+  kBarScanFree0 = kBarScanFull0 + kScanSlots,    // kScanSlots: the helper is done with the slot
+  kNumBars = kBarScanFree0 + kScanSlots
 };
 static_assert(kNumBars <= 64, "phase bits of a 64-bit mask");
 // every group of barriers has its own slots: the next group starts past its last one
@@ -143,6 +147,14 @@ struct PassDesc {
   float r[kHeads][kTile];  // 2^(c_i - m) on the pass's rows, else 0
 };
 constexpr uint32_t kDescBytes = (sizeof(PassDesc) + 127) / 128 * 128;
+// One tile's c (inclusive cumsum of dt A in log2 units from the tile start) and dt of both
+// heads, rows past the tile's end zero.  With y the helper keeps c of the current tile in
+// the first slot; with final states only the scan warp hands the helper a ring of them.
+struct ScanTile {
+  float c[kHeads][kTile];
+  float dt[kHeads][kTile];
+};
+constexpr uint32_t kScanBytes = sizeof(ScanTile);
 
 // Shared memory.  The final-state-only variant (no C, no y, no state copy) spends what
 // those take on two U buffers of its own: x is read into registers and its stage released
@@ -162,8 +174,8 @@ struct Layout {
   // final-state-only variant a pad of one atom, so the read stays inside the CTA's memory.
   static constexpr uint32_t kHtBytes = kStateOnly ? (NS == 64 ? kAtom : 0) : kHeads * NS * 128;
   static constexpr uint32_t desc = ht + kHtBytes;                   // PassDesc[kDescSlots]
-  static constexpr uint32_t scan = desc + kDescSlots * kDescBytes; // helper: c[2][128]
-  static constexpr uint32_t sdt = scan + kHeads * kTile * 4;       // float[stage][128 tok][4 heads]
+  static constexpr uint32_t scan = desc + kDescSlots * kDescBytes; // ScanTile[kScanSlots]
+  static constexpr uint32_t sdt = scan + kScanSlots * kScanBytes;  // float[stage][128 tok][4 heads]
   static constexpr uint32_t bars = sdt + kDtStages * kTile * 16;   // uint64[kNumBars]
   static constexpr uint32_t flag = bars + kNumBars * 8;            // int: a wait gave up
   static constexpr uint32_t bytes = flag + 16;
@@ -251,47 +263,49 @@ __device__ __noinline__ RangePlan plan_of(const Problem& pb, int64_t w0, int64_t
   return rp;
 }
 
-// Loads piece `pi` (processing order) into c; false when it has no tiles.
-__device__ __noinline__ bool load_piece(const Problem& pb, const RangePlan& rp, int pi, TileCursor& c) {
-  int u, kb, ke;
-  if (rp.npieces == 1) {
-    u = rp.u0, kb = rp.k0, ke = rp.ke1;
-  } else if (pi == 0) {  // the truncated last piece first
-    u = rp.u1, kb = 0, ke = rp.ke1;
-  } else if (pi < rp.npieces - 1) {  // whole units
-    u = rp.u0 + pi, kb = 0, ke = unit_tiles(pb, rp.u0 + pi);
-  } else {  // the first piece last: it may need the previous CTA's state
-    u = rp.u0, kb = rp.k0, ke = unit_tiles(pb, rp.u0);
+// The cursor at the first tile of the first piece pi' >= pi (processing order) that has
+// tiles, or one with piece = -1 when there is none.  Everything is passed and returned by
+// value, so the callers' cursors stay in registers.
+__device__ __noinline__ TileCursor cursor_from(const Problem& pb, RangePlan rp, int pi) {
+  TileCursor c{};
+  c.piece = -1;
+  for (; pi < rp.npieces; ++pi) {
+    int u, kb, ke;
+    if (rp.npieces == 1) {
+      u = rp.u0, kb = rp.k0, ke = rp.ke1;
+    } else if (pi == 0) {  // the truncated last piece first
+      u = rp.u1, kb = 0, ke = rp.ke1;
+    } else if (pi < rp.npieces - 1) {  // whole units
+      u = rp.u0 + pi, kb = 0, ke = unit_tiles(pb, rp.u0 + pi);
+    } else {  // the first piece last: it may need the previous CTA's state
+      u = rp.u0, kb = rp.k0, ke = unit_tiles(pb, rp.u0);
+    }
+    if (ke <= kb) continue;
+    const int s = u / (pb.H / kHeads);
+    c.unit = u;
+    c.tb = (int)seq_off(pb, s);
+    c.len = (int)(seq_off(pb, s + 1) - c.tb);
+    c.k0 = kb * kTile;
+    c.kend = min(ke * kTile, c.len);
+    c.piece = pi;
+    const bool unit_end = ke == unit_tiles(pb, u);
+    c.flags = (kb > 0 ? kCarryIn : 0) | (unit_end ? kUnitEnd : kCarryOut);
+    return c;
   }
-  if (ke <= kb) return false;
-  const int pairs = pb.H / kHeads;
-  const int s = u / pairs;
-  c.unit = u;
-  c.tb = (int)seq_off(pb, s);
-  c.len = (int)(seq_off(pb, s + 1) - c.tb);
-  c.k0 = kb * kTile;
-  c.kend = min(ke * kTile, c.len);
-  c.piece = pi;
-  const bool unit_end = ke == unit_tiles(pb, u);
-  c.flags = (kb > 0 ? kCarryIn : 0) | (unit_end ? kUnitEnd : kCarryOut);
-  return true;
-}
-
-__device__ __noinline__ bool cursor_from(const Problem& pb, const RangePlan& rp, int pi, TileCursor& c) {
-  for (; pi < rp.npieces; ++pi)
-    if (load_piece(pb, rp, pi, c)) return true;
-  return false;
+  return c;
 }
 
 __device__ __forceinline__ bool cursor_first(const Problem& pb, const RangePlan& rp, TileCursor& c) {
-  return cursor_from(pb, rp, 0, c);
+  c = cursor_from(pb, rp, 0);
+  return c.piece >= 0;
 }
 
 // Advances to the next tile of this CTA's range; false when done.
 __device__ __forceinline__ bool cursor_next(const Problem& pb, const RangePlan& rp, TileCursor& c) {
   c.k0 += kTile;
   if (c.k0 < c.kend) return true;
-  return cursor_from(pb, rp, c.piece + 1, c);
+  c = cursor_from(pb, rp, c.piece + 1);
+  return c.piece >= 0;
 }
 
 // One arrival for the whole warp, after every lane's prior work (the lanes' own fences
@@ -583,7 +597,7 @@ __device__ __noinline__ void weigh_tile(const Problem& pb, int64_t st, float4* p
 // The weights of problems with many sequence tiles per SM, ahead of the fused kernel: one
 // block per sequence tile, several resident per SM, so the dt loads of many tiles overlap.
 constexpr int kWeightThreads = 512;
-__global__ void __launch_bounds__(kWeightThreads) tile_weight_kernel(Problem pb) {
+__global__ void __launch_bounds__(kWeightThreads) tile_weight_kernel(const __grid_constant__ Problem pb) {
   __shared__ float4 part[kWeightThreads];
   if (pb.cu && *pb.nchunks < 0) return;  // cu_seqlens rejected by the table kernel
   const int64_t seqtiles = seq_tile0(pb, pb.nseq);
@@ -1195,6 +1209,145 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
   }
 }
 
+// ------------------------------------------------------------------ scan warp
+// With final states only, a warp of its own loads each tile's dt by TMA into a ring
+// (kDtStages tiles in flight) and hands the helper both heads' dt and c, the inclusive
+// cumsum of dt A in log2 units from the tile start, through a ring of kScanSlots.
+struct ScanState {
+  TileCursor ahead, cur;  // dt loads run up to kDtStages tiles ahead on a cursor of their own
+  bool have_ahead, have;
+  int dt_issued, t, a_unit;
+  float a2[kHeads];  // A log2(e) of the current unit's heads
+  Phases ph;         // dt barriers (and, in the scan warp, the slots' barriers)
+};
+
+template <int NS, int MODE>
+__device__ __forceinline__ void scan_issue_dt(ScanState& S, const CUtensorMap* tm_dt, const Problem& pb,
+                                              const RangePlan& rp, uint8_t* smem, uint64_t* bars) {
+  using L = Layout<NS, MODE>;
+  if ((threadIdx.x & 31) == 0) {
+    const int st = S.dt_issued % kDtStages;
+    const int h0 = (S.ahead.unit % (pb.H / kHeads)) * kHeads;
+    mbar_expect_tx(&bars[kBarDt0 + st], kTile * 16);
+    tma_load_2d(smem + L::sdt + st * kTile * 16, tm_dt, h0 & ~3, S.ahead.tb + S.ahead.k0, &bars[kBarDt0 + st]);
+  }
+  ++S.dt_issued;
+  S.have_ahead = cursor_next(pb, rp, S.ahead);
+}
+
+template <int NS, int MODE>
+__device__ void scan_init(ScanState& S, const CUtensorMap* tm_dt, const Problem& pb, const RangePlan& rp,
+                          uint8_t* smem, uint64_t* bars) {
+  S.have_ahead = cursor_first(pb, rp, S.ahead);
+  S.have = cursor_first(pb, rp, S.cur);
+  S.dt_issued = S.t = 0;
+  S.a_unit = -1;
+  S.a2[0] = S.a2[1] = 0.f;
+  for (int k = 0; k < kDtStages && S.have_ahead; ++k) scan_issue_dt<NS, MODE>(S, tm_dt, pb, rp, smem, bars);
+}
+
+// The scan step of tile S.t (S.have): lane's rows 4 lane .. 4 lane + 3 of c and dt into
+// cth and dtt, c also into o.c and, if `with_dt`, dt into o.dt; then on to the next tile.
+// Whole warp; false if the dt wait gave up.
+template <int NS, int MODE>
+__device__ __forceinline__ bool scan_tile(ScanState& S, float (&cth)[kHeads][4], float (&dtt)[kHeads][4],
+                                          ScanTile& o, bool with_dt, const CUtensorMap* tm_dt, const Problem& pb,
+                                          const RangePlan& rp, uint8_t* smem, uint64_t* bars,
+                                          volatile int* abort_flag) {
+  using L = Layout<NS, MODE>;
+  const int lane = threadIdx.x & 31;
+  const TileCursor& cur = S.cur;
+  const int h0 = (cur.unit % (pb.H / kHeads)) * kHeads;
+  if (cur.unit != S.a_unit) {
+    S.a_unit = cur.unit;
+#pragma unroll
+    for (int hh = 0; hh < kHeads; ++hh) S.a2[hh] = pb.A[h0 + hh] * 1.4426950408889634f;  // log2 units
+  }
+  const int rem = min(kTile, cur.len - cur.k0);
+  const int dst = S.t % kDtStages;
+  if (!warp_wait(&bars[kBarDt0 + dst], S.ph.parity(kBarDt0 + dst), abort_flag, pb.wait_limit)) return false;
+  S.ph.flip(kBarDt0 + dst);
+  // row 4 lane + j holds the 4 heads' dt of one token; a lane reads its rows in the order
+  // j = (k + rot) & 3, rot = (lane / 2) & 3, so each quarter warp's 16-byte loads fall in
+  // distinct banks
+  {
+    const float4* rows = reinterpret_cast<const float4*>(smem + L::sdt + dst * kTile * 16) + 4 * lane;
+    const int rot = (lane >> 1) & 3, c0 = h0 & 3;  // the pair's first column in the 4-head row
+    float v0[4], v1[4];
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float4 qv = rows[(k + rot) & 3];
+      v0[k] = c0 == 0 ? qv.x : qv.z;
+      v1[k] = c0 == 0 ? qv.y : qv.w;
+    }
+    const int left = rem - 4 * lane;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {  // token j came in as k = (j - rot) & 3
+      const int k = (j - rot) & 3;
+      const float x0 = k == 0 ? v0[0] : k == 1 ? v0[1] : k == 2 ? v0[2] : v0[3];
+      const float x1 = k == 0 ? v1[0] : k == 1 ? v1[1] : k == 2 ? v1[2] : v1[3];
+      dtt[0][j] = j < left ? dt_of(pb, x0, h0) : 0.f;
+      dtt[1][j] = j < left ? dt_of(pb, x1, h0 + 1) : 0.f;
+    }
+  }
+  // the dt stage is read: refill it
+  __syncwarp();
+  if (S.have_ahead) scan_issue_dt<NS, MODE>(S, tm_dt, pb, rp, smem, bars);
+#pragma unroll
+  for (int hh = 0; hh < kHeads; ++hh) {
+    const float a2 = S.a2[hh];
+    float c0 = dtt[hh][0] * a2, c1 = c0 + dtt[hh][1] * a2, c2 = c1 + dtt[hh][2] * a2, c3 = c2 + dtt[hh][3] * a2;
+    float v = c3;
+#pragma unroll
+    for (int k = 1; k < 32; k <<= 1) {
+      const float u = __shfl_up_sync(0xffffffffu, v, k);
+      if (lane >= k) v += u;
+    }
+    const float base = v - c3;  // cumsum before token 4 lane
+    cth[hh][0] = c0 + base, cth[hh][1] = c1 + base, cth[hh][2] = c2 + base, cth[hh][3] = c3 + base;
+    reinterpret_cast<float4*>(o.c[hh])[lane] = make_float4(cth[hh][0], cth[hh][1], cth[hh][2], cth[hh][3]);
+    if (with_dt)
+      reinterpret_cast<float4*>(o.dt[hh])[lane] = make_float4(dtt[hh][0], dtt[hh][1], dtt[hh][2], dtt[hh][3]);
+  }
+  __syncwarp();
+  ++S.t;
+  S.have = cursor_next(pb, rp, S.cur);
+  return true;
+}
+
+// After a failure: the dt loads still in flight land before the CTA ends (bounded).
+__device__ __forceinline__ void scan_drain(const ScanState& S, const Problem& pb, uint64_t* bars) {
+  if ((threadIdx.x & 31) == 0)
+    for (int n = S.t; n < S.dt_issued; ++n)
+      mbar_wait_bounded(&bars[kBarDt0 + n % kDtStages], (n / kDtStages) & 1, pb.wait_limit);
+}
+
+// The scan warp (final states only, whose compute warps wait for the helper): the scan
+// step, kScanSlots tiles ahead of the helper.
+template <int NS, int MODE>
+__device__ void scan_loop(const CUtensorMap* tm_dt, const Problem& pb, const RangePlan& rp, uint8_t* smem,
+                          uint64_t* bars, volatile int* abort_flag) {
+  using L = Layout<NS, MODE>;
+  ScanTile* ring = reinterpret_cast<ScanTile*>(smem + L::scan);
+  ScanState S;
+  scan_init<NS, MODE>(S, tm_dt, pb, rp, smem, bars);
+  bool ok = true;
+  while (S.have) {
+    const int slot = S.t % kScanSlots, k = kBarScanFree0 + slot;
+    if (S.t >= kScanSlots) {
+      if (!(ok = warp_wait(&bars[k], S.ph.parity(k), abort_flag, pb.wait_limit))) break;
+      S.ph.flip(k);
+    }
+    float cth[kHeads][4], dtt[kHeads][4];
+    if (!(ok = scan_tile<NS, MODE>(S, cth, dtt, ring[slot], true, tm_dt, pb, rp, smem, bars, abort_flag))) break;
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&bars[kBarScanFull0 + slot]);
+  }
+  if (!ok) {
+    *abort_flag = 1;
+    scan_drain(S, pb, bars);
+  }
+}
+
 // ------------------------------------------------------------------ helper warp
 // The helper walks the CTA's tile sequence ahead of the compute warps, loads each
 // tile's dt by TMA into a ring of its own (kDtStages tiles in flight), and writes one
@@ -1202,7 +1355,8 @@ __device__ void compute_loop(const CUtensorMap* tm_y32, const Problem& pb, uint8
 // factors u and r of both heads, the state scalings and the piece flags.  Per tile it
 // forms c (the inclusive cumsum of dt A in log2 units from the tile start, both heads),
 // keeps or re-centres each head's reference and cuts the valid rows into passes: one
-// pass unless a head decays by more than 2^-(2 kRangeHalf) across the tile.
+// pass unless a head decays by more than 2^-(2 kRangeHalf) across the tile.  With final
+// states only, dt and c come from the scan warp instead.
 template <int NS, int MODE>
 __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, const RangePlan& rp, uint8_t* smem,
                             uint64_t* bars, volatile int* abort_flag) {
@@ -1233,7 +1387,10 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, const R
     ++dt_issued;
     have_ahead = cursor_next(pb, rp, ahead);
   };
+  constexpr bool from_scan = MODE == kModeState;  // dt and c from the scan warp
+  if (from_scan) have_ahead = false;
   for (int k = 0; k < kDtStages && have_ahead; ++k) issue_dt();
+  const ScanTile* ring = reinterpret_cast<const ScanTile*>(smem + L::scan);
 
   TileCursor cur;
   bool have = cursor_first(pb, rp, cur);
@@ -1279,51 +1436,64 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, const R
     }
     const int rem = min(kTile, cur.len - cur.k0);
 
-    // this tile's dt: row 4 lane + j holds the 4 heads' dt of one token; a lane reads its
-    // rows in the order j = (k + rot) & 3, rot = (lane / 2) & 3, so each quarter warp's
-    // 16-byte loads fall in distinct banks
-    if (!(ok = wait(kBarDt0 + t % kDtStages))) break;
-    float dtt[kHeads][4];
-    {
-      const float4* rows = reinterpret_cast<const float4*>(sdt + (t % kDtStages) * kTile * 16) + 4 * lane;
-      const int rot = (lane >> 1) & 3, c0 = h0 & 3;  // the pair's first column in the 4-head row
-      float v0[4], v1[4];
+    float dtt[kHeads][4], cth[kHeads][4];
+    const float* sct = sc;  // c[head][128] of this tile
+    const int sslot = t % kScanSlots;
+    if constexpr (from_scan) {  // lane: rows 4 lane .. 4 lane + 3
+      if (!(ok = wait(kBarScanFull0 + sslot))) break;
+      sct = ring[sslot].c[0];
 #pragma unroll
-      for (int k = 0; k < 4; ++k) {
-        const float4 qv = rows[(k + rot) & 3];
-        v0[k] = c0 == 0 ? qv.x : qv.z;
-        v1[k] = c0 == 0 ? qv.y : qv.w;
+      for (int hh = 0; hh < kHeads; ++hh) {
+        const float4 cv = reinterpret_cast<const float4*>(ring[sslot].c[hh])[lane];
+        const float4 dv = reinterpret_cast<const float4*>(ring[sslot].dt[hh])[lane];
+        cth[hh][0] = cv.x, cth[hh][1] = cv.y, cth[hh][2] = cv.z, cth[hh][3] = cv.w;
+        dtt[hh][0] = dv.x, dtt[hh][1] = dv.y, dtt[hh][2] = dv.z, dtt[hh][3] = dv.w;
       }
-      const int left = rem - 4 * lane;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {  // token j came in as k = (j - rot) & 3
-        const int k = (j - rot) & 3;
-        const float x0 = k == 0 ? v0[0] : k == 1 ? v0[1] : k == 2 ? v0[2] : v0[3];
-        const float x1 = k == 0 ? v1[0] : k == 1 ? v1[1] : k == 2 ? v1[2] : v1[3];
-        dtt[0][j] = j < left ? dt_of(pb, x0, h0) : 0.f;
-        dtt[1][j] = j < left ? dt_of(pb, x1, h0 + 1) : 0.f;
+    } else {
+      // this tile's dt: row 4 lane + j holds the 4 heads' dt of one token; a lane reads its
+      // rows in the order j = (k + rot) & 3, rot = (lane / 2) & 3, so each quarter warp's
+      // 16-byte loads fall in distinct banks
+      if (!(ok = wait(kBarDt0 + t % kDtStages))) break;
+      {
+        const float4* rows = reinterpret_cast<const float4*>(sdt + (t % kDtStages) * kTile * 16) + 4 * lane;
+        const int rot = (lane >> 1) & 3, c0 = h0 & 3;  // the pair's first column in the 4-head row
+        float v0[4], v1[4];
+  #pragma unroll
+        for (int k = 0; k < 4; ++k) {
+          const float4 qv = rows[(k + rot) & 3];
+          v0[k] = c0 == 0 ? qv.x : qv.z;
+          v1[k] = c0 == 0 ? qv.y : qv.w;
+        }
+        const int left = rem - 4 * lane;
+  #pragma unroll
+        for (int j = 0; j < 4; ++j) {  // token j came in as k = (j - rot) & 3
+          const int k = (j - rot) & 3;
+          const float x0 = k == 0 ? v0[0] : k == 1 ? v0[1] : k == 2 ? v0[2] : v0[3];
+          const float x1 = k == 0 ? v1[0] : k == 1 ? v1[1] : k == 2 ? v1[2] : v1[3];
+          dtt[0][j] = j < left ? dt_of(pb, x0, h0) : 0.f;
+          dtt[1][j] = j < left ? dt_of(pb, x1, h0 + 1) : 0.f;
+        }
       }
+      // the dt stage is read: refill it
+      __syncwarp();
+      if (have_ahead) issue_dt();
+      // inclusive cumsum c of dt A (log2 units) from the tile start, both heads
+  #pragma unroll
+      for (int hh = 0; hh < kHeads; ++hh) {
+        float c0 = dtt[hh][0] * a2[hh], c1 = c0 + dtt[hh][1] * a2[hh], c2 = c1 + dtt[hh][2] * a2[hh],
+              c3 = c2 + dtt[hh][3] * a2[hh];
+        float v = c3;
+  #pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const float u = __shfl_up_sync(0xffffffffu, v, o);
+          if (lane >= o) v += u;
+        }
+        const float base = v - c3;  // cumsum before token 4 lane
+        cth[hh][0] = c0 + base, cth[hh][1] = c1 + base, cth[hh][2] = c2 + base, cth[hh][3] = c3 + base;
+        reinterpret_cast<float4*>(sc + hh * kTile)[lane] = make_float4(cth[hh][0], cth[hh][1], cth[hh][2], cth[hh][3]);
+      }
+      __syncwarp();
     }
-    // the dt stage is read: refill it
-    __syncwarp();
-    if (have_ahead) issue_dt();
-    // inclusive cumsum c of dt A (log2 units) from the tile start, both heads
-    float cth[kHeads][4];
-#pragma unroll
-    for (int hh = 0; hh < kHeads; ++hh) {
-      float c0 = dtt[hh][0] * a2[hh], c1 = c0 + dtt[hh][1] * a2[hh], c2 = c1 + dtt[hh][2] * a2[hh],
-            c3 = c2 + dtt[hh][3] * a2[hh];
-      float v = c3;
-#pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        const float u = __shfl_up_sync(0xffffffffu, v, o);
-        if (lane >= o) v += u;
-      }
-      const float base = v - c3;  // cumsum before token 4 lane
-      cth[hh][0] = c0 + base, cth[hh][1] = c1 + base, cth[hh][2] = c2 + base, cth[hh][3] = c3 + base;
-      reinterpret_cast<float4*>(sc + hh * kTile)[lane] = make_float4(cth[hh][0], cth[hh][1], cth[hh][2], cth[hh][3]);
-    }
-    __syncwarp();
 
     // passes over rows [0, rem).  A head keeps its reference m (sg[hh] = m - c_before(lo),
     // carried over from the pass before) while every remaining row stays within
@@ -1335,8 +1505,8 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, const R
       bool keep[kHeads];
 #pragma unroll
       for (int hh = 0; hh < kHeads; ++hh) {
-        c0[hh] = lo > 0 ? sc[hh * kTile + lo - 1] : 0.f;
-        clo[hh] = sc[hh * kTile + lo];
+        c0[hh] = lo > 0 ? sct[hh * kTile + lo - 1] : 0.f;
+        clo[hh] = sct[hh * kTile + lo];
         bool out = piece_start;
 #pragma unroll
         for (int j = 0; j < 4; ++j) {
@@ -1366,7 +1536,7 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, const R
       int rescale = 0;
 #pragma unroll
       for (int hh = 0; hh < kHeads; ++hh) {
-        const float* ch_ = sc + hh * kTile;
+        const float* ch_ = sct + hh * kTile;
         const float m = keep[hh] ? c0[hh] + sg[hh] : 0.5f * (clo[hh] + ch_[hi - 1]);
         float u[4], r[4];
 #pragma unroll
@@ -1408,6 +1578,10 @@ __device__ void helper_loop(const CUtensorMap* tm_dt, const Problem& pb, const R
       lo = hi;
     }
     if (!ok) break;
+    if constexpr (from_scan) {  // the slot is used up: the scan warp may refill it
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars[kBarScanFree0 + sslot]);
+    }
     cur = nxt;
     have = have_next;
   }
@@ -1423,7 +1597,7 @@ template <int NS, int MODE>
 __global__ void __launch_bounds__(kThreads, 1)
     ssd_fused_tc_kernel(const __grid_constant__ CUtensorMap tm_x, const __grid_constant__ CUtensorMap tm_b,
                         const __grid_constant__ CUtensorMap tm_c, const __grid_constant__ CUtensorMap tm_y32,
-                        const __grid_constant__ CUtensorMap tm_dt, Problem pb) {
+                        const __grid_constant__ CUtensorMap tm_dt, const __grid_constant__ Problem pb) {
   using L = Layout<NS, MODE>;
   extern __shared__ uint8_t smem_raw[];
   __shared__ uint32_t s_tmem_base;
@@ -1466,6 +1640,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&bars[kBarDescFree0 + k], kComputeWarps + 1);
     }
     for (int k = 0; k < kHeads * 4; ++k) mbar_init(&bars[kBarPair0 + k], 1);
+    for (int k = 0; k < kScanSlots; ++k) {
+      mbar_init(&bars[kBarScanFull0 + k], 1);
+      mbar_init(&bars[kBarScanFree0 + k], 1);
+    }
     *abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     prefetch_tensormap(&tm_x);
@@ -1498,6 +1676,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     __syncwarp();
   } else if (warp == kHelperWarp) {
     helper_loop<NS, MODE>(&tm_dt, pb, rp, smem, bars, abort_flag);
+    __syncwarp();
+  } else if (warp == kScanWarp) {
+    if (MODE == kModeState) scan_loop<NS, MODE>(&tm_dt, pb, rp, smem, bars, abort_flag);
     __syncwarp();
   } else {
     compute_loop<NS, MODE>(&tm_y32, pb, smem, tmem, bars, abort_flag);
