@@ -492,18 +492,35 @@ int ssd_forward_host(const ssd_shape* s, const void* x, const float* dt, const f
   if (cu_seqlens && cudaStreamSynchronize(sin) != cudaSuccess) return fail(SSD_ERR_CUDA);  // pageable source
 
   auto at = [](void* base, size_t off) { return base ? (void*)((char*)base + off) : nullptr; };
-  for (int g = 0; g < ng && rc == SSD_OK; ++g) {
+  auto group_tokens = [&](int g, int64_t& t0, int64_t& nt) {
+    t0 = seq_start(gs[g]);
+    nt = (gs[g + 1] < nseq ? seq_start(gs[g + 1]) : tokens) - t0;
+  };
+  // Every group's inputs are queued on the input stream first, so the copies run back to
+  // back at the link's speed whatever the host takes to queue the groups' kernels.
+  for (int g = 0; g < ng; ++g) {
     const int64_t q0 = gs[g], q1 = gs[g + 1];
-    const int64_t t0 = seq_start(q0), t1 = q1 < nseq ? seq_start(q1) : tokens, nt = t1 - t0;
+    int64_t t0, nt;
+    group_tokens(g, t0, nt);
     const size_t p0 = (size_t)ptok[g];  // first token of the group in the device buffers
-    const char* hx = (const char*)x;
-    if (!h2d(at(dev[0], p0 * tok_x), hx + t0 * tok_x, nt * tok_x) ||
+    if (!h2d(at(dev[0], p0 * tok_x), (const char*)x + t0 * tok_x, nt * tok_x) ||
         !h2d(at(dev[1], p0 * tok_dt), (const char*)dt + t0 * tok_dt, nt * tok_dt) ||
         !h2d(at(dev[3], p0 * tok_bc), (const char*)B + t0 * tok_bc, nt * tok_bc) ||
         !h2d(at(dev[4], p0 * tok_bc), (const char*)C + t0 * tok_bc, nt * tok_bc) ||
         (init_state && !h2d(at(dev[6], seq_off[g]), (const char*)init_state + q0 * seq_state,
                             (q1 - q0) * seq_state)) ||
-        cudaEventRecord(ev[2 * g], sin) != cudaSuccess || cudaStreamWaitEvent(st, ev[2 * g], 0) != cudaSuccess) {
+        cudaEventRecord(ev[2 * g], sin) != cudaSuccess) {
+      rc = SSD_ERR_CUDA;
+      break;
+    }
+  }
+  // Then each group's compute once its inputs are in, and its outputs out once computed.
+  for (int g = 0; g < ng && rc == SSD_OK; ++g) {
+    const int64_t q0 = gs[g], q1 = gs[g + 1];
+    int64_t t0, nt;
+    group_tokens(g, t0, nt);
+    const size_t p0 = (size_t)ptok[g];
+    if (cudaStreamWaitEvent(st, ev[2 * g], 0) != cudaSuccess) {
       rc = SSD_ERR_CUDA;
       break;
     }
