@@ -296,12 +296,16 @@ uint64_t ssd_kernel_launch_count(void);
  * after `wait_limit_cycles` SM clock cycles (0 = the default, 2^32, about 2 s) it gives
  * up, the kernel drains its in-flight copies and tensor-core work, frees tensor memory
  * and returns, and ssd_query_status() reports SSD_ERR_DEVICE_TIMEOUT; the outputs of
- * that call are then undefined.  withhold_carry = 1 makes every CTA keep back the flag
- * that hands its state on to the next CTA (the state itself is still written), so the
- * CTAs that wait for it run out of time: the only way a test makes a wait fail.
- * Returns SSD_OK, or SSD_ERR_INVALID_ARG for a negative limit.
+ * that call are then undefined.  `withhold` is a bit mask of flags to keep back, the only
+ * way a test makes a wait fail:
+ *   bit 0 (1): every CTA keeps back the flag that hands its state on to the next CTA (the
+ *              state itself is still written), so the CTAs that wait for it run out of time;
+ *   bit 1 (2): CTA 0 keeps back its flag of the barrier after the work split's tile weights
+ *              (launches that weigh their tiles in the kernel), so every CTA's wait there
+ *              runs out of time and no CTA takes any work.
+ * Returns SSD_OK, or SSD_ERR_INVALID_ARG for a negative limit or other bits.
  */
-int ssd_set_test_hooks(int64_t wait_limit_cycles, int withhold_carry);
+int ssd_set_test_hooks(int64_t wait_limit_cycles, int withhold);
 
 #ifdef __cplusplus
 }

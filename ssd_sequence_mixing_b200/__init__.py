@@ -503,11 +503,13 @@ def kernel_launch_count() -> int:
     return int(_lib.ssd_kernel_launch_count())
 
 
-def set_test_hooks(wait_limit_cycles: int = 0, withhold_carry: bool = False) -> None:
+def set_test_hooks(wait_limit_cycles: int = 0, withhold_carry: bool = False, withhold_split: bool = False) -> None:
     """Test hooks of the tensor-core kernel's failure path: the cycle limit of every
-    device-side wait (0 = the default, about 2 s) and whether CTAs withhold the flag that
-    hands their state on (so that the CTAs waiting for it time out).  Defaults restore
-    normal operation."""
-    rc = _lib.ssd_set_test_hooks(int(wait_limit_cycles), 1 if withhold_carry else 0)
+    device-side wait (0 = the default, about 2 s), whether CTAs withhold the flag that
+    hands their state on (so that the CTAs waiting for it time out) and whether CTA 0
+    withholds its flag of the barrier after the work split's tile weights (so that every
+    CTA's wait there times out).  Defaults restore normal operation."""
+    bits = (1 if withhold_carry else 0) | (2 if withhold_split else 0)
+    rc = _lib.ssd_set_test_hooks(int(wait_limit_cycles), bits)
     if rc:
         raise SsdError(rc, "ssd_set_test_hooks")

@@ -603,10 +603,10 @@ int ssd_profile_dominant(ssd_event_t start, ssd_event_t stop) {
 
 uint64_t ssd_kernel_launch_count(void) { return g_launches.load(); }
 
-int ssd_set_test_hooks(int64_t wait_limit_cycles, int withhold_carry) {
-  if (wait_limit_cycles < 0) return SSD_ERR_INVALID_ARG;
+int ssd_set_test_hooks(int64_t wait_limit_cycles, int withhold) {
+  if (wait_limit_cycles < 0 || (withhold & ~3)) return SSD_ERR_INVALID_ARG;
   g_wait_limit.store(wait_limit_cycles ? (long long)wait_limit_cycles : kDefaultWaitLimit);
-  g_withhold_carry.store(withhold_carry ? 1 : 0);
+  g_withhold_carry.store(withhold);
   return SSD_OK;
 }
 

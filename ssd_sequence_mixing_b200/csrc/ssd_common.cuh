@@ -54,7 +54,8 @@ struct Problem {
   int weights_ready;     // tile_w already holds this problem's weights (no barrier)
   int ranges;            // CTAs of the tensor-core launch
   long long wait_limit;  // SM cycles a device-side wait may take before it gives up
-  int withhold_carry;    // test hook: CTAs never publish the state they hand on
+  int withhold_carry;    // test hook, bits: 1 CTAs never publish the state they hand on,
+                         // 2 CTA 0 never publishes its flag of the split's weight barrier
   // tensor-core launches on a column range of a wider state: this launch's state columns
   // are [n_off, n_off + N) of rows n_stride long, and y_accum adds its y to the y in memory
   int n_off, n_stride, y_accum;

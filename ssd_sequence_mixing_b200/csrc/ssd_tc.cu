@@ -1,9 +1,10 @@
 // ssd_tc.cu -- the tensor-core path: one fused sm_100a kernel for the whole chunked
 // SSD forward pass ("Transformers are SSMs", wikillm.com card, Method step 5, sec. 6).
 //
-// One persistent CTA per SM walks an equal share of the flat list of 128-token tiles
-// (the tcgen05 M) of all units (sequence, pair of heads sharing a B/C group), handing
-// the state on through global memory where its share starts or ends inside a unit.
+// One persistent CTA per SM walks a share of the flat list of 128-token tiles (the
+// tcgen05 M) of all units (sequence, pair of heads sharing a B/C group), cut at equal
+// shares of a per-tile weight, handing the state on through global memory where its
+// share starts or ends inside a unit.
 // The P x N state of each head never leaves the chip: it stays in fp32 in tensor
 // memory, with a bf16 copy in shared memory as an MMA operand.
 //
@@ -37,12 +38,14 @@
 // each over a run of rows whose range fits (on the pages' input distributions,
 // 1 - 3 % of tiles).
 //
-// Roles: 16 compute warps (Û, the mask, the state step, the epilogue), one MMA warp
-// (every tcgen05.mma), one load warp (every TMA load of x, B, C) and one helper warp
-// (dt loads, the per-pass descriptors: passes, references, row factors, flags).
+// Roles: 16 compute warps (U, the mask, the state step, the epilogue), one MMA warp
+// (every tcgen05.mma), one load warp (every TMA load of x, B, C), one helper warp (dt
+// loads, the per-pass descriptors: passes, references, row factors, flags) and, with
+// final states only, a scan warp that takes the helper's dt loads and cumsums.
 // Tensor memory: two S/P buffers of 128 columns (P is written in place over S),
 // Y 128, H 128.  Shared memory: x (two stages; U and then y are written in place),
-// a ring of three B/C tiles, the bf16 state, the descriptors and the dt stages.
+// a ring of three B/C tiles, the bf16 state, the descriptors, the cumsums and the dt
+// stages; with final states only, two U buffers in place of C and the state copy.
 // Every wait is bounded; a wait that gives up records SSD_ERR_DEVICE_TIMEOUT in the
 // status word, drains what is in flight (bounded), frees tensor memory and exits.
 #include <cuda.h>
@@ -193,11 +196,12 @@ static_assert(kDynSmem<128, kModeFull> <= 227 * 1024 && kDynSmem<128, kModeState
 
 // Work split.  The tiles of all units (sequence, head pair), unit by unit and each
 // unit's 128-token tiles in order, form one flat list; CTA r takes the contiguous
-// range [W r / R, W (r + 1) / R).  A range may start inside a unit (it then needs the
-// state the previous CTA reached there: "carry in") and end inside one (it then hands
-// its state on: "carry out").  A CTA processes its last, truncated piece first, so the
-// state it hands on is ready early; then the whole units; then the piece that needs a
-// carry.  The load, helper and compute roles walk the same sequence.
+// range that holds share r of R of the tiles' weights (below).  A range may start
+// inside a unit (it then needs the state the previous CTA reached there: "carry in")
+// and end inside one (it then hands its state on: "carry out").  A CTA processes its
+// last, truncated piece first, so the state it hands on is ready early; then the whole
+// units; then the piece that needs a carry.  The load, helper and compute roles walk
+// the same sequence.
 struct TileCursor {
   int unit, k0, len;  // k0: token offset of the tile in the sequence
   int tb;             // first token of the sequence (tokens < 2^31 on this path)
@@ -609,7 +613,7 @@ __global__ void __launch_bounds__(kWeightThreads) tile_weight_kernel(const __gri
 // is the same for all threads of the CTA; false if a wait gave up.
 __device__ __noinline__ bool weights_barrier(const Problem& pb, volatile int* abort_flag) {
   __syncthreads();  // this CTA's weight bytes are written
-  if (threadIdx.x == 0) {
+  if (threadIdx.x == 0 && !(blockIdx.x == 0 && (pb.withhold_carry & 2))) {
     __threadfence();
     st_release_gpu_u64(&pb.split_flag[blockIdx.x], pb.epoch);
   }
@@ -919,7 +923,7 @@ __device__ __noinline__ void put_state(const Problem& pb, const PassDesc& d, int
   if (!to_final) {
     __threadfence();
     __syncwarp();
-    if ((threadIdx.x & 31) == 0 && !pb.withhold_carry)
+    if ((threadIdx.x & 31) == 0 && !(pb.withhold_carry & 1))
       st_release_gpu_u64(&pb.carry_flag[blockIdx.x * kComputeWarps + wid], pb.epoch);
     __syncwarp();
   }
@@ -1778,7 +1782,7 @@ cudaError_t launch_mode(const Problem& pb, cudaStream_t st) {
     if (getenv("SSD_DEBUG")) fprintf(stderr, "ssd: smem attribute failed: %s\n", cudaGetErrorString(e));
     return e;
   }
-  // One CTA per SM (at most), each on an equal share of the flat tile list; a flat tile
+  // One CTA per SM (at most), each on a weighted share of the flat tile list; a flat tile
   // count is not known on the host for packed batches, so the grid covers every SM and
   // ranges may be empty when there are fewer tiles than SMs.
   const int grid = pb.ranges;
