@@ -118,6 +118,21 @@ def test_dense_many_tiles_per_cta(case):
     check(prob, y, fin)
 
 
+@pytest.mark.parametrize("batch", [18, 19], ids=["in_kernel", "weight_kernel"])
+def test_split_weights_either_side_of_the_threshold(batch):
+    """The work split's tile weights come from the fused kernel's own CTAs (one flag barrier)
+    while there are at most two sequence tiles per SM, and from a kernel of their own beyond
+    that: batch 18 x 16 tiles (288) and 19 x 16 (304) fall either side of 2 x 148."""
+    if torch.cuda.get_device_properties(0).multi_processor_count != 148:
+        pytest.skip("the threshold is set for 148 SMs")
+    wl = workloads.custom(batch, 2048, H=64, P=64, N=128, G=1, chunk=256, dtype="bf16", init=True)
+    prob = workloads.generate(wl, seed=23)
+    dev = to_device(prob)
+    assert ssd.select_path(ssd.make_shape(dev["x"], dev["B"], dev["cu_seqlens"]), wl.chunk) == ssd.PATH_TC
+    y, fin = run(prob, dev=dev)
+    check(prob, y, fin, pairs=sample_pairs(prob, k=8))
+
+
 def test_packed_passes_and_hand_ons():
     """Heads that decay too fast for one pass per tile (A = -1e4 and -60), in packed
     sequences long enough to be cut across CTAs."""
